@@ -1,0 +1,126 @@
+"""MoE expert-parallel dispatch / combine over virtual ranks.
+
+Test infrastructure only (see ``oracle/__init__.py``).
+
+Follows the vLLM collectives tutorial (gsyq.cn/news/307221), section 8.4
+("MoE Dispatch / Combine"): with experts split evenly over the EP ranks
+(rank 0 holds experts 0,1 and rank 1 holds 2,3 in its example), dispatch sends
+every token to the rank that holds each expert it was routed to; combine sends
+the expert outputs back by original token ownership.  Section 8.2 says the
+per-peer lengths then differ, i.e. an all-to-all-v.
+
+Readings taken (the pages are silent on these):
+
+* Expert e lives on rank e // (E / N).
+* One dispatched row per (token, chosen expert) pair; a token routed to two
+  experts on the same rank is sent twice (no per-rank de-duplication).
+* Send order on source s: by destination rank, then expert id ascending, then
+  token index ascending (destination-major equals expert-major because
+  experts are assigned to ranks in contiguous blocks).  Receive order on
+  destination d: by source rank ascending (tutorial 8.1, "[from 0, from 1,
+  ...]"), then the sender's order.
+* A token's K expert ids are distinct and lie in [0, E).
+* The expert between dispatch and combine is the identity (expert compute is
+  out of scope); tests may scale rows per expert to catch mix-ups.
+* combine: ``acc = fl32(w_0 * y_0)``, then ``acc = fl32(acc + fl32(w_k * y_k))``
+  for k = 1 .. K-1 (k ascending, products and sums each rounded to binary32,
+  no fused multiply-add), then one rounding to the storage type.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .numerics import narrow, widen
+
+
+def moe_route(topk_ids, n_experts: int):
+    """Split matrix and row positions of every (token, k) pair.
+
+    Returns (send_counts[N,N], send_displs[N,N], recv_displs[N,N] (indexed
+    [d][s]), pos: list of int64 [T*K] arrays -- the row of pair (t, k) in the
+    receive buffer of rank topk_ids[t,k] // (E/N)).
+    """
+    n = len(topk_ids)
+    assert n_experts % n == 0
+    epr = n_experts // n
+    send_counts = np.zeros((n, n), dtype=np.int64)
+    for s in range(n):
+        ids = np.asarray(topk_ids[s]).reshape(-1)
+        assert ids.size == 0 or (ids.min() >= 0 and ids.max() < n_experts)
+        cnt = np.bincount(ids, minlength=n_experts)
+        for d in range(n):
+            send_counts[s, d] = cnt[d * epr:(d + 1) * epr].sum()
+    send_displs = np.zeros((n, n), dtype=np.int64)
+    for s in range(n):
+        for d in range(1, n):
+            send_displs[s, d] = send_displs[s, d - 1] + send_counts[s, d - 1]
+    recv_displs = np.zeros((n, n), dtype=np.int64)  # [d][s]
+    for d in range(n):
+        for s in range(1, n):
+            recv_displs[d, s] = recv_displs[d, s - 1] + send_counts[s - 1, d]
+    pos = []
+    for s in range(n):
+        ids2 = np.asarray(topk_ids[s])
+        t_, k_ = ids2.shape
+        for t in range(t_):
+            assert len(set(ids2[t].tolist())) == k_, "a token's experts must be distinct"
+        e = ids2.reshape(-1).astype(np.int64)
+        tok = np.repeat(np.arange(t_, dtype=np.int64), k_)
+        order = np.lexsort((tok, e))  # primary key: expert, then token
+        send_pos = np.empty(e.size, dtype=np.int64)
+        send_pos[order] = np.arange(e.size, dtype=np.int64)
+        d = e // epr
+        pos.append(recv_displs[d, s] + send_pos - send_displs[s, d])
+    return send_counts, send_displs, recv_displs, pos
+
+
+def moe_permute_send(xs, topk_ids, n_experts: int, hidden: int):
+    """The sender-side layout: rank s's rows in send order (dest, expert, token)."""
+    out = []
+    for s in range(len(xs)):
+        ids2 = np.asarray(topk_ids[s])
+        t_, k_ = ids2.shape
+        e = ids2.reshape(-1)
+        tok = np.repeat(np.arange(t_), k_)
+        order = np.lexsort((tok, e))
+        x = np.asarray(xs[s]).reshape(t_, hidden)
+        out.append(x[tok[order]].reshape(-1))
+    return out
+
+
+def moe_dispatch(xs, topk_ids, pos, recv_bufs, n_experts: int, hidden: int):
+    """recv[d][pos(s,t,k)] = x[s][t] for every source s, token t and choice k."""
+    n = len(xs)
+    epr = n_experts // n
+    outs = [np.array(b, copy=True) for b in recv_bufs]
+    for s in range(n):
+        ids2 = np.asarray(topk_ids[s])
+        t_, k_ = ids2.shape
+        x = np.asarray(xs[s]).reshape(t_, hidden)
+        for j in range(t_ * k_):
+            t, d = j // k_, int(ids2.reshape(-1)[j]) // epr
+            p = int(pos[s][j])
+            outs[d][p * hidden:(p + 1) * hidden] = x[t]
+    return outs
+
+
+def moe_combine(ys, topk_ids, pos, topk_w, n_experts: int, hidden: int, dtype: str):
+    """out[s][t] = round( sum_k w[s][t][k] * y[d_k][pos(s,t,k)] ), k ascending."""
+    n = len(topk_ids)
+    epr = n_experts // n
+    outs = []
+    for s in range(n):
+        ids2 = np.asarray(topk_ids[s])
+        w = np.asarray(topk_w[s], dtype=np.float32)
+        t_, k_ = ids2.shape
+        acc = np.zeros((t_, hidden), dtype=np.float32)
+        for k in range(k_):
+            rows = np.empty((t_, hidden), dtype=np.float32)
+            for t in range(t_):
+                d = int(ids2[t, k]) // epr
+                p = int(pos[s][t * k_ + k])
+                rows[t] = widen(np.asarray(ys[d])[p * hidden:(p + 1) * hidden], dtype)
+            prod = (w[:, k:k + 1] * rows).astype(np.float32)
+            acc = prod if k == 0 else (acc + prod).astype(np.float32)
+        outs.append(narrow(acc.reshape(-1), dtype))
+    return outs
