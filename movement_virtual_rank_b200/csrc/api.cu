@@ -1,0 +1,646 @@
+// The extern "C" entry points of include/coll.h: argument validation, the
+// overlap rules, the N == 1 and count == 0 shortcuts, and the choice of
+// kernel.  No entry point allocates memory or synchronises the stream.
+#include <algorithm>
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "coll.h"
+#include "internal.h"
+
+namespace mvr {
+
+// per-dtype launchers defined in reduce_<dtype>.cu
+int launch_reduce_bf16(const ReduceArgs&, coll_op_t, int, bool, int, cudaStream_t);
+int launch_reduce_fp16(const ReduceArgs&, coll_op_t, int, bool, int, cudaStream_t);
+int launch_reduce_fp32(const ReduceArgs&, coll_op_t, int, bool, int, cudaStream_t);
+int launch_reduce_int32(const ReduceArgs&, coll_op_t, int, bool, int, cudaStream_t);
+int launch_ring_bf16(const RingStepArgs&, coll_op_t, bool, cudaStream_t);
+int launch_ring_fp16(const RingStepArgs&, coll_op_t, bool, cudaStream_t);
+int launch_ring_fp32(const RingStepArgs&, coll_op_t, bool, cudaStream_t);
+int launch_ring_int32(const RingStepArgs&, coll_op_t, bool, cudaStream_t);
+
+enum { kAll = 0, kBlock = 1, kSame = 2, kOneShot = 3 };  // mirrors ReduceMode
+
+static thread_local char g_cuda_msg[256];
+
+int launch_status(cudaError_t e) {
+  if (e == cudaSuccess) return COLL_OK;
+  std::snprintf(g_cuda_msg, sizeof(g_cuda_msg), "CUDA error %d: %s", static_cast<int>(e), cudaGetErrorString(e));
+  return COLL_ERR_CUDA;
+}
+
+int num_sms() {
+  static std::atomic<int> cache[COLL_MAX_RANKS];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= COLL_MAX_RANKS) return 148;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+  cache[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+
+int elem_size(coll_dtype_t dt) {
+  switch (dt) {
+    case COLL_BF16:
+    case COLL_FP16: return 2;
+    case COLL_FP32:
+    case COLL_INT32: return 4;
+  }
+  return 0;
+}
+
+int launch_reduce(const ReduceArgs& a, coll_dtype_t dt, coll_op_t op, int mode, bool vec, int bps, cudaStream_t s) {
+  switch (dt) {
+    case COLL_BF16: return launch_reduce_bf16(a, op, mode, vec, bps, s);
+    case COLL_FP16: return launch_reduce_fp16(a, op, mode, vec, bps, s);
+    case COLL_FP32: return launch_reduce_fp32(a, op, mode, vec, bps, s);
+    case COLL_INT32: return launch_reduce_int32(a, op, mode, vec, bps, s);
+  }
+  return COLL_ERR_UNSUPPORTED;
+}
+
+int launch_ring_rs_step(const RingStepArgs& a, coll_dtype_t dt, coll_op_t op, bool vec, cudaStream_t s) {
+  switch (dt) {
+    case COLL_BF16: return launch_ring_bf16(a, op, vec, s);
+    case COLL_FP16: return launch_ring_fp16(a, op, vec, s);
+    case COLL_FP32: return launch_ring_fp32(a, op, vec, s);
+    case COLL_INT32: return launch_ring_int32(a, op, vec, s);
+  }
+  return COLL_ERR_UNSUPPORTED;
+}
+
+}  // namespace mvr
+
+using namespace mvr;
+
+namespace {
+
+inline cudaStream_t S(coll_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+inline uintptr_t U(const void* p) { return reinterpret_cast<uintptr_t>(p); }
+inline bool al16(const void* p) { return (U(p) & 15) == 0; }
+
+// [a, a+an) and [b, b+bn) share a byte
+inline bool overlap(const void* a, size_t an, const void* b, size_t bn) {
+  if (an == 0 || bn == 0) return false;
+  return U(a) < U(b) + bn && U(b) < U(a) + an;
+}
+
+inline bool valid_n(int n) { return n >= 1 && n <= COLL_MAX_RANKS; }
+inline bool valid_op(coll_op_t op) { return op >= COLL_SUM && op <= COLL_PROD; }
+
+template <typename P>
+bool all_nonnull(P const* p, int n) {
+  if (p == nullptr) return false;
+  for (int i = 0; i < n; ++i)
+    if (p[i] == nullptr) return false;
+  return true;
+}
+
+// outputs pairwise disjoint
+bool outputs_disjoint(void* const* out, int n, size_t bytes) {
+  for (int i = 0; i < n; ++i)
+    for (int j = i + 1; j < n; ++j)
+      if (overlap(out[i], bytes, out[j], bytes)) return false;
+  return true;
+}
+
+size_t seg_elems(size_t count, int n, int es) {
+  const size_t g = 16 / es;
+  const size_t per = (count + n - 1) / n;
+  return (per + g - 1) / g * g;
+}
+
+int blocks_per_slice(uint64_t slice_units, int nslices) {
+  uint64_t want = (slice_units + kBlockThreads - 1) / kBlockThreads;
+  const uint64_t cap = std::max<uint64_t>(1, static_cast<uint64_t>(num_sms()) * 8 / nslices);
+  want = std::min(want, cap);
+  return static_cast<int>(std::max<uint64_t>(want, 1));
+}
+
+int copy_one(const void* src, void* dst, size_t bytes, cudaStream_t s) {
+  if (src == dst || bytes == 0) return COLL_OK;
+  CopyJob j{static_cast<const char*>(src), static_cast<char*>(dst), bytes};
+  return launch_copy_jobs(&j, 1, s);
+}
+
+size_t ring_ws(size_t count) { return (count * 4 + 255) / 256 * 256; }
+
+}  // namespace
+
+extern "C" {
+
+int coll_version(void) { return 10000; }
+
+const char* coll_strerror(int status) {
+  switch (status) {
+    case COLL_OK: return "ok";
+    case COLL_ERR_INVALID_ARG: return "invalid argument";
+    case COLL_ERR_UNSUPPORTED: return "unsupported dtype / op / algorithm";
+    case COLL_ERR_ALIAS: return "buffers overlap in a way this collective does not allow";
+    case COLL_ERR_CUDA: return g_cuda_msg[0] ? g_cuda_msg : "CUDA error";
+    case COLL_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+  }
+  return "unknown status";
+}
+
+// ------------------------------------------------------------- Broadcast ----
+int coll_broadcast(void* const* bufs, int nranks, size_t count, coll_dtype_t dtype, int src, coll_stream_t stream) {
+  const int es = elem_size(dtype);
+  if (!es) return COLL_ERR_UNSUPPORTED;
+  if (!valid_n(nranks) || src < 0 || src >= nranks || !all_nonnull(bufs, nranks)) return COLL_ERR_INVALID_ARG;
+  const size_t bytes = count * es;
+  if (bytes == 0 || nranks == 1) return COLL_OK;
+  if (!outputs_disjoint(bufs, nranks, bytes)) return COLL_ERR_ALIAS;
+  FanoutArgs a{};
+  a.src[0] = static_cast<const char*>(bufs[src]);
+  a.ns = 1;
+  for (int q = 0; q < nranks; ++q)
+    if (q != src) a.dst[a.nd++] = static_cast<char*>(bufs[q]);
+  a.bytes = bytes;
+  a.dst_stride = 0;
+  return launch_fanout(a, S(stream));
+}
+
+// ---------------------------------------------------------------- Gather ----
+int coll_gather(const void* const* send, void* recv_dst, int nranks, size_t rows, size_t cols_per_rank,
+                coll_dtype_t dtype, int dst, coll_stream_t stream) {
+  const int es = elem_size(dtype);
+  if (!es) return COLL_ERR_UNSUPPORTED;
+  if (!valid_n(nranks) || dst < 0 || dst >= nranks || !all_nonnull(send, nranks) || recv_dst == nullptr || rows == 0)
+    return COLL_ERR_INVALID_ARG;
+  const size_t blk = rows * cols_per_rank * es;  // one rank's block
+  if (blk == 0) return COLL_OK;
+  const size_t total = blk * nranks;
+  char* out = static_cast<char*>(recv_dst);
+  for (int r = 0; r < nranks; ++r) {
+    if (!overlap(send[r], blk, out, total)) continue;
+    const bool in_place = rows == 1 && r == dst && send[r] == out + static_cast<size_t>(r) * blk;
+    if (!in_place) return COLL_ERR_ALIAS;
+  }
+  if (rows == 1) {
+    std::vector<CopyJob> jobs;
+    for (int r = 0; r < nranks; ++r) {
+      char* d = out + static_cast<size_t>(r) * blk;
+      if (send[r] != d) jobs.push_back({static_cast<const char*>(send[r]), d, blk});
+    }
+    return launch_copy_jobs(jobs.data(), static_cast<int>(jobs.size()), S(stream));
+  }
+  GatherRowsArgs a{};
+  for (int r = 0; r < nranks; ++r) a.src[r] = static_cast<const char*>(send[r]);
+  a.dst = out;
+  a.rows = rows;
+  a.row_bytes = cols_per_rank * es;
+  a.dst_pitch = a.row_bytes * nranks;
+  a.n = nranks;
+  return launch_gather_rows(a, S(stream));
+}
+
+// ---------------------------------------------------------------- Reduce ----
+int coll_reduce(const void* const* send, void* recv_dst, int nranks, size_t count, coll_dtype_t dtype, coll_op_t op,
+                int dst, coll_stream_t stream) {
+  const int es = elem_size(dtype);
+  if (!es) return COLL_ERR_UNSUPPORTED;
+  if (!valid_op(op)) return COLL_ERR_UNSUPPORTED;
+  if (!valid_n(nranks) || dst < 0 || dst >= nranks || !all_nonnull(send, nranks) || recv_dst == nullptr)
+    return COLL_ERR_INVALID_ARG;
+  const size_t bytes = count * es;
+  if (bytes == 0) return COLL_OK;
+  for (int r = 0; r < nranks; ++r)
+    if (overlap(send[r], bytes, recv_dst, bytes) && !(r == dst && send[r] == recv_dst)) return COLL_ERR_ALIAS;
+  if (nranks == 1) return copy_one(send[0], recv_dst, bytes, S(stream));
+  ReduceArgs a{};
+  bool vec = al16(recv_dst);
+  for (int r = 0; r < nranks; ++r) {
+    a.in[r] = static_cast<const char*>(send[r]);
+    vec = vec && al16(send[r]);
+  }
+  a.out[0] = static_cast<char*>(recv_dst);
+  a.count = count;
+  a.seg = count;
+  a.nin = nranks;
+  a.nout = 1;
+  a.nslices = 1;
+  const int bps = blocks_per_slice(vec ? count * es / 16 : count, 1);
+  return launch_reduce(a, dtype, op, kSame, vec, bps, S(stream));
+}
+
+// --------------------------------------------------------------- Scatter ----
+int coll_scatter(const void* send_src, void* const* recv, int nranks, size_t count_per_rank, coll_dtype_t dtype,
+                 int src, coll_stream_t stream) {
+  const int es = elem_size(dtype);
+  if (!es) return COLL_ERR_UNSUPPORTED;
+  if (!valid_n(nranks) || src < 0 || src >= nranks || send_src == nullptr || !all_nonnull(recv, nranks))
+    return COLL_ERR_INVALID_ARG;
+  const size_t blk = count_per_rank * es;
+  if (blk == 0) return COLL_OK;
+  const char* in = static_cast<const char*>(send_src);
+  if (!outputs_disjoint(recv, nranks, blk)) return COLL_ERR_ALIAS;
+  std::vector<CopyJob> jobs;
+  for (int r = 0; r < nranks; ++r) {
+    const char* sp = in + static_cast<size_t>(r) * blk;
+    if (overlap(recv[r], blk, in, blk * nranks)) {
+      if (!(r == src && recv[r] == sp)) return COLL_ERR_ALIAS;
+      continue;  // already in place
+    }
+    jobs.push_back({sp, static_cast<char*>(recv[r]), blk});
+  }
+  return launch_copy_jobs(jobs.data(), static_cast<int>(jobs.size()), S(stream));
+}
+
+// --------------------------------------------------------- ReduceScatter ----
+int coll_reduce_scatter(const void* const* send, void* const* recv, int nranks, size_t recv_count,
+                        coll_dtype_t dtype, coll_op_t op, coll_stream_t stream) {
+  const int es = elem_size(dtype);
+  if (!es) return COLL_ERR_UNSUPPORTED;
+  if (!valid_op(op)) return COLL_ERR_UNSUPPORTED;
+  if (!valid_n(nranks) || !all_nonnull(send, nranks) || !all_nonnull(recv, nranks)) return COLL_ERR_INVALID_ARG;
+  const size_t blk = recv_count * es;
+  if (blk == 0) return COLL_OK;
+  const size_t in_bytes = blk * nranks;
+  if (!outputs_disjoint(recv, nranks, blk)) return COLL_ERR_ALIAS;
+  for (int q = 0; q < nranks; ++q)
+    for (int r = 0; r < nranks; ++r)
+      if (overlap(recv[q], blk, send[r], in_bytes) &&
+          !(q == r && recv[q] == static_cast<const char*>(send[r]) + static_cast<size_t>(q) * blk))
+        return COLL_ERR_ALIAS;
+  if (nranks == 1) return copy_one(send[0], recv[0], blk, S(stream));
+  ReduceArgs a{};
+  bool vec = (blk % 16) == 0;
+  for (int r = 0; r < nranks; ++r) {
+    a.in[r] = static_cast<const char*>(send[r]);
+    a.out[r] = static_cast<char*>(recv[r]);
+    vec = vec && al16(send[r]) && al16(recv[r]);
+  }
+  a.count = recv_count * nranks;
+  a.seg = recv_count;
+  a.nin = nranks;
+  a.nout = 1;
+  a.nslices = nranks;
+  const int bps = blocks_per_slice(vec ? blk / 16 : recv_count, nranks);
+  return launch_reduce(a, dtype, op, kBlock, vec, bps, S(stream));
+}
+
+// ------------------------------------------------------------- AllReduce ----
+size_t coll_all_reduce_workspace_size(int nranks, size_t count, coll_dtype_t dtype, coll_algo_t algo) {
+  if (algo != COLL_ALGO_RING || !valid_n(nranks) || !elem_size(dtype)) return 0;
+  return ring_ws(count);
+}
+
+int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size_t count, coll_dtype_t dtype,
+                    coll_op_t op, coll_algo_t algo, void* workspace, size_t workspace_bytes, coll_stream_t stream) {
+  const int es = elem_size(dtype);
+  if (!es) return COLL_ERR_UNSUPPORTED;
+  if (!valid_op(op) || algo < COLL_ALGO_AUTO || algo > COLL_ALGO_RING) return COLL_ERR_UNSUPPORTED;
+  if (!valid_n(nranks) || !all_nonnull(send, nranks) || !all_nonnull(recv, nranks)) return COLL_ERR_INVALID_ARG;
+  const size_t bytes = count * es;
+  if (bytes == 0) return COLL_OK;
+  if (algo == COLL_ALGO_AUTO) algo = COLL_ALGO_TWOSHOT;
+  if (!outputs_disjoint(recv, nranks, bytes)) return COLL_ERR_ALIAS;
+  for (int q = 0; q < nranks; ++q)
+    for (int r = 0; r < nranks; ++r)
+      if (overlap(recv[q], bytes, send[r], bytes) && !(q == r && recv[q] == send[r] && algo != COLL_ALGO_ONESHOT))
+        return COLL_ERR_ALIAS;
+  if (algo == COLL_ALGO_RING && nranks > 1) {
+    if (workspace == nullptr || workspace_bytes < ring_ws(count) || !al16(workspace)) return COLL_ERR_WORKSPACE;
+    if (overlap(workspace, ring_ws(count), recv[0], bytes)) {
+      // the partials must not live inside any rank's buffer
+      return COLL_ERR_ALIAS;
+    }
+    for (int r = 0; r < nranks; ++r)
+      if (overlap(workspace, ring_ws(count), send[r], bytes) || overlap(workspace, ring_ws(count), recv[r], bytes))
+        return COLL_ERR_ALIAS;
+  }
+  if (nranks == 1) return copy_one(send[0], recv[0], bytes, S(stream));
+  bool vec = true;
+  for (int r = 0; r < nranks; ++r) vec = vec && al16(send[r]) && al16(recv[r]);
+  const size_t seg = seg_elems(count, nranks, es);
+  if (algo == COLL_ALGO_RING) {
+    RingStepArgs a{};
+    for (int r = 0; r < nranks; ++r) {
+      a.in[r] = static_cast<const char*>(send[r]);
+      a.out[r] = static_cast<char*>(recv[r]);
+    }
+    a.partial = static_cast<char*>(workspace);
+    a.count = count;
+    a.seg = seg;
+    a.n = nranks;
+    for (int k = 1; k < nranks; ++k) {  // reduce-scatter phase
+      a.k = k;
+      const int st = launch_ring_rs_step(a, dtype, op, vec, S(stream));
+      if (st != COLL_OK) return st;
+    }
+    std::vector<CopyJob> jobs(nranks);
+    for (int j = 1; j < nranks; ++j) {  // all-gather phase: rank c+j copies chunk c from rank c+j-1
+      int nj = 0;
+      for (int c = 0; c < nranks; ++c) {
+        const size_t lo = std::min(count, c * seg), hi = std::min(count, lo + seg);
+        jobs[nj++] = {static_cast<const char*>(recv[(c + j - 1) % nranks]) + lo * es,
+                      static_cast<char*>(recv[(c + j) % nranks]) + lo * es, (hi - lo) * es};
+      }
+      const int st = launch_copy_jobs(jobs.data(), nj, S(stream));
+      if (st != COLL_OK) return st;
+    }
+    return COLL_OK;
+  }
+  ReduceArgs a{};
+  for (int r = 0; r < nranks; ++r) {
+    a.in[r] = static_cast<const char*>(send[r]);
+    a.out[r] = static_cast<char*>(recv[r]);
+  }
+  a.count = count;
+  a.nin = nranks;
+  a.nout = nranks;
+  a.nslices = nranks;
+  if (algo == COLL_ALGO_ONESHOT) {
+    a.seg = count;
+    const int bps = blocks_per_slice(vec ? bytes / 16 : count, nranks);
+    return launch_reduce(a, dtype, op, kOneShot, vec, bps, S(stream));
+  }
+  a.seg = seg;
+  const int bps = blocks_per_slice(vec ? seg * es / 16 : seg, nranks);
+  return launch_reduce(a, dtype, op, kAll, vec, bps, S(stream));
+}
+
+// ------------------------------------------------------------- AllGather ----
+int coll_all_gather(const void* const* send, void* const* recv, int nranks, size_t send_count, coll_dtype_t dtype,
+                    coll_stream_t stream) {
+  const int es = elem_size(dtype);
+  if (!es) return COLL_ERR_UNSUPPORTED;
+  if (!valid_n(nranks) || !all_nonnull(send, nranks) || !all_nonnull(recv, nranks)) return COLL_ERR_INVALID_ARG;
+  const size_t blk = send_count * es;
+  if (blk == 0) return COLL_OK;
+  const size_t total = blk * nranks;
+  if (!outputs_disjoint(recv, nranks, total)) return COLL_ERR_ALIAS;
+  bool all_in_place = true;
+  for (int r = 0; r < nranks; ++r) {
+    const bool in_place = send[r] == static_cast<char*>(recv[r]) + static_cast<size_t>(r) * blk;
+    all_in_place = all_in_place && in_place;
+    for (int q = 0; q < nranks; ++q)
+      if (overlap(send[r], blk, recv[q], total) && !(q == r && in_place)) return COLL_ERR_ALIAS;
+  }
+  FanoutArgs a{};
+  for (int r = 0; r < nranks; ++r) {
+    a.src[r] = static_cast<const char*>(send[r]);
+    a.dst[r] = static_cast<char*>(recv[r]);
+  }
+  a.ns = nranks;
+  a.nd = nranks;
+  a.bytes = blk;
+  a.dst_stride = blk;
+  a.skip_diag = all_in_place ? 1 : 0;  // a partly in-place call copies those blocks onto themselves
+  return launch_fanout(a, S(stream));
+}
+
+// ------------------------------------------------------------ All-to-All ----
+int coll_all_to_all(const void* const* send, void* const* recv, int nranks, size_t count, coll_dtype_t dtype,
+                    coll_stream_t stream) {
+  const int es = elem_size(dtype);
+  if (!es) return COLL_ERR_UNSUPPORTED;
+  if (!valid_n(nranks) || !all_nonnull(send, nranks) || !all_nonnull(recv, nranks)) return COLL_ERR_INVALID_ARG;
+  const size_t blk = count * es;
+  if (blk == 0) return COLL_OK;
+  const size_t total = blk * nranks;
+  if (!outputs_disjoint(recv, nranks, total)) return COLL_ERR_ALIAS;
+  for (int d = 0; d < nranks; ++d)
+    for (int s = 0; s < nranks; ++s)
+      if (overlap(recv[d], total, send[s], total)) return COLL_ERR_ALIAS;
+  std::vector<CopyJob> jobs;
+  jobs.reserve(static_cast<size_t>(nranks) * nranks);
+  for (int s = 0; s < nranks; ++s)
+    for (int d = 0; d < nranks; ++d)
+      jobs.push_back({static_cast<const char*>(send[s]) + static_cast<size_t>(d) * blk,
+                      static_cast<char*>(recv[d]) + static_cast<size_t>(s) * blk, blk});
+  return launch_copy_jobs(jobs.data(), static_cast<int>(jobs.size()), S(stream));
+}
+
+int coll_all_to_all_v(const void* const* send, void* const* recv, int nranks, const int64_t* send_counts,
+                      const int64_t* send_displs, const int64_t* recv_displs, const int64_t* send_capacity,
+                      const int64_t* recv_capacity, size_t row_elems, coll_dtype_t dtype, coll_stream_t stream) {
+  const int es = elem_size(dtype);
+  if (!es) return COLL_ERR_UNSUPPORTED;
+  if (!valid_n(nranks) || !all_nonnull(send, nranks) || !all_nonnull(recv, nranks) || !send_counts ||
+      !send_displs || !recv_displs)
+    return COLL_ERR_INVALID_ARG;
+  const size_t row = row_elems * es;
+  if (row == 0) return COLL_OK;
+  const int n = nranks;
+  std::vector<int64_t> recv_end(n, 0), send_end(n, 0);
+  for (int s = 0; s < n; ++s)
+    for (int d = 0; d < n; ++d) {
+      const int64_t c = send_counts[s * n + d], so = send_displs[s * n + d], ro = recv_displs[d * n + s];
+      if (c < 0 || so < 0 || ro < 0) return COLL_ERR_INVALID_ARG;
+      if (c == 0) continue;
+      send_end[s] = std::max(send_end[s], so + c);
+      recv_end[d] = std::max(recv_end[d], ro + c);
+      if (send_capacity && so + c > send_capacity[s]) return COLL_ERR_INVALID_ARG;
+      if (recv_capacity && ro + c > recv_capacity[d]) return COLL_ERR_INVALID_ARG;
+    }
+  // receive blocks of one destination must not overlap each other
+  for (int d = 0; d < n; ++d) {
+    std::vector<std::pair<int64_t, int64_t>> iv;
+    for (int s = 0; s < n; ++s)
+      if (send_counts[s * n + d] > 0) iv.push_back({recv_displs[d * n + s], recv_displs[d * n + s] + send_counts[s * n + d]});
+    std::sort(iv.begin(), iv.end());
+    for (size_t i = 1; i < iv.size(); ++i)
+      if (iv[i].first < iv[i - 1].second) return COLL_ERR_ALIAS;
+  }
+  for (int d = 0; d < n; ++d)
+    for (int e = 0; e < n; ++e) {
+      if (e > d && overlap(recv[d], recv_end[d] * row, recv[e], recv_end[e] * row)) return COLL_ERR_ALIAS;
+      if (overlap(recv[d], recv_end[d] * row, send[e], send_end[e] * row)) return COLL_ERR_ALIAS;
+    }
+  std::vector<CopyJob> jobs;
+  jobs.reserve(static_cast<size_t>(n) * n);
+  for (int s = 0; s < n; ++s)
+    for (int d = 0; d < n; ++d) {
+      const int64_t c = send_counts[s * n + d];
+      if (c == 0) continue;
+      jobs.push_back({static_cast<const char*>(send[s]) + static_cast<size_t>(send_displs[s * n + d]) * row,
+                      static_cast<char*>(recv[d]) + static_cast<size_t>(recv_displs[d * n + s]) * row,
+                      static_cast<size_t>(c) * row});
+    }
+  return launch_copy_jobs(jobs.data(), static_cast<int>(jobs.size()), S(stream));
+}
+
+// --------------------------------------------------------------- packets ----
+size_t coll_packed_bytes(size_t bytes, coll_proto_t proto) {
+  switch (proto) {
+    case COLL_PROTO_SIMPLE: return bytes;
+    case COLL_PROTO_LL: return 8 * ((bytes + 3) / 4);
+    case COLL_PROTO_LL128: return 128 * ((bytes + 119) / 120);
+  }
+  return 0;
+}
+
+static bool valid_step(coll_proto_t proto, uint64_t step) {
+  if (step == 0) return false;
+  if (proto == COLL_PROTO_LL && static_cast<uint32_t>(step) == 0) return false;
+  return true;
+}
+
+int coll_ll_pack(const void* src, void* packed, size_t bytes, coll_proto_t proto, uint64_t step, coll_stream_t stream) {
+  if (proto != COLL_PROTO_LL && proto != COLL_PROTO_LL128) return COLL_ERR_UNSUPPORTED;
+  if (src == nullptr || packed == nullptr || !valid_step(proto, step) || !al16(packed)) return COLL_ERR_INVALID_ARG;
+  if (bytes == 0) return COLL_OK;
+  if (overlap(src, bytes, packed, coll_packed_bytes(bytes, proto))) return COLL_ERR_ALIAS;
+  return launch_ll_pack(src, packed, bytes, proto, step, S(stream));
+}
+
+int coll_ll_unpack(const void* packed, void* dst, size_t bytes, coll_proto_t proto, uint64_t step, int* d_status,
+                   coll_stream_t stream) {
+  if (proto != COLL_PROTO_LL && proto != COLL_PROTO_LL128) return COLL_ERR_UNSUPPORTED;
+  if (dst == nullptr || packed == nullptr || !valid_step(proto, step) || !al16(packed)) return COLL_ERR_INVALID_ARG;
+  if (bytes == 0) return COLL_OK;
+  if (overlap(dst, bytes, packed, coll_packed_bytes(bytes, proto))) return COLL_ERR_ALIAS;
+  return launch_ll_unpack(packed, dst, bytes, proto, step, d_status, S(stream));
+}
+
+int coll_all_reduce_packed(const void* const* packed_in, void* const* packed_out, int nranks, size_t count,
+                           coll_dtype_t dtype, coll_op_t op, coll_proto_t proto, uint64_t step, int* d_status,
+                           coll_stream_t stream) {
+  if (proto == COLL_PROTO_SIMPLE)
+    return coll_all_reduce(packed_in, packed_out, nranks, count, dtype, op, COLL_ALGO_TWOSHOT, nullptr, 0, stream);
+  const int es = elem_size(dtype);
+  if (!es) return COLL_ERR_UNSUPPORTED;
+  if (!valid_op(op) || (proto != COLL_PROTO_LL && proto != COLL_PROTO_LL128)) return COLL_ERR_UNSUPPORTED;
+  if (!valid_n(nranks) || !all_nonnull(packed_in, nranks) || !all_nonnull(packed_out, nranks) ||
+      !valid_step(proto, step))
+    return COLL_ERR_INVALID_ARG;
+  const size_t payload = count * es;
+  if (payload == 0) return COLL_OK;
+  const size_t pbytes = coll_packed_bytes(payload, proto);
+  for (int r = 0; r < nranks; ++r)
+    if (!al16(packed_in[r]) || !al16(packed_out[r])) return COLL_ERR_INVALID_ARG;
+  if (!outputs_disjoint(packed_out, nranks, pbytes)) return COLL_ERR_ALIAS;
+  for (int q = 0; q < nranks; ++q)
+    for (int r = 0; r < nranks; ++r)
+      if (overlap(packed_out[q], pbytes, packed_in[r], pbytes) && !(q == r && packed_out[q] == packed_in[r]))
+        return COLL_ERR_ALIAS;
+  PackedReduceArgs a{};
+  for (int r = 0; r < nranks; ++r) {
+    a.in[r] = static_cast<const char*>(packed_in[r]);
+    a.out[r] = static_cast<char*>(packed_out[r]);
+  }
+  a.nlines = pbytes / (proto == COLL_PROTO_LL ? 8 : 128);
+  a.payload_bytes = payload;
+  a.step = step;
+  a.n = nranks;
+  a.status = d_status;
+  return launch_all_reduce_packed(a, dtype, op, proto, S(stream));
+}
+
+// ------------------------------------------------------------------- MoE ----
+static bool moe_shape_ok(int nranks, int tokens, int topk, int n_experts) {
+  if (!valid_n(nranks) || tokens < 0 || topk < 1 || topk > 32) return false;
+  if (n_experts < nranks || n_experts > COLL_MAX_EXPERTS || n_experts % nranks != 0) return false;
+  if (static_cast<int64_t>(nranks) * tokens * topk >= (int64_t{1} << 31)) return false;
+  return true;
+}
+
+size_t coll_moe_route_workspace_size(int nranks, int tokens, int topk, int n_experts) {
+  if (!moe_shape_ok(nranks, tokens, topk, n_experts)) return 0;
+  return moe_route_workspace(nranks, tokens, topk, n_experts);
+}
+
+int coll_moe_route(const int32_t* const* topk_ids, int nranks, int tokens, int topk, int n_experts,
+                   int64_t* d_send_counts, int64_t* d_send_displs, int64_t* d_recv_displs, int32_t* const* d_pos,
+                   int* d_status, void* workspace, size_t workspace_bytes, coll_stream_t stream) {
+  if (!moe_shape_ok(nranks, tokens, topk, n_experts)) return COLL_ERR_INVALID_ARG;
+  if (!all_nonnull(topk_ids, nranks) || !all_nonnull(d_pos, nranks) || !d_send_counts || !d_send_displs ||
+      !d_recv_displs)
+    return COLL_ERR_INVALID_ARG;
+  const size_t need = moe_route_workspace(nranks, tokens, topk, n_experts);
+  if (workspace == nullptr || workspace_bytes < need || (U(workspace) & 255) != 0) return COLL_ERR_WORKSPACE;
+  MoeRouteArgs a{};
+  for (int r = 0; r < nranks; ++r) {
+    a.ids[r] = topk_ids[r];
+    a.pos[r] = d_pos[r];
+  }
+  a.send_counts = d_send_counts;
+  a.send_displs = d_send_displs;
+  a.recv_displs = d_recv_displs;
+  a.n = nranks;
+  a.tokens = tokens;
+  a.topk = topk;
+  a.n_experts = n_experts;
+  a.tiles = std::max(1, (tokens + 255) / 256);
+  const size_t cells = static_cast<size_t>(nranks) * n_experts * a.tiles;
+  a.tile_cnt = static_cast<int32_t*>(workspace);
+  a.tile_base = reinterpret_cast<int64_t*>(static_cast<char*>(workspace) + (cells * 4 + 255) / 256 * 256);
+  a.status = d_status;
+  return launch_moe_route(a, S(stream));
+}
+
+int coll_moe_dispatch(const void* const* x, const int32_t* const* topk_ids, const int32_t* const* d_pos,
+                      void* const* recv, int nranks, int tokens, int topk, int n_experts, size_t hidden,
+                      coll_dtype_t dtype, int64_t recv_capacity_rows, int* d_status, coll_stream_t stream) {
+  const int es = elem_size(dtype);
+  if (!es) return COLL_ERR_UNSUPPORTED;
+  if (!moe_shape_ok(nranks, tokens, topk, n_experts) || recv_capacity_rows < 0) return COLL_ERR_INVALID_ARG;
+  if (!all_nonnull(x, nranks) || !all_nonnull(topk_ids, nranks) || !all_nonnull(d_pos, nranks) ||
+      !all_nonnull(recv, nranks))
+    return COLL_ERR_INVALID_ARG;
+  const size_t row = hidden * es;
+  if (row == 0 || tokens == 0) return COLL_OK;
+  const size_t in_bytes = row * tokens, out_bytes = row * static_cast<size_t>(recv_capacity_rows);
+  if (!outputs_disjoint(recv, nranks, out_bytes)) return COLL_ERR_ALIAS;
+  for (int d = 0; d < nranks; ++d)
+    for (int s = 0; s < nranks; ++s)
+      if (overlap(recv[d], out_bytes, x[s], in_bytes)) return COLL_ERR_ALIAS;
+  MoeMoveArgs a{};
+  for (int r = 0; r < nranks; ++r) {
+    a.x[r] = static_cast<const char*>(x[r]);
+    a.y[r] = static_cast<char*>(recv[r]);
+    a.ids[r] = topk_ids[r];
+    a.pos[r] = d_pos[r];
+  }
+  a.row_bytes = row;
+  a.capacity = recv_capacity_rows;
+  a.status = d_status;
+  a.n = nranks;
+  a.tokens = tokens;
+  a.topk = topk;
+  a.epr = n_experts / nranks;
+  return launch_moe_dispatch(a, S(stream));
+}
+
+int coll_moe_combine(const void* const* y, const int32_t* const* topk_ids, const int32_t* const* d_pos,
+                     const float* const* topk_w, void* const* out, int nranks, int tokens, int topk, int n_experts,
+                     size_t hidden, coll_dtype_t dtype, int64_t recv_capacity_rows, int* d_status,
+                     coll_stream_t stream) {
+  const int es = elem_size(dtype);
+  if (!es || dtype == COLL_INT32) return COLL_ERR_UNSUPPORTED;
+  if (!moe_shape_ok(nranks, tokens, topk, n_experts) || recv_capacity_rows < 0) return COLL_ERR_INVALID_ARG;
+  if (!all_nonnull(y, nranks) || !all_nonnull(topk_ids, nranks) || !all_nonnull(d_pos, nranks) ||
+      !all_nonnull(topk_w, nranks) || !all_nonnull(out, nranks))
+    return COLL_ERR_INVALID_ARG;
+  const size_t row = hidden * es;
+  if (row == 0 || tokens == 0) return COLL_OK;
+  const size_t out_bytes = row * tokens, in_bytes = row * static_cast<size_t>(recv_capacity_rows);
+  if (!outputs_disjoint(out, nranks, out_bytes)) return COLL_ERR_ALIAS;
+  for (int d = 0; d < nranks; ++d)
+    for (int s = 0; s < nranks; ++s)
+      if (overlap(out[d], out_bytes, y[s], in_bytes)) return COLL_ERR_ALIAS;
+  MoeMoveArgs a{};
+  for (int r = 0; r < nranks; ++r) {
+    a.x[r] = static_cast<const char*>(y[r]);
+    a.y[r] = static_cast<char*>(out[r]);
+    a.ids[r] = topk_ids[r];
+    a.pos[r] = d_pos[r];
+    a.w[r] = topk_w[r];
+  }
+  a.row_bytes = row;
+  a.capacity = recv_capacity_rows;
+  a.status = d_status;
+  a.n = nranks;
+  a.tokens = tokens;
+  a.topk = topk;
+  a.epr = n_experts / nranks;
+  return launch_moe_combine(a, dtype, S(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,202 @@
+// Movement kernels: bit copies between virtual-rank buffers.
+//
+//  k_fanout      one read, many writes: broadcast (vLLM collectives tutorial
+//                section 1.1) and all-gather (section 7.1) read every source
+//                element once and store it to every destination.
+//  k_copy_jobs   a list of independent 1-D copies, partitioned over the grid
+//                by byte ranges so that very unequal blocks (all-to-all-v,
+//                section 8.2) still spread evenly: scatter, flat gather,
+//                all-to-all, all-to-all-v and the ring's all-gather steps.
+//  k_gather_rows the last-dimension gather of section 2.2.1: rank r's
+//                [rows, cols] block lands at columns [r*cols, (r+1)*cols).
+//
+// All three move 16-byte units when every address and length allows it and
+// fall back to narrower units otherwise.
+#include <algorithm>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace mvr {
+
+static int pick_unit(uint64_t bits) {
+  // largest power of two <= 16 that divides every address / length OR-ed into `bits`
+  if ((bits & 15) == 0) return 16;
+  if ((bits & 7) == 0) return 8;
+  if ((bits & 3) == 0) return 4;
+  if ((bits & 1) == 0) return 2;
+  return 1;
+}
+
+static unsigned grid_for(uint64_t units, int slices) {
+  uint64_t want = (units + kThreads - 1) / kThreads;
+  const uint64_t cap = std::max<uint64_t>(1, static_cast<uint64_t>(num_sms()) * 8 / std::max(1, slices));
+  want = std::min(want, cap);
+  return static_cast<unsigned>(std::max<uint64_t>(1, want) * slices);
+}
+
+// ------------------------------------------------------------- fan-out ----
+
+template <int U>
+__global__ void __launch_bounds__(kThreads) k_fanout(const __grid_constant__ FanoutArgs a) {
+  const int r = blockIdx.x % a.ns;
+  const int part = blockIdx.x / a.ns;
+  const int parts = gridDim.x / a.ns;
+  const uint64_t units = a.bytes / U;
+  const uint64_t stride = static_cast<uint64_t>(parts) * blockDim.x;
+  const char* src = a.src[r];
+  const uint64_t roff = static_cast<uint64_t>(r) * a.dst_stride;
+  for (uint64_t u = static_cast<uint64_t>(part) * blockDim.x + threadIdx.x; u < units; u += stride) {
+    const auto x = ldu<U>(src + u * U);
+#pragma unroll 8
+    for (int q = 0; q < a.nd; ++q) {
+      if (a.skip_diag && q == r) continue;
+      stu<U>(a.dst[q] + roff + u * U, x);
+    }
+  }
+  if (part == 0) {  // bytes beyond the last whole unit
+    const uint64_t b = units * U + threadIdx.x;
+    if (b < a.bytes) {
+      const char x = src[b];
+      for (int q = 0; q < a.nd; ++q) {
+        if (a.skip_diag && q == r) continue;
+        a.dst[q][roff + b] = x;
+      }
+    }
+  }
+}
+
+int launch_fanout(const FanoutArgs& a, cudaStream_t s) {
+  if (a.bytes == 0 || a.ns == 0 || a.nd == 0) return COLL_OK;
+  uint64_t bits = a.dst_stride;
+  for (int r = 0; r < a.ns; ++r) bits |= reinterpret_cast<uintptr_t>(a.src[r]);
+  for (int q = 0; q < a.nd; ++q) bits |= reinterpret_cast<uintptr_t>(a.dst[q]);
+  const int U = pick_unit(bits);
+  const unsigned grid = grid_for(a.bytes / U, a.ns);
+  switch (U) {
+    case 16: k_fanout<16><<<grid, kThreads, 0, s>>>(a); break;
+    case 8: k_fanout<8><<<grid, kThreads, 0, s>>>(a); break;
+    case 4: k_fanout<4><<<grid, kThreads, 0, s>>>(a); break;
+    case 2: k_fanout<2><<<grid, kThreads, 0, s>>>(a); break;
+    default: k_fanout<1><<<grid, kThreads, 0, s>>>(a); break;
+  }
+  return launch_status(cudaGetLastError());
+}
+
+// ------------------------------------------------------------ copy jobs ----
+
+struct JobU {
+  const char* src;
+  char* dst;
+  uint64_t start;  // first unit of this job in the concatenation of all jobs
+};
+constexpr int kMaxJobs = 960;  // 960 * 24 B + header < 32 KB of kernel parameters
+struct CopyJobsArgs {
+  uint64_t total;  // units over all jobs
+  int njobs;
+  JobU job[kMaxJobs + 1];  // job[njobs].start == total (sentinel)
+};
+
+template <int U>
+__global__ void __launch_bounds__(kThreads) k_copy_jobs(const __grid_constant__ CopyJobsArgs a) {
+  // block b owns the contiguous unit range [b*total/B, (b+1)*total/B)
+  const uint64_t B = gridDim.x;
+  const uint64_t lo = a.total * blockIdx.x / B;
+  const uint64_t hi = a.total * (blockIdx.x + 1) / B;
+  if (lo >= hi) return;
+  // first job holding `lo` (binary search; uniform over the block)
+  int j0 = 0, j1 = a.njobs - 1;
+  while (j0 < j1) {
+    const int m = (j0 + j1 + 1) >> 1;
+    if (a.job[m].start <= lo) j0 = m;
+    else j1 = m - 1;
+  }
+  int j = j0;
+  for (uint64_t u = lo + threadIdx.x; u < hi; u += blockDim.x) {
+    while (u >= a.job[j + 1].start) ++j;
+    const uint64_t off = (u - a.job[j].start) * U;
+    stu<U>(a.job[j].dst + off, ldu<U>(a.job[j].src + off));
+  }
+}
+
+int launch_copy_jobs(const CopyJob* jobs, int njobs, cudaStream_t s) {
+  // drop empty jobs; choose one unit for all jobs of a launch
+  std::vector<CopyJob> v;
+  v.reserve(njobs);
+  uint64_t bits = 0;
+  for (int i = 0; i < njobs; ++i) {
+    if (jobs[i].bytes == 0) continue;
+    v.push_back(jobs[i]);
+    bits |= reinterpret_cast<uintptr_t>(jobs[i].src) | reinterpret_cast<uintptr_t>(jobs[i].dst) | jobs[i].bytes;
+  }
+  if (v.empty()) return COLL_OK;
+  const int U = pick_unit(bits);
+  static thread_local CopyJobsArgs args;  // ~23 KB: keep it off the stack
+  for (size_t first = 0; first < v.size(); first += kMaxJobs) {
+    const int nj = static_cast<int>(std::min<size_t>(kMaxJobs, v.size() - first));
+    uint64_t acc = 0;
+    for (int i = 0; i < nj; ++i) {
+      args.job[i].src = v[first + i].src;
+      args.job[i].dst = v[first + i].dst;
+      args.job[i].start = acc;
+      acc += v[first + i].bytes / U;
+    }
+    args.job[nj].src = nullptr;
+    args.job[nj].dst = nullptr;
+    args.job[nj].start = acc;
+    args.total = acc;
+    args.njobs = nj;
+    uint64_t want = (acc + 4ull * kThreads - 1) / (4ull * kThreads);
+    want = std::min<uint64_t>(std::max<uint64_t>(want, 1), static_cast<uint64_t>(num_sms()) * 8);
+    const unsigned grid = static_cast<unsigned>(want);
+    switch (U) {
+      case 16: k_copy_jobs<16><<<grid, kThreads, 0, s>>>(args); break;
+      case 8: k_copy_jobs<8><<<grid, kThreads, 0, s>>>(args); break;
+      case 4: k_copy_jobs<4><<<grid, kThreads, 0, s>>>(args); break;
+      case 2: k_copy_jobs<2><<<grid, kThreads, 0, s>>>(args); break;
+      default: k_copy_jobs<1><<<grid, kThreads, 0, s>>>(args); break;
+    }
+    const int st = launch_status(cudaGetLastError());
+    if (st != COLL_OK) return st;
+  }
+  return COLL_OK;
+}
+
+// ---------------------------------------------------------- row gather ----
+
+template <int U>
+__global__ void __launch_bounds__(kThreads) k_gather_rows(const __grid_constant__ GatherRowsArgs a) {
+  // blockIdx.x = part * n + r ; parts stride over rows, threads over columns
+  const int r = blockIdx.x % a.n;
+  const int part = blockIdx.x / a.n;
+  const int parts = gridDim.x / a.n;
+  const uint64_t ru = a.row_bytes / U;
+  const char* src = a.src[r];
+  char* dst = a.dst + static_cast<uint64_t>(r) * a.row_bytes;
+  for (uint64_t row = part; row < a.rows; row += parts) {
+    const char* sp = src + row * a.row_bytes;
+    char* dp = dst + row * a.dst_pitch;
+    for (uint64_t u = threadIdx.x; u < ru; u += blockDim.x) stu<U>(dp + u * U, ldu<U>(sp + u * U));
+  }
+}
+
+int launch_gather_rows(const GatherRowsArgs& a, cudaStream_t s) {
+  if (a.rows == 0 || a.row_bytes == 0) return COLL_OK;
+  uint64_t bits = a.row_bytes | a.dst_pitch | reinterpret_cast<uintptr_t>(a.dst);
+  for (int r = 0; r < a.n; ++r) bits |= reinterpret_cast<uintptr_t>(a.src[r]);
+  const int U = pick_unit(bits);
+  // about 4 units per thread per row chunk; at most 8 CTAs per SM in total
+  uint64_t parts = std::min<uint64_t>(a.rows, std::max<uint64_t>(1, static_cast<uint64_t>(num_sms()) * 8 / a.n));
+  const unsigned grid = static_cast<unsigned>(parts * a.n);
+  switch (U) {
+    case 16: k_gather_rows<16><<<grid, kThreads, 0, s>>>(a); break;
+    case 8: k_gather_rows<8><<<grid, kThreads, 0, s>>>(a); break;
+    case 4: k_gather_rows<4><<<grid, kThreads, 0, s>>>(a); break;
+    case 2: k_gather_rows<2><<<grid, kThreads, 0, s>>>(a); break;
+    default: k_gather_rows<1><<<grid, kThreads, 0, s>>>(a); break;
+  }
+  return launch_status(cudaGetLastError());
+}
+
+}  // namespace mvr

@@ -1,0 +1,118 @@
+// Host-side interface between the C-ABI layer (api.cu) and the kernel files.
+// Argument structs are passed to kernels by value as __grid_constant__
+// parameters (sm_100a accepts up to 32 KB of kernel parameters).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "coll.h"
+
+namespace mvr {
+
+constexpr int kMaxRanksH = COLL_MAX_RANKS;
+constexpr int kBlockThreads = 256;  // threads per CTA of the element-wise kernels
+
+int num_sms();                      // SM count of the current device (cached)
+int elem_size(coll_dtype_t dt);     // 2 or 4, 0 for an unknown dtype
+int launch_status(cudaError_t e);   // COLL_OK or COLL_ERR_CUDA (remembers the error text)
+
+// ----------------------------------------------------------- reductions ----
+struct ReduceArgs {
+  const char* in[kMaxRanksH];
+  char* out[kMaxRanksH];
+  uint64_t count;   // elements of the reduced index range of every input
+  uint64_t seg;     // elements per slice (owner segment / output block); ignored by ONESHOT
+  int nin;          // ranks reduced
+  int nout;         // M_ALL: output ranks written
+  int nslices;      // slices interleaved over blockIdx.x
+};
+// mode: mvr::ReduceMode.  vec: all addresses and slice starts 16-byte aligned.
+int launch_reduce(const ReduceArgs& a, coll_dtype_t dt, coll_op_t op, int mode, bool vec,
+                  int blocks_per_slice, cudaStream_t s);
+
+struct RingStepArgs {
+  const char* in[kMaxRanksH];
+  char* out[kMaxRanksH];
+  char* partial;    // arithmetic-type partials, indexed by element
+  uint64_t count, seg;
+  int n, k;         // ranks, step 1 .. n-1 of the reduce-scatter phase
+};
+int launch_ring_rs_step(const RingStepArgs& a, coll_dtype_t dt, coll_op_t op, bool vec,
+                        cudaStream_t s);
+
+// ---------------------------------------------------------------- copies ----
+struct FanoutArgs {
+  const char* src[kMaxRanksH];
+  char* dst[kMaxRanksH];
+  uint64_t bytes;       // bytes per source
+  uint64_t dst_stride;  // dst for (source r, destination q) = dst[q] + r * dst_stride
+  int ns, nd;
+  int skip_diag;        // skip q == r (in-place all-gather)
+};
+int launch_fanout(const FanoutArgs& a, cudaStream_t s);
+
+struct CopyJob {
+  const char* src;
+  char* dst;
+  uint64_t bytes;
+};
+// any number of independent 1-D copies (split over several launches if needed)
+int launch_copy_jobs(const CopyJob* jobs, int njobs, cudaStream_t s);
+
+struct GatherRowsArgs {
+  const char* src[kMaxRanksH];
+  char* dst;
+  uint64_t rows, row_bytes, dst_pitch;
+  int n;
+};
+int launch_gather_rows(const GatherRowsArgs& a, cudaStream_t s);
+
+// --------------------------------------------------------------- packets ----
+int launch_ll_pack(const void* src, void* packed, size_t bytes, int proto, uint64_t step,
+                   cudaStream_t s);
+int launch_ll_unpack(const void* packed, void* dst, size_t bytes, int proto, uint64_t step,
+                     int* status, cudaStream_t s);
+
+struct PackedReduceArgs {
+  const char* in[kMaxRanksH];
+  char* out[kMaxRanksH];
+  uint64_t nlines;       // lines per rank
+  uint64_t payload_bytes;
+  uint64_t step;
+  int n;
+  int* status;
+};
+int launch_all_reduce_packed(const PackedReduceArgs& a, coll_dtype_t dt, coll_op_t op, int proto,
+                             cudaStream_t s);
+
+// -------------------------------------------------------------------- MoE ----
+struct MoeRouteArgs {
+  const int32_t* ids[kMaxRanksH];
+  int32_t* pos[kMaxRanksH];
+  int64_t* send_counts;  // [N*N]
+  int64_t* send_displs;  // [N*N]
+  int64_t* recv_displs;  // [N*N] (d-major)
+  int32_t* tile_cnt;     // workspace [N][E][tiles]
+  int64_t* tile_base;    // workspace [N][E][tiles]
+  int* status;
+  int n, tokens, topk, n_experts, tiles;
+};
+size_t moe_route_workspace(int n, int tokens, int topk, int n_experts);
+int launch_moe_route(const MoeRouteArgs& a, cudaStream_t s);
+
+struct MoeMoveArgs {
+  const char* x[kMaxRanksH];      // dispatch: token rows; combine: expert outputs y
+  char* y[kMaxRanksH];            // dispatch: receive buffers; combine: outputs
+  const int32_t* ids[kMaxRanksH];
+  const int32_t* pos[kMaxRanksH];
+  const float* w[kMaxRanksH];
+  uint64_t row_bytes;
+  int64_t capacity;
+  int* status;
+  int n, tokens, topk, epr;
+};
+int launch_moe_dispatch(const MoeMoveArgs& a, cudaStream_t s);
+int launch_moe_combine(const MoeMoveArgs& a, coll_dtype_t dt, cudaStream_t s);
+
+}  // namespace mvr

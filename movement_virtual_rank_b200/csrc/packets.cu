@@ -1,0 +1,334 @@
+// LL and LL128 packets ("From NCCL Ring LL to PCIe IPC AllReduce", section
+// "Traditional LL Protocols"): an LL line is [4 B data | 4 B flag], an LL128
+// line is [120 B data | 8 B flag].  The receive side of the page's section
+// "Pro5000 ?" reads 16-byte groups and accepts the data only when every flag
+// in the group equals the current step; here that check is a validation of
+// stream-ordered data, counted into the device status, never a wait.
+//
+// LL:    one thread per 16-byte group = two lines; a thread of pack reads 16
+//        message bytes and writes 32 packet bytes.
+// LL128: eight threads per 128-byte line, thread j owning packet bytes
+//        [16j, 16j+16); thread 7's chunk carries 8 data bytes and the flag.
+//        Message offsets 120L + 16j are only 8-byte aligned, so message-side
+//        accesses are 8 bytes wide, packet-side ones 16.
+#include "common.cuh"
+#include "internal.h"
+
+namespace mvr {
+
+static unsigned grid_units(uint64_t units) {
+  uint64_t want = (units + kThreads - 1) / kThreads;
+  const uint64_t cap = static_cast<uint64_t>(num_sms()) * 8;
+  if (want > cap) want = cap;
+  if (want < 1) want = 1;
+  return static_cast<unsigned>(want);
+}
+
+// little-endian bytes [off, off+len) of src, zero beyond `bytes`, as a u32/u64
+__device__ __forceinline__ uint32_t load_word_tail(const uint8_t* src, uint64_t off, uint64_t bytes) {
+  uint32_t w = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (off + i < bytes) w |= static_cast<uint32_t>(src[off + i]) << (8 * i);
+  return w;
+}
+__device__ __forceinline__ uint2 load8_any(const uint8_t* src, uint64_t off, uint64_t bytes, bool al8) {
+  if (off + 8 <= bytes && al8) return ld8(src + off);
+  return make_uint2(load_word_tail(src, off, bytes), load_word_tail(src, off + 4, bytes));
+}
+__device__ __forceinline__ void store_bytes(uint8_t* dst, uint64_t off, uint64_t bytes, uint32_t w) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (off + i < bytes) dst[off + i] = static_cast<uint8_t>(w >> (8 * i));
+}
+__device__ __forceinline__ void store8_any(uint8_t* dst, uint64_t off, uint64_t bytes, uint2 v, bool al8) {
+  if (off + 8 <= bytes && al8) {
+    st8(dst + off, v);
+  } else {
+    store_bytes(dst, off, bytes, v.x);
+    store_bytes(dst, off + 4, bytes, v.y);
+  }
+}
+
+// ------------------------------------------------------------------ LL ----
+
+__global__ void __launch_bounds__(kThreads) k_ll_pack(const uint8_t* __restrict__ src, uint8_t* __restrict__ packed,
+                                                      uint64_t bytes, uint32_t flag, int src_al16) {
+  const uint64_t nlines = (bytes + 3) / 4;
+  const uint64_t ngroups = nlines / 4;  // groups of 4 lines = 16 message bytes
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  const uint64_t t0 = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const uint64_t full = src_al16 ? bytes / 16 : 0;  // groups read with one 16-byte load
+  for (uint64_t g = t0; g < ngroups; g += stride) {
+    uint4 x;
+    if (g < full) {
+      x = ld16(src + 16 * g);
+    } else {
+      x.x = load_word_tail(src, 16 * g, bytes);
+      x.y = load_word_tail(src, 16 * g + 4, bytes);
+      x.z = load_word_tail(src, 16 * g + 8, bytes);
+      x.w = load_word_tail(src, 16 * g + 12, bytes);
+    }
+    st16(packed + 32 * g, make_uint4(x.x, flag, x.y, flag));
+    st16(packed + 32 * g + 16, make_uint4(x.z, flag, x.w, flag));
+  }
+  for (uint64_t L = 4 * ngroups + t0; L < nlines; L += stride)  // last 1..3 lines
+    st8(packed + 8 * L, make_uint2(load_word_tail(src, 4 * L, bytes), flag));
+}
+
+__global__ void __launch_bounds__(kThreads) k_ll_unpack(const uint8_t* __restrict__ packed, uint8_t* __restrict__ dst,
+                                                        uint64_t bytes, uint32_t flag, int dst_al16, int* status) {
+  const uint64_t nlines = (bytes + 3) / 4;
+  const uint64_t ngroups = nlines / 4;
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  const uint64_t t0 = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  int bad = 0;
+  for (uint64_t g = t0; g < ngroups; g += stride) {
+    const uint4 a = ld16(packed + 32 * g);
+    const uint4 b = ld16(packed + 32 * g + 16);
+    bad += (a.y != flag) + (a.w != flag) + (b.y != flag) + (b.w != flag);
+    if (dst_al16 && 16 * g + 16 <= bytes) {
+      st16(dst + 16 * g, make_uint4(a.x, a.z, b.x, b.z));
+    } else {
+      store_bytes(dst, 16 * g, bytes, a.x);
+      store_bytes(dst, 16 * g + 4, bytes, a.z);
+      store_bytes(dst, 16 * g + 8, bytes, b.x);
+      store_bytes(dst, 16 * g + 12, bytes, b.z);
+    }
+  }
+  for (uint64_t L = 4 * ngroups + t0; L < nlines; L += stride) {
+    const uint2 v = ld8(packed + 8 * L);
+    bad += (v.y != flag);
+    store_bytes(dst, 4 * L, bytes, v.x);
+  }
+  report_warp(status, COLL_DEV_FLAG_MISMATCH, bad);
+}
+
+// --------------------------------------------------------------- LL128 ----
+
+__global__ void __launch_bounds__(kThreads) k_ll128_pack(const uint8_t* __restrict__ src, uint8_t* __restrict__ packed,
+                                                         uint64_t bytes, uint64_t step, int src_al8) {
+  const uint64_t nlines = (bytes + 119) / 120;
+  const uint64_t nthreads = nlines * 8;
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  for (uint64_t t = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < nthreads; t += stride) {
+    const uint64_t L = t >> 3;
+    const int j = static_cast<int>(t & 7);
+    const uint64_t off = 120 * L + 16 * j;
+    const uint2 lo = load8_any(src, off, bytes, src_al8);
+    uint2 hi;
+    if (j < 7) hi = load8_any(src, off + 8, bytes, src_al8);
+    else hi = make_uint2(static_cast<uint32_t>(step), static_cast<uint32_t>(step >> 32));
+    st16(packed + 128 * L + 16 * j, make_uint4(lo.x, lo.y, hi.x, hi.y));
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) k_ll128_unpack(const uint8_t* __restrict__ packed, uint8_t* __restrict__ dst,
+                                                           uint64_t bytes, uint64_t step, int dst_al8, int* status) {
+  const uint64_t nlines = (bytes + 119) / 120;
+  const uint64_t nthreads = nlines * 8;
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  int bad = 0;
+  for (uint64_t t = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < nthreads; t += stride) {
+    const uint64_t L = t >> 3;
+    const int j = static_cast<int>(t & 7);
+    const uint4 x = ld16(packed + 128 * L + 16 * j);
+    const uint64_t off = 120 * L + 16 * j;
+    store8_any(dst, off, bytes, make_uint2(x.x, x.y), dst_al8);
+    if (j < 7) {
+      store8_any(dst, off + 8, bytes, make_uint2(x.z, x.w), dst_al8);
+    } else {
+      const uint64_t f = static_cast<uint64_t>(x.z) | (static_cast<uint64_t>(x.w) << 32);
+      bad += (f != step);
+    }
+  }
+  report_warp(status, COLL_DEV_FLAG_MISMATCH, bad);
+}
+
+int launch_ll_pack(const void* src, void* packed, size_t bytes, int proto, uint64_t step, cudaStream_t s) {
+  if (bytes == 0) return COLL_OK;
+  const auto* sp = static_cast<const uint8_t*>(src);
+  auto* pp = static_cast<uint8_t*>(packed);
+  if (proto == COLL_PROTO_LL) {
+    const uint64_t nlines = (bytes + 3) / 4;
+    k_ll_pack<<<grid_units(nlines / 4 + 1), kThreads, 0, s>>>(sp, pp, bytes, static_cast<uint32_t>(step),
+                                                               (reinterpret_cast<uintptr_t>(src) & 15) == 0);
+  } else {
+    const uint64_t nlines = (bytes + 119) / 120;
+    k_ll128_pack<<<grid_units(nlines * 8), kThreads, 0, s>>>(sp, pp, bytes, step,
+                                                              (reinterpret_cast<uintptr_t>(src) & 7) == 0);
+  }
+  return launch_status(cudaGetLastError());
+}
+
+int launch_ll_unpack(const void* packed, void* dst, size_t bytes, int proto, uint64_t step, int* status,
+                     cudaStream_t s) {
+  if (bytes == 0) return COLL_OK;
+  const auto* pp = static_cast<const uint8_t*>(packed);
+  auto* dp = static_cast<uint8_t*>(dst);
+  if (proto == COLL_PROTO_LL) {
+    const uint64_t nlines = (bytes + 3) / 4;
+    k_ll_unpack<<<grid_units(nlines / 4 + 1), kThreads, 0, s>>>(pp, dp, bytes, static_cast<uint32_t>(step),
+                                                                 (reinterpret_cast<uintptr_t>(dst) & 15) == 0, status);
+  } else {
+    const uint64_t nlines = (bytes + 119) / 120;
+    k_ll128_unpack<<<grid_units(nlines * 8), kThreads, 0, s>>>(pp, dp, bytes, step,
+                                                                (reinterpret_cast<uintptr_t>(dst) & 7) == 0, status);
+  }
+  return launch_status(cudaGetLastError());
+}
+
+// ------------------------------------------------- packetised all-reduce ----
+
+// the elements of one 32-bit data word, zeroed at and beyond `limit`
+template <int DT, int OP>
+struct WordOps {
+  static constexpr int kE = 4 / Elem<DT>::kSize;
+  using A = typename Elem<DT>::A;
+  static __device__ __forceinline__ void widen(uint32_t w, A (&o)[kE]) {
+    if constexpr (kE == 2) {
+      o[0] = widen1<DT>(static_cast<uint16_t>(w & 0xFFFFu));
+      o[1] = widen1<DT>(static_cast<uint16_t>(w >> 16));
+    } else {
+      o[0] = widen1<DT>(w);
+    }
+  }
+  static __device__ __forceinline__ void step(A (&acc)[kE], uint32_t w) {
+    A v[kE];
+    widen(w, v);
+#pragma unroll
+    for (int i = 0; i < kE; ++i) acc[i] = op_step<OP>(acc[i], v[i]);
+  }
+  // elem0: element index of the word's first element; count: payload elements
+  static __device__ __forceinline__ uint32_t narrow(const A (&acc)[kE], uint64_t elem0, uint64_t count) {
+    if constexpr (kE == 2) {
+      const uint32_t lo = elem0 < count ? narrow1<DT>(acc[0]) : 0u;
+      const uint32_t hi = elem0 + 1 < count ? narrow1<DT>(acc[1]) : 0u;
+      return lo | (hi << 16);
+    } else {
+      return elem0 < count ? narrow1<DT>(acc[0]) : 0u;
+    }
+  }
+};
+
+// LL: thread = one 8-byte line per rank when `single`, else two lines (16 B)
+template <int DT, int OP>
+__global__ void __launch_bounds__(kThreads) k_ar_ll(const __grid_constant__ PackedReduceArgs a) {
+  using W = WordOps<DT, OP>;
+  using A = typename Elem<DT>::A;
+  constexpr int kE = W::kE;
+  const uint32_t flag = static_cast<uint32_t>(a.step);
+  const uint64_t count = a.payload_bytes / Elem<DT>::kSize;
+  const uint64_t ngroups = a.nlines / 2;
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  const uint64_t t0 = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  int bad = 0;
+  for (uint64_t g = t0; g < ngroups; g += stride) {
+    A acc0[kE], acc1[kE];
+    uint4 x = ld16(a.in[0] + 16 * g);
+    bad += (x.y != flag) + (x.w != flag);
+    W::widen(x.x, acc0);
+    W::widen(x.z, acc1);
+    for (int r = 1; r < a.n; ++r) {
+      x = ld16(a.in[r] + 16 * g);
+      bad += (x.y != flag) + (x.w != flag);
+      W::step(acc0, x.x);
+      W::step(acc1, x.z);
+    }
+    const uint64_t e0 = 2 * g * kE;  // first element of line 2g
+    const uint4 o = make_uint4(W::narrow(acc0, e0, count), flag, W::narrow(acc1, e0 + kE, count), flag);
+    for (int q = 0; q < a.n; ++q) st16(a.out[q] + 16 * g, o);
+  }
+  if ((a.nlines & 1) && t0 == 0) {  // odd last line
+    const uint64_t L = a.nlines - 1;
+    A acc[kE];
+    uint2 x = ld8(a.in[0] + 8 * L);
+    bad += (x.y != flag);
+    W::widen(x.x, acc);
+    for (int r = 1; r < a.n; ++r) {
+      x = ld8(a.in[r] + 8 * L);
+      bad += (x.y != flag);
+      W::step(acc, x.x);
+    }
+    const uint2 o = make_uint2(W::narrow(acc, L * kE, count), flag);
+    for (int q = 0; q < a.n; ++q) st8(a.out[q] + 8 * L, o);
+  }
+  report_warp(a.status, COLL_DEV_FLAG_MISMATCH, bad);
+}
+
+// LL128: eight threads per line, thread j owns packet bytes [16j, 16j+16)
+template <int DT, int OP>
+__global__ void __launch_bounds__(kThreads) k_ar_ll128(const __grid_constant__ PackedReduceArgs a) {
+  using W = WordOps<DT, OP>;
+  using A = typename Elem<DT>::A;
+  constexpr int kE = W::kE;
+  constexpr int ES = Elem<DT>::kSize;
+  const uint64_t count = a.payload_bytes / ES;
+  const uint64_t nthreads = a.nlines * 8;
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+  int bad = 0;
+  for (uint64_t t = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < nthreads; t += stride) {
+    const uint64_t L = t >> 3;
+    const int j = static_cast<int>(t & 7);
+    const uint64_t poff = 128 * L + 16 * j;
+    const uint64_t e0 = (120 * L + 16 * j) / ES;  // first element of this chunk
+    A acc[4][kE];
+    uint4 x = ld16(a.in[0] + poff);
+    if (j == 7) bad += ((static_cast<uint64_t>(x.z) | (static_cast<uint64_t>(x.w) << 32)) != a.step);
+    W::widen(x.x, acc[0]);
+    W::widen(x.y, acc[1]);
+    W::widen(x.z, acc[2]);
+    W::widen(x.w, acc[3]);
+    for (int r = 1; r < a.n; ++r) {
+      x = ld16(a.in[r] + poff);
+      if (j == 7) bad += ((static_cast<uint64_t>(x.z) | (static_cast<uint64_t>(x.w) << 32)) != a.step);
+      W::step(acc[0], x.x);
+      W::step(acc[1], x.y);
+      W::step(acc[2], x.z);
+      W::step(acc[3], x.w);
+    }
+    uint4 o;
+    o.x = W::narrow(acc[0], e0, count);
+    o.y = W::narrow(acc[1], e0 + kE, count);
+    if (j < 7) {
+      o.z = W::narrow(acc[2], e0 + 2 * kE, count);
+      o.w = W::narrow(acc[3], e0 + 3 * kE, count);
+    } else {
+      o.z = static_cast<uint32_t>(a.step);
+      o.w = static_cast<uint32_t>(a.step >> 32);
+    }
+    for (int q = 0; q < a.n; ++q) st16(a.out[q] + poff, o);
+  }
+  report_warp(a.status, COLL_DEV_FLAG_MISMATCH, bad);
+}
+
+template <int DT, int OP>
+static int launch_ar_packed_t(const PackedReduceArgs& a, int proto, cudaStream_t s) {
+  if (proto == COLL_PROTO_LL) k_ar_ll<DT, OP><<<grid_units(a.nlines / 2 + 1), kThreads, 0, s>>>(a);
+  else k_ar_ll128<DT, OP><<<grid_units(a.nlines * 8), kThreads, 0, s>>>(a);
+  return launch_status(cudaGetLastError());
+}
+
+template <int DT>
+static int launch_ar_packed_dt(const PackedReduceArgs& a, coll_op_t op, int proto, cudaStream_t s) {
+  switch (op) {
+    case COLL_SUM: return launch_ar_packed_t<DT, COLL_SUM>(a, proto, s);
+    case COLL_MAX: return launch_ar_packed_t<DT, COLL_MAX>(a, proto, s);
+    case COLL_MIN: return launch_ar_packed_t<DT, COLL_MIN>(a, proto, s);
+    case COLL_PROD: return launch_ar_packed_t<DT, COLL_PROD>(a, proto, s);
+  }
+  return COLL_ERR_UNSUPPORTED;
+}
+
+int launch_all_reduce_packed(const PackedReduceArgs& a, coll_dtype_t dt, coll_op_t op, int proto, cudaStream_t s) {
+  if (a.nlines == 0) return COLL_OK;
+  switch (dt) {
+    case COLL_BF16: return launch_ar_packed_dt<COLL_BF16>(a, op, proto, s);
+    case COLL_FP16: return launch_ar_packed_dt<COLL_FP16>(a, op, proto, s);
+    case COLL_FP32: return launch_ar_packed_dt<COLL_FP32>(a, op, proto, s);
+    case COLL_INT32: return launch_ar_packed_dt<COLL_INT32>(a, op, proto, s);
+  }
+  return COLL_ERR_UNSUPPORTED;
+}
+
+}  // namespace mvr

@@ -1,0 +1,4 @@
+// Reduction kernels instantiated for one element type (see reduce_impl.cuh).
+#include "reduce_impl.cuh"
+
+MVR_REDUCE_INSTANCE(int32, COLL_INT32)

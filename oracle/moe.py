@@ -104,8 +104,12 @@ def moe_dispatch(xs, topk_ids, pos, recv_bufs, n_experts: int, hidden: int):
     return outs
 
 
-def moe_combine(ys, topk_ids, pos, topk_w, n_experts: int, hidden: int, dtype: str):
-    """out[s][t] = round( sum_k w[s][t][k] * y[d_k][pos(s,t,k)] ), k ascending."""
+def moe_combine(ys, topk_ids, pos, topk_w, n_experts: int, hidden: int, dtype: str, tokens=None):
+    """out[s][t] = round( sum_k w[s][t][k] * y[d_k][pos(s,t,k)] ), k ascending.
+
+    ``tokens`` (optional, per source a list of token indices) restricts the
+    computation to those tokens; the result then holds their rows in order.
+    """
     n = len(topk_ids)
     epr = n_experts // n
     outs = []
@@ -113,14 +117,15 @@ def moe_combine(ys, topk_ids, pos, topk_w, n_experts: int, hidden: int, dtype: s
         ids2 = np.asarray(topk_ids[s])
         w = np.asarray(topk_w[s], dtype=np.float32)
         t_, k_ = ids2.shape
-        acc = np.zeros((t_, hidden), dtype=np.float32)
+        sel = list(range(t_)) if tokens is None else list(tokens[s])
+        acc = np.zeros((len(sel), hidden), dtype=np.float32)
         for k in range(k_):
-            rows = np.empty((t_, hidden), dtype=np.float32)
-            for t in range(t_):
+            rows = np.empty((len(sel), hidden), dtype=np.float32)
+            for i, t in enumerate(sel):
                 d = int(ids2[t, k]) // epr
                 p = int(pos[s][t * k_ + k])
-                rows[t] = widen(np.asarray(ys[d])[p * hidden:(p + 1) * hidden], dtype)
-            prod = (w[:, k:k + 1] * rows).astype(np.float32)
+                rows[i] = widen(np.asarray(ys[d])[p * hidden:(p + 1) * hidden], dtype)
+            prod = (w[sel, k:k + 1] * rows).astype(np.float32)
             acc = prod if k == 0 else (acc + prod).astype(np.float32)
         outs.append(narrow(acc.reshape(-1), dtype))
     return outs

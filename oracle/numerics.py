@@ -10,8 +10,10 @@ Readings taken (the pages fix none of these; the workloads do):
   (numpy float32 arithmetic), then ONE rounding to the storage type.
   Starting from x_0 rather than +0 keeps -0 when every input is -0.
 * Rounding to bf16 / fp16: round to nearest, ties to even (IEEE 754
-  roundTiesToEven); overflow goes to +-inf; NaN becomes the canonical quiet
-  NaN (bf16 0x7FC0, fp16 0x7E00), sign dropped.
+  roundTiesToEven); overflow goes to +-inf.  A NaN result of any float type
+  becomes the canonical quiet NaN (bf16 0x7FC0, fp16 0x7E00, fp32
+  0x7FC00000), sign and payload dropped: IEEE leaves NaN payloads to the
+  implementation, and x86 and the GPU pick different ones.
 * MAX / MIN (the tutorial's section 3.1 lists SUM, MAX, MIN, PROD): the
   running value is replaced only by a strictly greater (smaller) value, so
   between equal values (+0 / -0) the earlier rank wins; a NaN, once met,
@@ -107,7 +109,9 @@ def narrow(acc: np.ndarray, dtype: str) -> np.ndarray:
     if dtype == "fp16":
         return f32_to_f16_bits(acc)
     if dtype == "fp32":
-        return np.asarray(acc, dtype=np.float32)
+        out = np.array(acc, dtype=np.float32, copy=True)
+        out.view(np.uint32)[np.isnan(out)] = 0x7FC00000
+        return out
     if dtype == "int32":
         return np.asarray(acc, dtype=np.int32)
     raise ValueError(dtype)

@@ -1,0 +1,171 @@
+"""The C-ABI library on the CPU: it loads, exports every entry point that
+include/coll.h declares, and rejects bad arguments on the host before any
+launch.  No kernel runs here (these tests are skipped where a GPU is
+visible, because they pass made-up pointer values that must never reach a
+kernel)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import movement_virtual_rank_b200 as M
+import oracle
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "coll.h")
+no_gpu = pytest.mark.skipif(torch.cuda.is_available(), reason="host-only argument checks use fake pointers")
+
+
+def declared():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"^COLL_API\s+[\w\s\*]+?\b(coll_\w+)\s*\(", txt, flags=re.M)))
+
+
+def test_header_declarations_are_exported():
+    names = declared()
+    assert len(names) >= 20
+    L = M.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    # the binding covers exactly the declared entry points
+    assert sorted(M.symbols()) == names
+
+
+def test_exports_match_nm():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", M.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert set(declared()) <= exported
+    assert {e for e in exported if e.startswith("coll_")} == set(declared())
+
+
+def test_version_and_strerror():
+    assert M.coll_version() == 10000
+    for code in (0, -1, -2, -3, -4, -5):
+        assert M.coll_strerror(code)
+    assert M.coll_strerror(-99) == "unknown status"
+
+
+def test_packed_bytes_matches_oracle():
+    for nbytes in (0, 1, 3, 4, 5, 119, 120, 121, 1 << 20, (1 << 28) + 7):
+        for proto in (M.LL, M.LL128):
+            assert M.coll_packed_bytes(nbytes, proto) == oracle.packed_bytes(nbytes, proto)
+        assert M.coll_packed_bytes(nbytes, M.SIMPLE) == nbytes
+
+
+def test_workspace_sizes():
+    L = M.lib()
+    assert L.coll_all_reduce_workspace_size(8, 1000, M.BF16, M.TWOSHOT) == 0
+    ws = L.coll_all_reduce_workspace_size(8, 1000, M.BF16, M.RING)
+    assert ws >= 4000 and ws % 256 == 0
+    assert L.coll_moe_route_workspace_size(8, 4096, 8, 256) > 0
+    assert L.coll_moe_route_workspace_size(8, 4096, 8, 250) == 0  # experts not divisible by ranks
+    assert L.coll_moe_route_workspace_size(8, 4096, 8, 2048) == 0  # too many experts
+
+
+def _arr(vals):
+    a = (ctypes.c_void_p * len(vals))(*vals)
+    return ctypes.cast(a, ctypes.POINTER(ctypes.c_void_p)), a
+
+
+BASE = 0x7F0000000000  # made-up, 256-byte aligned addresses; never dereferenced
+
+
+@no_gpu
+def test_invalid_arguments_rejected_on_host():
+    L = M.lib()
+    p, _k = _arr([BASE + i * 0x100000 for i in range(4)])
+    q, _k2 = _arr([BASE + 0x10000000 + i * 0x100000 for i in range(4)])
+    null, _k3 = _arr([BASE, 0, BASE + 0x200000, BASE + 0x300000])
+    # rank counts, null pointers, out-of-range roots
+    assert L.coll_all_reduce(p, q, 0, 16, M.BF16, M.SUM, M.TWOSHOT, None, 0, None) == -1
+    assert L.coll_all_reduce(p, q, 65, 16, M.BF16, M.SUM, M.TWOSHOT, None, 0, None) == -1
+    assert L.coll_all_reduce(null, q, 4, 16, M.BF16, M.SUM, M.TWOSHOT, None, 0, None) == -1
+    assert L.coll_broadcast(p, 4, 16, M.BF16, 4, None) == -1
+    assert L.coll_broadcast(p, 4, 16, M.BF16, -1, None) == -1
+    assert L.coll_gather(p, BASE + 0x40000000, 4, 0, 16, M.FP32, 0, None) == -1
+    assert L.coll_reduce(p, BASE + 0x40000000, 4, 16, M.BF16, M.SUM, 7, None) == -1
+    # unsupported dtype / op / algo
+    assert L.coll_all_reduce(p, q, 4, 16, 9, M.SUM, M.TWOSHOT, None, 0, None) == -2
+    assert L.coll_all_reduce(p, q, 4, 16, M.BF16, 9, M.TWOSHOT, None, 0, None) == -2
+    assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, 9, None, 0, None) == -2
+    assert L.coll_moe_combine(p, p, p, p, q, 4, 8, 2, 8, 16, M.INT32, 100, None, None) == -2
+    # ring without workspace
+    assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, M.RING, None, 0, None) == -5
+    assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, M.RING, BASE + 0x50000000, 8, None) == -5
+    # packets: step 0, LL step with zero low word, misaligned packet buffer
+    assert L.coll_ll_pack(BASE, BASE + 0x100000, 64, M.LL, 0, None) == -1
+    assert L.coll_ll_pack(BASE, BASE + 0x100000, 64, M.LL, 1 << 32, None) == -1
+    assert L.coll_ll_pack(BASE, BASE + 0x100008, 64, M.LL128, 1, None) == -1
+    assert L.coll_ll_unpack(BASE, BASE + 0x100000, 64, M.LL, 0, None, None) == -1
+    assert L.coll_ll_pack(BASE, BASE + 0x100000, 64, 7, 1, None) == -2
+    assert L.coll_all_reduce_packed(p, q, 4, 16, M.BF16, M.SUM, M.LL128, 0, None, None) == -1
+    # MoE shapes
+    assert L.coll_moe_route(p, 4, 16, 0, 8, BASE, BASE, BASE, q, None, BASE, 1 << 20, None) == -1
+    assert L.coll_moe_route(p, 4, 16, 2, 6, BASE, BASE, BASE, q, None, BASE, 1 << 20, None) == -1
+    assert L.coll_moe_route(p, 4, 16, 2, 8, BASE, BASE, BASE, q, None, BASE, 16, None) == -5
+    assert L.coll_moe_route(p, 4, 16, 2, 8, BASE, BASE, BASE, q, None, BASE + 8, 1 << 20, None) == -5
+    # all-to-all-v: negative counts, overflowing a stated capacity
+    n = 2
+    cnt = np.array([1, 1, 1, 1], np.int64)
+    neg = np.array([1, -1, 1, 1], np.int64)
+    dsp = np.array([0, 1, 0, 1], np.int64)
+    cap = np.array([1, 1], np.int64)
+    P = ctypes.POINTER(ctypes.c_int64)
+    pp, _k4 = _arr([BASE, BASE + 0x1000])
+    qq, _k5 = _arr([BASE + 0x10000, BASE + 0x11000])
+    f = L.coll_all_to_all_v
+    assert f(pp, qq, n, neg.ctypes.data_as(P), dsp.ctypes.data_as(P), dsp.ctypes.data_as(P), None, None, 4, M.BF16, None) == -1
+    assert f(pp, qq, n, cnt.ctypes.data_as(P), dsp.ctypes.data_as(P), dsp.ctypes.data_as(P), cap.ctypes.data_as(P), None, 4, M.BF16, None) == -1
+    # two sources landing on the same receive rows
+    same = np.array([0, 0, 0, 0], np.int64)
+    assert f(pp, qq, n, cnt.ctypes.data_as(P), dsp.ctypes.data_as(P), same.ctypes.data_as(P), None, None, 4, M.BF16, None) == -3
+
+
+@no_gpu
+def test_alias_rules_on_host():
+    L = M.lib()
+    n, count = 4, 1024
+    b = 2 * count
+    send, _k1 = _arr([BASE + i * 0x100000 for i in range(n)])
+    # outputs overlapping each other
+    bad, _k2 = _arr([BASE + 0x10000000, BASE + 0x10000000 + b // 2, BASE + 0x10100000, BASE + 0x10200000])
+    assert L.coll_all_reduce(send, bad, n, count, M.BF16, M.SUM, M.TWOSHOT, None, 0, None) == -3
+    # an output overlapping another rank's input
+    cross, _k3 = _arr([BASE + 0x100000, BASE + 0x20000000, BASE + 0x20100000, BASE + 0x20200000])
+    assert L.coll_all_reduce(send, cross, n, count, M.BF16, M.SUM, M.TWOSHOT, None, 0, None) == -3
+    # in place is an error for one-shot
+    assert L.coll_all_reduce(send, send, n, count, M.BF16, M.SUM, M.ONESHOT, None, 0, None) == -3
+    # broadcast buffers must be disjoint
+    ov, _k4 = _arr([BASE, BASE + 16, BASE + 0x100000, BASE + 0x200000])
+    assert L.coll_broadcast(ov, n, count, M.BF16, 0, None) == -3
+    # reduce-scatter output inside another rank's input
+    rs_out, _k5 = _arr([BASE + 0x100000 + 8, BASE + 0x30000000, BASE + 0x30100000, BASE + 0x30200000])
+    assert L.coll_reduce_scatter(send, rs_out, n, count // n, M.BF16, M.SUM, None) == -3
+    # all-to-all input and output overlap
+    assert L.coll_all_to_all(send, send, n, count // n, M.BF16, None) == -3
+
+
+@no_gpu
+def test_zero_counts_are_noops_on_host():
+    L = M.lib()
+    p, _k = _arr([BASE + i * 0x100000 for i in range(4)])
+    q, _k2 = _arr([BASE + 0x10000000 + i * 0x100000 for i in range(4)])
+    assert L.coll_all_reduce(p, q, 4, 0, M.BF16, M.SUM, M.RING, None, 0, None) == 0
+    assert L.coll_broadcast(p, 4, 0, M.INT32, 1, None) == 0
+    assert L.coll_all_gather(p, q, 4, 0, M.BF16, None) == 0
+    assert L.coll_ll_pack(BASE, BASE + 0x100000, 0, M.LL, 1, None) == 0
+    # a single rank in place does nothing
+    assert L.coll_all_reduce(p, p, 1, 100, M.BF16, M.SUM, M.TWOSHOT, None, 0, None) == 0
+    assert L.coll_broadcast(p, 1, 100, M.BF16, 0, None) == 0
+
+
+def test_binding_rejects_cpu_tensors():
+    x = [torch.zeros(8, dtype=torch.bfloat16) for _ in range(2)]
+    with pytest.raises(ValueError):
+        M.coll_all_reduce(x, x)
+    with pytest.raises(ValueError):
+        M.coll_broadcast(x, 0)

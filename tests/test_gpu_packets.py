@@ -1,0 +1,178 @@
+"""GPU parity: LL / LL128 codecs and the packetised all-reduce vs the oracle.
+
+Packed bytes are compared bit for bit with the oracle's encoding; decode
+round-trips; corrupted flags are counted exactly in the device status (a
+host-made corruption: no kernel waits, so nothing can hang); the
+packetised all-reduce matches the oracle's and, once decoded, the Simple
+two-shot all-reduce.
+"""
+import numpy as np
+import pytest
+import torch
+
+import movement_virtual_rank_b200 as M
+import oracle
+import workloads as W
+from gpu_util import from_dev, need_gpu, status_tensor, to_dev
+
+pytestmark = pytest.mark.gpu
+SIZES = [1, 2, 3, 4, 5, 15, 16, 17, 31, 32, 33, 119, 120, 121, 239, 240, 241, 1000, 4097, 65536 + 12, 1 << 20]
+
+
+def u8(nbytes, salt):
+    return W.rng(W.W_MISC, 2, salt=salt).integers(0, 256, nbytes).astype(np.uint8)
+
+
+@pytest.mark.parametrize("proto", [M.LL, M.LL128])
+@pytest.mark.parametrize("nbytes", SIZES)
+@pytest.mark.parametrize("src_off", [0, 1, 8])
+def test_pack_unpack(proto, nbytes, src_off):
+    need_gpu()
+    msg = u8(nbytes, nbytes + src_off)
+    step = 0x1234_5678 + nbytes if proto == M.LL else (0xABCD << 40) + nbytes
+    raw = torch.zeros(nbytes + 64, dtype=torch.uint8, device="cuda")
+    src = raw[src_off:src_off + nbytes]
+    src.copy_(torch.from_numpy(msg).cuda())
+    pb = M.coll_packed_bytes(nbytes, proto)
+    packed = torch.full((pb + 32,), 0xEE, dtype=torch.uint8, device="cuda")
+    M.coll_ll_pack(src, packed[:pb], proto, step)
+    torch.cuda.synchronize()
+    assert np.array_equal(packed[:pb].cpu().numpy(), oracle.pack(msg, proto, step))
+    assert (packed[pb:] == 0xEE).all()
+    out_raw = torch.full((nbytes + 64,), 0x33, dtype=torch.uint8, device="cuda")
+    dst = out_raw[src_off + 3:src_off + 3 + nbytes]
+    st = status_tensor()
+    M.coll_ll_unpack(packed[:pb], dst, proto, step, status=st)
+    torch.cuda.synchronize()
+    assert np.array_equal(dst.cpu().numpy(), msg)
+    o = out_raw.cpu().numpy()
+    assert (o[:src_off + 3] == 0x33).all() and (o[src_off + 3 + nbytes:] == 0x33).all()
+    assert st.tolist() == [0, 0]
+
+
+@pytest.mark.parametrize("proto", [M.LL, M.LL128])
+def test_unpack_counts_bad_flags(proto):
+    """Lines whose flag differs from the step (a stale or torn packet) are
+    counted exactly; the kernel returns normally."""
+    need_gpu()
+    nbytes = 100003
+    msg = u8(nbytes, 1)
+    step = 41
+    packed_np = oracle.pack(msg, proto, step)
+    line = 8 if proto == M.LL else 128
+    flag_at = 4 if proto == M.LL else 120
+    nlines = packed_np.size // line
+    g = W.rng(W.W_MISC, 3, salt=proto)
+    lines = np.unique(g.integers(0, nlines, 57))
+    bad = packed_np.copy()
+    for L in lines:
+        bad[L * line + flag_at] ^= 0x40
+    packed = torch.from_numpy(bad).cuda()
+    dst = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    st = status_tensor()
+    M.coll_ll_unpack(packed, dst, proto, step, status=st)
+    torch.cuda.synchronize()
+    _, want_bad = oracle.unpack(bad, nbytes, proto, step)
+    assert want_bad == lines.size
+    assert st.tolist() == [M.DEV_FLAG_MISMATCH, lines.size]
+    assert np.array_equal(dst.cpu().numpy(), msg)  # data is still delivered
+    # a stale step fails every line
+    st.zero_()
+    M.coll_ll_unpack(torch.from_numpy(packed_np).cuda(), dst, proto, step + 1, status=st)
+    torch.cuda.synchronize()
+    assert st.tolist() == [M.DEV_FLAG_MISMATCH, nlines]
+
+
+@pytest.mark.parametrize("proto", [M.LL, M.LL128])
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("n", [1, 2, 3, 8])
+@pytest.mark.parametrize("count", [1, 2, 3, 59, 60, 61, 1000, 30001])
+def test_all_reduce_packed(proto, dtype, n, count):
+    need_gpu()
+    xs = W.ranks_values(W.W_LL_SWEEP, n, count, dtype, "uniform", salt=count)
+    step = 7
+    esize = 2 if dtype == "bf16" else 4
+    pin = [oracle.pack(x, proto, step) for x in xs]
+    want, want_bad = oracle.all_reduce_packed(pin, count, dtype, 0, proto, step)
+    dev_in = [torch.from_numpy(p).cuda() for p in pin]
+    dev_out = [torch.full_like(p, 0x99) for p in dev_in]
+    st = status_tensor()
+    M.coll_all_reduce_packed(dev_in, dev_out, count, torch.bfloat16 if dtype == "bf16" else torch.float32,
+                             proto, step, status=st)
+    torch.cuda.synchronize()
+    assert st.tolist() == [0, 0] and want_bad == 0
+    for q in range(n):
+        assert np.array_equal(dev_out[q].cpu().numpy(), want[q]), q
+    # decoded, it equals the Simple (two-shot) all-reduce
+    simple = oracle.all_reduce_two_shot(xs, 0, dtype)
+    data, _ = oracle.unpack(want[0], count * esize, proto, step)
+    assert np.array_equal(data.view(simple[0].dtype), simple[0])
+
+
+@pytest.mark.parametrize("proto", [M.LL, M.LL128])
+def test_all_reduce_packed_in_place_and_bad_flags(proto):
+    need_gpu()
+    n, count = 4, 5000
+    xs = W.ranks_values(W.W_LL_SWEEP, n, count, "bf16", "uniform", salt=3)
+    step = 3
+    pin = [oracle.pack(x, proto, step) for x in xs]
+    line = 8 if proto == M.LL else 128
+    flag_at = 4 if proto == M.LL else 120
+    pin[2][5 * line + flag_at] ^= 1  # one stale line on rank 2
+    want, want_bad = oracle.all_reduce_packed(pin, count, "bf16", 0, proto, step)
+    dev = [torch.from_numpy(p).cuda() for p in pin]
+    st = status_tensor()
+    M.coll_all_reduce_packed(dev, dev, count, torch.bfloat16, proto, step, status=st)
+    torch.cuda.synchronize()
+    assert want_bad == 1 and st.tolist() == [M.DEV_FLAG_MISMATCH, 1]
+    for q in range(n):
+        assert np.array_equal(dev[q].cpu().numpy(), want[q])
+
+
+@pytest.mark.parametrize("log2", [10, 16, 20, 24, 28])
+def test_ll_sweep_sizes_sampled(log2):
+    """The LL / LL128 sweep sizes (8 ranks, 1 KB .. 256 MB per rank): packed
+    output compared in full on the device with the packed Simple result, and
+    4096 sampled lines against the oracle's encoding."""
+    need_gpu()
+    n, nbytes = 8, 1 << log2
+    count = nbytes // 2
+    xs = W.ll_message(nbytes, n)
+    send = [to_dev(x, "bf16") for x in xs]
+    simple = [torch.empty_like(t) for t in send]
+    M.coll_all_reduce(send, simple, algo=M.TWOSHOT)
+    for proto in (M.LL, M.LL128):
+        step = log2 + 1
+        pb = M.coll_packed_bytes(nbytes, proto)
+        packed = [torch.empty(pb, dtype=torch.uint8, device="cuda") for _ in range(n)]
+        for r in range(n):
+            M.coll_ll_pack(send[r], packed[r], proto, step)
+        out = [torch.empty(pb, dtype=torch.uint8, device="cuda") for _ in range(n)]
+        st = status_tensor()
+        M.coll_all_reduce_packed(packed, out, count, torch.bfloat16, proto, step, status=st)
+        ref = torch.empty(pb, dtype=torch.uint8, device="cuda")
+        M.coll_ll_pack(simple[0], ref, proto, step)
+        dec = torch.empty_like(send[0])
+        M.coll_ll_unpack(out[3], dec, proto, step, status=st)
+        torch.cuda.synchronize()
+        assert st.tolist() == [0, 0]
+        for q in range(n):
+            assert torch.equal(out[q], ref)
+        assert torch.equal(dec.view(torch.int16), simple[0].view(torch.int16))
+        line = 8 if proto == M.LL else 128
+        nl = pb // line
+        g = W.rng(W.W_MISC, 4, salt=log2 + proto)
+        lines = np.unique(g.integers(0, nl, 4096))
+        want_full = oracle.all_reduce_two_shot([x for x in xs], 0, "bf16")[0] if log2 <= 20 else None
+        host = out[0].cpu().numpy().reshape(nl, line)
+        if want_full is not None:
+            enc = oracle.pack(want_full, proto, step).reshape(nl, line)
+            assert np.array_equal(host[lines], enc[lines])
+        else:  # oracle on the sampled lines only
+            per = 4 if proto == M.LL else 120
+            for L in lines[:256]:
+                lo, hi = L * per // 2, min(count, (L + 1) * per // 2)
+                red = oracle.reduce([x[lo:hi] for x in xs], 0, "bf16")
+                seg = np.zeros(per // 2, np.uint16)
+                seg[:hi - lo] = red
+                assert np.array_equal(host[L, :per].view(np.uint16), seg)
