@@ -390,17 +390,49 @@ def time_oracle(ops, min_s: float = 10.0, max_s: float = 30.0):
     return (nbytes / secs / 1e9 if secs > 0 else None), sample, secs
 
 
+def graph_latency(ops, stream, reps: int = 50, max_bytes_per_rank: int = 256 * 1024):
+    """Latency floor of the small ops: ``reps`` back-to-back calls captured in
+    one CUDA graph (no host launch cost, L2 warm), device time per call."""
+    import torch
+    out = {}
+    for op in ops:
+        if op.meta.get("bytes_per_rank", 1 << 62) > max_bytes_per_rank:
+            continue
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            op.run()  # warm the call path on the capture stream
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                op.run()
+        for _ in range(3):
+            g.replay()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        out[id(op)] = round(a.elapsed_time(b) * 1e3 / reps, 3)
+        del g
+    return out
+
+
 # ------------------------------------------------------------------ main ----
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="tp_decode", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--lead-us", type=float, default=300.0, help="sleep before each timed op (outside the events)")
     args = ap.parse_args()
     rank, world, local = dist_env()
 
@@ -423,9 +455,16 @@ def main():
     evs = {id(op): [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                     for _ in range(args.steps)] for op in ops}
 
+    # Lead time: a bounded sleep kernel between the flush and the start event
+    # keeps the GPU busy while the host enqueues the op, so the events time
+    # the op's kernels back to back on the device, not the host's launch path
+    # (that path is in the end-to-end number).
+    lead_cycles = int(args.lead_us * 1e-6 * torch.cuda.get_device_properties(local).clock_rate * 1e3)
+
     def one_step(timed_index=None):
         for op in ops:
             flush.zero_()
+            torch.cuda._sleep(lead_cycles)
             if timed_index is None:
                 op.run()
             else:
@@ -434,19 +473,21 @@ def main():
                 op.run()
                 b.record(stream)
 
-    for _ in range(max(args.warmup, 3)):
-        one_step()
-    torch.cuda.synchronize()
-    barrier(world)
     with Clocks(local) as clk:
+        time.sleep(0.5)  # let the sampler start
+        for _ in range(max(args.warmup, 3)):
+            one_step()
+        torch.cuda.synchronize()
+        barrier(world)
         torch.cuda.synchronize()
         wall0 = time.perf_counter()
         for k in range(args.steps):
             one_step(k)
         torch.cuda.synchronize()
         wall = time.perf_counter() - wall0
-    barrier(world)
+        barrier(world)
     clocks = clk.summary()
+    graph_us = graph_latency(ops, stream) if not args.no_graph else {}
     for op in ops:
         op.times = [a.elapsed_time(b) * 1e-3 for a, b in evs[id(op)]]
     step_s = [sum(op.times[k] for op in ops) for k in range(args.steps)]
@@ -488,7 +529,8 @@ def main():
     for op in ops:
         med = statistics.median(op.times)
         gbs = op.alg_bytes / med / 1e9
-        per_op.append({**op.meta, "us": round(med * 1e6, 3), "us_p10": round(np.percentile(op.times, 10) * 1e6, 3),
+        extra = {"graph_us": graph_us[id(op)]} if id(op) in graph_us else {}
+        per_op.append({**op.meta, **extra, "us": round(med * 1e6, 3), "us_p10": round(np.percentile(op.times, 10) * 1e6, 3),
                        "us_p90": round(np.percentile(op.times, 90) * 1e6, 3), "gbs": round(gbs, 1),
                        "frac_measured_hbm": round(gbs / hbm, 4), "frac_8tbs": round(gbs / 8000, 4)})
         k = by_kernel.setdefault(op.kernel, {"time": 0.0, "bytes": 0, "launches": 0, "ops": 0})
@@ -521,7 +563,9 @@ def main():
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic", "impl": "ours",
                 "config": {**cfg, "parallelism": f"replicas x{world} (virtual ranks inside each GPU)",
-                           "l2": "flushed before every op (memset of 2x L2, outside the timed events)"},
+                           "l2": "flushed before every op (memset of 2x L2, outside the timed events)",
+                           "timing": f"CUDA events around each op on its stream, after a {args.lead_us:.0f} us "
+                                     "sleep kernel so the op's kernels run back to back"},
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
                 "clocks": clocks, "wall_s_timed_region": round(wall, 3), "ops": per_op}
         print(json.dumps(line), flush=True)

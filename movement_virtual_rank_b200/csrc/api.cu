@@ -550,9 +550,10 @@ int coll_moe_route(const int32_t* const* topk_ids, int nranks, int tokens, int t
                    int64_t* d_send_counts, int64_t* d_send_displs, int64_t* d_recv_displs, int32_t* const* d_pos,
                    int* d_status, void* workspace, size_t workspace_bytes, coll_stream_t stream) {
   if (!moe_shape_ok(nranks, tokens, topk, n_experts)) return COLL_ERR_INVALID_ARG;
-  if (!all_nonnull(topk_ids, nranks) || !all_nonnull(d_pos, nranks) || !d_send_counts || !d_send_displs ||
-      !d_recv_displs)
+  if (topk_ids == nullptr || d_pos == nullptr || !d_send_counts || !d_send_displs || !d_recv_displs)
     return COLL_ERR_INVALID_ARG;
+  // with no tokens the per-rank arrays are empty and never touched
+  if (tokens > 0 && (!all_nonnull(topk_ids, nranks) || !all_nonnull(d_pos, nranks))) return COLL_ERR_INVALID_ARG;
   const size_t need = moe_route_workspace(nranks, tokens, topk, n_experts);
   if (workspace == nullptr || workspace_bytes < need || (U(workspace) & 255) != 0) return COLL_ERR_WORKSPACE;
   MoeRouteArgs a{};

@@ -11,6 +11,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "coll.h"
 #include "internal.h"
 
@@ -222,6 +224,32 @@ __device__ __forceinline__ typename UnitT<U>::T ldu(const char* p) {
 template <int U>
 __device__ __forceinline__ void stu(char* p, const typename UnitT<U>::T& v) {
   *reinterpret_cast<typename UnitT<U>::T*>(p) = v;
+}
+
+// ------------------------------------------- programmatic dependent launch ----
+// Every kernel is launched with programmatic stream serialisation allowed, so
+// the hardware may schedule its CTAs while the previous kernel in the stream
+// is still draining.  pdl_wait() (griddepcontrol.wait) blocks until that
+// predecessor has completed and its memory is visible, and is the first thing
+// every kernel does; it returns at once when there is no such predecessor.
+// pdl_trigger() lets the next kernel in the stream start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // ------------------------------------------------------ device status ----

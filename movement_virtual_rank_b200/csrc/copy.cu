@@ -40,6 +40,8 @@ static unsigned grid_for(uint64_t units, int slices) {
 
 template <int U>
 __global__ void __launch_bounds__(kThreads) k_fanout(const __grid_constant__ FanoutArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x % a.ns;
   const int part = blockIdx.x / a.ns;
   const int parts = gridDim.x / a.ns;
@@ -75,11 +77,11 @@ int launch_fanout(const FanoutArgs& a, cudaStream_t s) {
   const int U = pick_unit(bits);
   const unsigned grid = grid_for(a.bytes / U, a.ns);
   switch (U) {
-    case 16: k_fanout<16><<<grid, kThreads, 0, s>>>(a); break;
-    case 8: k_fanout<8><<<grid, kThreads, 0, s>>>(a); break;
-    case 4: k_fanout<4><<<grid, kThreads, 0, s>>>(a); break;
-    case 2: k_fanout<2><<<grid, kThreads, 0, s>>>(a); break;
-    default: k_fanout<1><<<grid, kThreads, 0, s>>>(a); break;
+    case 16: launch_pdl(k_fanout<16>, dim3(grid), dim3(kThreads), 0, s, a); break;
+    case 8: launch_pdl(k_fanout<8>, dim3(grid), dim3(kThreads), 0, s, a); break;
+    case 4: launch_pdl(k_fanout<4>, dim3(grid), dim3(kThreads), 0, s, a); break;
+    case 2: launch_pdl(k_fanout<2>, dim3(grid), dim3(kThreads), 0, s, a); break;
+    default: launch_pdl(k_fanout<1>, dim3(grid), dim3(kThreads), 0, s, a); break;
   }
   return launch_status(cudaGetLastError());
 }
@@ -100,6 +102,8 @@ struct CopyJobsArgs {
 
 template <int U>
 __global__ void __launch_bounds__(kThreads) k_copy_jobs(const __grid_constant__ CopyJobsArgs a) {
+  pdl_wait();
+  pdl_trigger();
   // block b owns the contiguous unit range [b*total/B, (b+1)*total/B)
   const uint64_t B = gridDim.x;
   const uint64_t lo = a.total * blockIdx.x / B;
@@ -147,15 +151,15 @@ int launch_copy_jobs(const CopyJob* jobs, int njobs, cudaStream_t s) {
     args.job[nj].start = acc;
     args.total = acc;
     args.njobs = nj;
-    uint64_t want = (acc + 4ull * kThreads - 1) / (4ull * kThreads);
+    uint64_t want = (acc + kThreads - 1) / kThreads;  // about one unit per thread: latency first
     want = std::min<uint64_t>(std::max<uint64_t>(want, 1), static_cast<uint64_t>(num_sms()) * 8);
     const unsigned grid = static_cast<unsigned>(want);
     switch (U) {
-      case 16: k_copy_jobs<16><<<grid, kThreads, 0, s>>>(args); break;
-      case 8: k_copy_jobs<8><<<grid, kThreads, 0, s>>>(args); break;
-      case 4: k_copy_jobs<4><<<grid, kThreads, 0, s>>>(args); break;
-      case 2: k_copy_jobs<2><<<grid, kThreads, 0, s>>>(args); break;
-      default: k_copy_jobs<1><<<grid, kThreads, 0, s>>>(args); break;
+      case 16: launch_pdl(k_copy_jobs<16>, dim3(grid), dim3(kThreads), 0, s, args); break;
+      case 8: launch_pdl(k_copy_jobs<8>, dim3(grid), dim3(kThreads), 0, s, args); break;
+      case 4: launch_pdl(k_copy_jobs<4>, dim3(grid), dim3(kThreads), 0, s, args); break;
+      case 2: launch_pdl(k_copy_jobs<2>, dim3(grid), dim3(kThreads), 0, s, args); break;
+      default: launch_pdl(k_copy_jobs<1>, dim3(grid), dim3(kThreads), 0, s, args); break;
     }
     const int st = launch_status(cudaGetLastError());
     if (st != COLL_OK) return st;
@@ -167,6 +171,8 @@ int launch_copy_jobs(const CopyJob* jobs, int njobs, cudaStream_t s) {
 
 template <int U>
 __global__ void __launch_bounds__(kThreads) k_gather_rows(const __grid_constant__ GatherRowsArgs a) {
+  pdl_wait();
+  pdl_trigger();
   // blockIdx.x = part * n + r ; parts stride over rows, threads over columns
   const int r = blockIdx.x % a.n;
   const int part = blockIdx.x / a.n;
@@ -190,11 +196,11 @@ int launch_gather_rows(const GatherRowsArgs& a, cudaStream_t s) {
   uint64_t parts = std::min<uint64_t>(a.rows, std::max<uint64_t>(1, static_cast<uint64_t>(num_sms()) * 8 / a.n));
   const unsigned grid = static_cast<unsigned>(parts * a.n);
   switch (U) {
-    case 16: k_gather_rows<16><<<grid, kThreads, 0, s>>>(a); break;
-    case 8: k_gather_rows<8><<<grid, kThreads, 0, s>>>(a); break;
-    case 4: k_gather_rows<4><<<grid, kThreads, 0, s>>>(a); break;
-    case 2: k_gather_rows<2><<<grid, kThreads, 0, s>>>(a); break;
-    default: k_gather_rows<1><<<grid, kThreads, 0, s>>>(a); break;
+    case 16: launch_pdl(k_gather_rows<16>, dim3(grid), dim3(kThreads), 0, s, a); break;
+    case 8: launch_pdl(k_gather_rows<8>, dim3(grid), dim3(kThreads), 0, s, a); break;
+    case 4: launch_pdl(k_gather_rows<4>, dim3(grid), dim3(kThreads), 0, s, a); break;
+    case 2: launch_pdl(k_gather_rows<2>, dim3(grid), dim3(kThreads), 0, s, a); break;
+    default: launch_pdl(k_gather_rows<1>, dim3(grid), dim3(kThreads), 0, s, a); break;
   }
   return launch_status(cudaGetLastError());
 }

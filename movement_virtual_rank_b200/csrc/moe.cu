@@ -40,6 +40,8 @@ size_t moe_route_workspace(int n, int tokens, int topk, int n_experts) {
 }
 
 __global__ void __launch_bounds__(kTile) k_moe_count(const __grid_constant__ MoeRouteArgs a) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint32_t bits[];  // [n_experts][kWords]
   const int s = blockIdx.x / a.tiles;
   const int tile = blockIdx.x % a.tiles;
@@ -87,6 +89,8 @@ __global__ void __launch_bounds__(kTile) k_moe_count(const __grid_constant__ Moe
 constexpr int kScanThreads = 1024;
 
 __global__ void __launch_bounds__(kScanThreads) k_moe_scan(const __grid_constant__ MoeRouteArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int64_t warp_sums[kScanThreads / 32];
   const int s = blockIdx.x;
   const int64_t m = static_cast<int64_t>(a.n_experts) * a.tiles;  // cells of this source
@@ -141,6 +145,8 @@ __global__ void __launch_bounds__(kScanThreads) k_moe_scan(const __grid_constant
 }
 
 __global__ void __launch_bounds__(kTile) k_moe_pos(const __grid_constant__ MoeRouteArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int64_t rdispl[kMaxRanks];  // recv_displs[d][s] for this block's s
   __shared__ int64_t sdispl[kMaxRanks];  // send_displs[s][d]
   const int s = blockIdx.x / a.tiles;
@@ -186,13 +192,13 @@ int launch_moe_route(const MoeRouteArgs& a, cudaStream_t s) {
                                                static_cast<int>(smem));
     if (e != cudaSuccess) return launch_status(e);
   }
-  k_moe_count<<<grid, kTile, smem, s>>>(a);  // tokens == 0 still zeroes the counts
+  launch_pdl(k_moe_count, dim3(grid), dim3(kTile), smem, s, a);  // tokens == 0 still zeroes the counts
   int st = launch_status(cudaGetLastError());
   if (st != COLL_OK) return st;
-  k_moe_scan<<<a.n, kScanThreads, 0, s>>>(a);
+  launch_pdl(k_moe_scan, dim3(a.n), dim3(kScanThreads), 0, s, a);
   st = launch_status(cudaGetLastError());
   if (st != COLL_OK) return st;
-  k_moe_pos<<<std::max(grid, 1u), kTile, 0, s>>>(a);
+  launch_pdl(k_moe_pos, dim3(std::max(grid, 1u)), dim3(kTile), 0, s, a);
   return launch_status(cudaGetLastError());
 }
 
@@ -204,6 +210,8 @@ struct RowTargets {
 
 template <int U>
 __global__ void __launch_bounds__(kMoveThreads) k_moe_dispatch(const __grid_constant__ MoeMoveArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ char* dst[kMaxTopk];
   __shared__ int nbad;
   const int64_t rows = static_cast<int64_t>(a.n) * a.tokens;
@@ -262,11 +270,11 @@ int launch_moe_dispatch(const MoeMoveArgs& a, cudaStream_t s) {
   for (int r = 0; r < a.n; ++r) bits |= reinterpret_cast<uintptr_t>(a.x[r]) | reinterpret_cast<uintptr_t>(a.y[r]);
   const unsigned grid = move_grid(rows);
   switch (pick_unit(bits)) {
-    case 16: k_moe_dispatch<16><<<grid, kMoveThreads, 0, s>>>(a); break;
-    case 8: k_moe_dispatch<8><<<grid, kMoveThreads, 0, s>>>(a); break;
-    case 4: k_moe_dispatch<4><<<grid, kMoveThreads, 0, s>>>(a); break;
-    case 2: k_moe_dispatch<2><<<grid, kMoveThreads, 0, s>>>(a); break;
-    default: k_moe_dispatch<1><<<grid, kMoveThreads, 0, s>>>(a); break;
+    case 16: launch_pdl(k_moe_dispatch<16>, dim3(grid), dim3(kMoveThreads), 0, s, a); break;
+    case 8: launch_pdl(k_moe_dispatch<8>, dim3(grid), dim3(kMoveThreads), 0, s, a); break;
+    case 4: launch_pdl(k_moe_dispatch<4>, dim3(grid), dim3(kMoveThreads), 0, s, a); break;
+    case 2: launch_pdl(k_moe_dispatch<2>, dim3(grid), dim3(kMoveThreads), 0, s, a); break;
+    default: launch_pdl(k_moe_dispatch<1>, dim3(grid), dim3(kMoveThreads), 0, s, a); break;
   }
   return launch_status(cudaGetLastError());
 }
@@ -275,6 +283,8 @@ int launch_moe_dispatch(const MoeMoveArgs& a, cudaStream_t s) {
 
 template <int DT, bool VEC>
 __global__ void __launch_bounds__(kMoveThreads) k_moe_combine(const __grid_constant__ MoeMoveArgs a) {
+  pdl_wait();
+  pdl_trigger();
   using S = typename Elem<DT>::S;
   constexpr int VN = Vec<DT>::kN;
   constexpr int ES = Elem<DT>::kSize;
@@ -344,8 +354,8 @@ static int launch_combine_dt(const MoeMoveArgs& a, cudaStream_t s) {
   uint64_t bits = a.row_bytes;
   for (int r = 0; r < a.n; ++r) bits |= reinterpret_cast<uintptr_t>(a.x[r]) | reinterpret_cast<uintptr_t>(a.y[r]);
   const unsigned grid = move_grid(rows);
-  if ((bits & 15) == 0) k_moe_combine<DT, true><<<grid, kMoveThreads, 0, s>>>(a);
-  else k_moe_combine<DT, false><<<grid, kMoveThreads, 0, s>>>(a);
+  if ((bits & 15) == 0) launch_pdl(k_moe_combine<DT, true>, dim3(grid), dim3(kMoveThreads), 0, s, a);
+  else launch_pdl(k_moe_combine<DT, false>, dim3(grid), dim3(kMoveThreads), 0, s, a);
   return launch_status(cudaGetLastError());
 }
 

@@ -54,6 +54,8 @@ __device__ __forceinline__ void store8_any(uint8_t* dst, uint64_t off, uint64_t 
 
 __global__ void __launch_bounds__(kThreads) k_ll_pack(const uint8_t* __restrict__ src, uint8_t* __restrict__ packed,
                                                       uint64_t bytes, uint32_t flag, int src_al16) {
+  pdl_wait();
+  pdl_trigger();
   const uint64_t nlines = (bytes + 3) / 4;
   const uint64_t ngroups = nlines / 4;  // groups of 4 lines = 16 message bytes
   const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
@@ -78,6 +80,8 @@ __global__ void __launch_bounds__(kThreads) k_ll_pack(const uint8_t* __restrict_
 
 __global__ void __launch_bounds__(kThreads) k_ll_unpack(const uint8_t* __restrict__ packed, uint8_t* __restrict__ dst,
                                                         uint64_t bytes, uint32_t flag, int dst_al16, int* status) {
+  pdl_wait();
+  pdl_trigger();
   const uint64_t nlines = (bytes + 3) / 4;
   const uint64_t ngroups = nlines / 4;
   const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
@@ -108,6 +112,8 @@ __global__ void __launch_bounds__(kThreads) k_ll_unpack(const uint8_t* __restric
 
 __global__ void __launch_bounds__(kThreads) k_ll128_pack(const uint8_t* __restrict__ src, uint8_t* __restrict__ packed,
                                                          uint64_t bytes, uint64_t step, int src_al8) {
+  pdl_wait();
+  pdl_trigger();
   const uint64_t nlines = (bytes + 119) / 120;
   const uint64_t nthreads = nlines * 8;
   const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
@@ -125,6 +131,8 @@ __global__ void __launch_bounds__(kThreads) k_ll128_pack(const uint8_t* __restri
 
 __global__ void __launch_bounds__(kThreads) k_ll128_unpack(const uint8_t* __restrict__ packed, uint8_t* __restrict__ dst,
                                                            uint64_t bytes, uint64_t step, int dst_al8, int* status) {
+  pdl_wait();
+  pdl_trigger();
   const uint64_t nlines = (bytes + 119) / 120;
   const uint64_t nthreads = nlines * 8;
   const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
@@ -151,11 +159,11 @@ int launch_ll_pack(const void* src, void* packed, size_t bytes, int proto, uint6
   auto* pp = static_cast<uint8_t*>(packed);
   if (proto == COLL_PROTO_LL) {
     const uint64_t nlines = (bytes + 3) / 4;
-    k_ll_pack<<<grid_units(nlines / 4 + 1), kThreads, 0, s>>>(sp, pp, bytes, static_cast<uint32_t>(step),
+    launch_pdl(k_ll_pack, dim3(grid_units(nlines / 4 + 1)), dim3(kThreads), 0, s, sp, pp, bytes, static_cast<uint32_t>(step),
                                                                (reinterpret_cast<uintptr_t>(src) & 15) == 0);
   } else {
     const uint64_t nlines = (bytes + 119) / 120;
-    k_ll128_pack<<<grid_units(nlines * 8), kThreads, 0, s>>>(sp, pp, bytes, step,
+    launch_pdl(k_ll128_pack, dim3(grid_units(nlines * 8)), dim3(kThreads), 0, s, sp, pp, bytes, step,
                                                               (reinterpret_cast<uintptr_t>(src) & 7) == 0);
   }
   return launch_status(cudaGetLastError());
@@ -168,11 +176,11 @@ int launch_ll_unpack(const void* packed, void* dst, size_t bytes, int proto, uin
   auto* dp = static_cast<uint8_t*>(dst);
   if (proto == COLL_PROTO_LL) {
     const uint64_t nlines = (bytes + 3) / 4;
-    k_ll_unpack<<<grid_units(nlines / 4 + 1), kThreads, 0, s>>>(pp, dp, bytes, static_cast<uint32_t>(step),
+    launch_pdl(k_ll_unpack, dim3(grid_units(nlines / 4 + 1)), dim3(kThreads), 0, s, pp, dp, bytes, static_cast<uint32_t>(step),
                                                                  (reinterpret_cast<uintptr_t>(dst) & 15) == 0, status);
   } else {
     const uint64_t nlines = (bytes + 119) / 120;
-    k_ll128_unpack<<<grid_units(nlines * 8), kThreads, 0, s>>>(pp, dp, bytes, step,
+    launch_pdl(k_ll128_unpack, dim3(grid_units(nlines * 8)), dim3(kThreads), 0, s, pp, dp, bytes, step,
                                                                 (reinterpret_cast<uintptr_t>(dst) & 7) == 0, status);
   }
   return launch_status(cudaGetLastError());
@@ -214,6 +222,8 @@ struct WordOps {
 // LL: thread = one 8-byte line per rank when `single`, else two lines (16 B)
 template <int DT, int OP>
 __global__ void __launch_bounds__(kThreads) k_ar_ll(const __grid_constant__ PackedReduceArgs a) {
+  pdl_wait();
+  pdl_trigger();
   using W = WordOps<DT, OP>;
   using A = typename Elem<DT>::A;
   constexpr int kE = W::kE;
@@ -259,6 +269,8 @@ __global__ void __launch_bounds__(kThreads) k_ar_ll(const __grid_constant__ Pack
 // LL128: eight threads per line, thread j owns packet bytes [16j, 16j+16)
 template <int DT, int OP>
 __global__ void __launch_bounds__(kThreads) k_ar_ll128(const __grid_constant__ PackedReduceArgs a) {
+  pdl_wait();
+  pdl_trigger();
   using W = WordOps<DT, OP>;
   using A = typename Elem<DT>::A;
   constexpr int kE = W::kE;
@@ -304,8 +316,8 @@ __global__ void __launch_bounds__(kThreads) k_ar_ll128(const __grid_constant__ P
 
 template <int DT, int OP>
 static int launch_ar_packed_t(const PackedReduceArgs& a, int proto, cudaStream_t s) {
-  if (proto == COLL_PROTO_LL) k_ar_ll<DT, OP><<<grid_units(a.nlines / 2 + 1), kThreads, 0, s>>>(a);
-  else k_ar_ll128<DT, OP><<<grid_units(a.nlines * 8), kThreads, 0, s>>>(a);
+  if (proto == COLL_PROTO_LL) launch_pdl(k_ar_ll<DT, OP>, dim3(grid_units(a.nlines / 2 + 1)), dim3(kThreads), 0, s, a);
+  else launch_pdl(k_ar_ll128<DT, OP>, dim3(grid_units(a.nlines * 8)), dim3(kThreads), 0, s, a);
   return launch_status(cudaGetLastError());
 }
 

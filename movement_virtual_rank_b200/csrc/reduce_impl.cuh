@@ -61,6 +61,8 @@ __device__ __forceinline__ void slice_range(const ReduceArgs& a, int slice, uint
 
 template <int DT, int OP, int NR, int MODE>
 __global__ void __launch_bounds__(kThreads) k_reduce_vec(const __grid_constant__ ReduceArgs a) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int VN = Vec<DT>::kN;
   constexpr int ES = Elem<DT>::kSize;
   const int n = NR > 0 ? NR : a.nin;
@@ -103,6 +105,8 @@ __global__ void __launch_bounds__(kThreads) k_reduce_vec(const __grid_constant__
 
 template <int DT, int OP, int MODE>
 __global__ void __launch_bounds__(kThreads) k_reduce_scalar(const __grid_constant__ ReduceArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int slice = blockIdx.x % a.nslices;
   const int part = blockIdx.x / a.nslices;
   const int parts = gridDim.x / a.nslices;
@@ -120,6 +124,8 @@ __global__ void __launch_bounds__(kThreads) k_reduce_scalar(const __grid_constan
 // writes the finished chunk to rank c's output.
 template <int DT, int OP, bool VEC>
 __global__ void __launch_bounds__(kThreads) k_ring_rs(const __grid_constant__ RingStepArgs a) {
+  pdl_wait();
+  pdl_trigger();
   using A = typename Elem<DT>::A;
   using S = typename Elem<DT>::S;
   constexpr int VN = Vec<DT>::kN;
@@ -195,17 +201,17 @@ int launch_reduce_nr(const ReduceArgs& a, int mode, bool vec, int bps, cudaStrea
   const dim3 grid(static_cast<unsigned>(a.nslices * bps));
   if (vec) {
     switch (mode) {
-      case M_ALL: k_reduce_vec<DT, OP, NR, M_ALL><<<grid, kThreads, 0, s>>>(a); break;
-      case M_BLOCK: k_reduce_vec<DT, OP, NR, M_BLOCK><<<grid, kThreads, 0, s>>>(a); break;
-      case M_SAME: k_reduce_vec<DT, OP, NR, M_SAME><<<grid, kThreads, 0, s>>>(a); break;
-      default: k_reduce_vec<DT, OP, NR, M_ONESHOT><<<grid, kThreads, 0, s>>>(a); break;
+      case M_ALL: launch_pdl(k_reduce_vec<DT, OP, NR, M_ALL>, dim3(grid), dim3(kThreads), 0, s, a); break;
+      case M_BLOCK: launch_pdl(k_reduce_vec<DT, OP, NR, M_BLOCK>, dim3(grid), dim3(kThreads), 0, s, a); break;
+      case M_SAME: launch_pdl(k_reduce_vec<DT, OP, NR, M_SAME>, dim3(grid), dim3(kThreads), 0, s, a); break;
+      default: launch_pdl(k_reduce_vec<DT, OP, NR, M_ONESHOT>, dim3(grid), dim3(kThreads), 0, s, a); break;
     }
   } else {
     switch (mode) {
-      case M_ALL: k_reduce_scalar<DT, OP, M_ALL><<<grid, kThreads, 0, s>>>(a); break;
-      case M_BLOCK: k_reduce_scalar<DT, OP, M_BLOCK><<<grid, kThreads, 0, s>>>(a); break;
-      case M_SAME: k_reduce_scalar<DT, OP, M_SAME><<<grid, kThreads, 0, s>>>(a); break;
-      default: k_reduce_scalar<DT, OP, M_ONESHOT><<<grid, kThreads, 0, s>>>(a); break;
+      case M_ALL: launch_pdl(k_reduce_scalar<DT, OP, M_ALL>, dim3(grid), dim3(kThreads), 0, s, a); break;
+      case M_BLOCK: launch_pdl(k_reduce_scalar<DT, OP, M_BLOCK>, dim3(grid), dim3(kThreads), 0, s, a); break;
+      case M_SAME: launch_pdl(k_reduce_scalar<DT, OP, M_SAME>, dim3(grid), dim3(kThreads), 0, s, a); break;
+      default: launch_pdl(k_reduce_scalar<DT, OP, M_ONESHOT>, dim3(grid), dim3(kThreads), 0, s, a); break;
     }
   }
   return launch_status(cudaGetLastError());
@@ -240,8 +246,8 @@ int launch_ring_op(const RingStepArgs& a, bool vec, cudaStream_t s) {
   if (want > cap) want = cap;
   if (want < 1) want = 1;
   const dim3 grid(static_cast<unsigned>(a.n * want));
-  if (vec) k_ring_rs<DT, OP, true><<<grid, kThreads, 0, s>>>(a);
-  else k_ring_rs<DT, OP, false><<<grid, kThreads, 0, s>>>(a);
+  if (vec) launch_pdl(k_ring_rs<DT, OP, true>, dim3(grid), dim3(kThreads), 0, s, a);
+  else launch_pdl(k_ring_rs<DT, OP, false>, dim3(grid), dim3(kThreads), 0, s, a);
   return launch_status(cudaGetLastError());
 }
 

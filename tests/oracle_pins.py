@@ -130,6 +130,11 @@ def pin_sum_order_and_single_rounding():
     assert int(oracle.reduce_ranks([big, big], SUM, "bf16")[0]) == 0x7F80
     inf, ninf = bf16([np.inf]), bf16([-np.inf])
     assert int(oracle.reduce_ranks([inf, ninf], SUM, "bf16")[0]) == 0x7FC0
+    # fp32 storage: every NaN result is the canonical quiet NaN 0x7FC00000
+    f_inf, f_ninf = np.array([np.inf], np.float32), np.array([-np.inf], np.float32)
+    assert int(oracle.reduce_ranks([f_inf, f_ninf], SUM, "fp32").view(np.uint32)[0]) == 0x7FC00000
+    neg_nan = np.array([0xFFC12345], np.uint32).view(np.float32)
+    assert int(oracle.reduce_ranks([neg_nan, f_inf], MAX, "fp32").view(np.uint32)[0]) == 0x7FC00000
 
 
 def pin_maxmin():

@@ -122,12 +122,11 @@ def test_bad_routes_and_overflow_are_reported():
     assert st.tolist() == [M.DEV_BAD_ROUTE, 2]  # a repeated expert on rank 0, an id beyond range on rank 1
     good = [np.array([[0, 1], [2, 3]], np.int32), np.array([[0, 2], [1, 3]], np.int32)]
     dids, sc, sd, rd, pos, st = route_on_device(good, experts)
-    x = [to_dev(np.arange(8, dtype=np.uint16), "bf16") for _ in range(n)]
-    recv = [torch.zeros(4, dtype=torch.bfloat16, device="cuda") for _ in range(n)]  # 2 rows, 4 needed
+    x = [to_dev(np.arange(8, dtype=np.uint16), "bf16") for _ in range(n)]  # 2 tokens of hidden 4
+    recv = [torch.zeros(8, dtype=torch.bfloat16, device="cuda") for _ in range(n)]  # 2 rows, 4 needed
     M.coll_moe_dispatch(x, dids, pos, recv, experts, status=st)
     torch.cuda.synchronize()
-    code, cnt = st.tolist()
-    assert code == M.DEV_SPLIT_OVERFLOW and cnt == 4
+    assert st.tolist() == [M.DEV_SPLIT_OVERFLOW, 4]  # rows 2 and 3 of both destinations
 
 
 def test_moe_workload():

@@ -42,8 +42,15 @@ def run_all_reduce(xs, dtype, op, algo, in_place=False):
     return [from_dev(t, dtype) for t in recv]
 
 
+def bits(a):
+    a = np.asarray(a)
+    return a.view(np.uint32) if a.dtype == np.float32 else a
+
+
 def assert_ranks_equal(got, want, what=""):
+    """Bit-for-bit equality (float32 arrays are compared as their bit patterns)."""
     for q, (g, w) in enumerate(zip(got, want)):
+        g, w = bits(g), bits(w)
         if not np.array_equal(g, w):
             bad = np.nonzero(g != w)[0]
             raise AssertionError(f"{what} rank {q}: {bad.size} mismatches, first at {bad[:5]}: "
@@ -180,11 +187,11 @@ def test_reduce(dtype, op):
         out = torch.empty_like(send[0])
         M.coll_reduce(send, out, dst, op=op)
         torch.cuda.synchronize()
-        assert np.array_equal(from_dev(out, dtype), oracle.reduce(xs, op, dtype))
+        assert np.array_equal(bits(from_dev(out, dtype)), bits(oracle.reduce(xs, op, dtype)))
     # in place on the destination
     M.coll_reduce(send, send[2], 2, op=op)
     torch.cuda.synchronize()
-    assert np.array_equal(from_dev(send[2], dtype), oracle.reduce(xs, op, dtype))
+    assert np.array_equal(bits(from_dev(send[2], dtype)), bits(oracle.reduce(xs, op, dtype)))
 
 
 def test_sp_prefill_reduce_scatter_full_size_sampled():
