@@ -371,6 +371,8 @@ def time_oracle(ops, min_s: float = 10.0, max_s: float = 30.0):
     about ``min_s`` seconds of CPU work (at most ``max_s``); returns
     (GB/s, sample description, seconds)."""
     refs = [op for op in ops if op.ref is not None]
+    if not refs:
+        return None, "no op of this workload has a CPU definition", 0.0
     secs, nbytes, passes, ops_done = 0.0, 0, 0, 0
     while secs < min_s:
         for op in refs:
