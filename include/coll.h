@@ -270,6 +270,34 @@ COLL_API int coll_moe_combine(const void* const* y, const int32_t* const* topk_i
                      coll_dtype_t dtype, int64_t recv_capacity_rows, int* d_status,
                      coll_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * All-reduce for callers that cannot allocate device memory.  The pages have
+ * no counterpart of this entry point: it exists for code that is handed only
+ * the ranks' buffers and may not call cudaMalloc -- a plug-in inside a host
+ * framework that owns every byte of device memory through its own pool, or a
+ * process whose memory was fully reserved (for example by a KV-cache pool) at
+ * start-up, so that any further allocation fails.
+ *
+ * It is the RING algorithm of coll_all_reduce, with the same result bit for
+ * bit, but its scratch (the fp32 / int32 partial sums that travel round the
+ * ring) lives in a fixed array of COLL_RING_NOALLOC_SCRATCH_BYTES compiled
+ * into this library: every GPU that loads the library holds that array until
+ * the process exits.  No cudaMalloc, cudaFree or other allocating routine is
+ * called.
+ *  - count may be at most COLL_RING_NOALLOC_MAX_COUNT elements; larger
+ *    calls return COLL_ERR_WORKSPACE and enqueue nothing.
+ *  - The first call on a device (with that device current) looks up the
+ *    array's device address; make that first call before any stream capture.
+ *  - All calls share the one array, so calls whose work overlaps on the GPU
+ *    (other streams, other threads) race: serialise them.  The array keeps
+ *    the last call's partials; nothing in it needs to start at zero, because
+ *    every partial is written before it is read.
+ * In place (recv[r] == send[r]) is allowed. */
+#define COLL_RING_NOALLOC_SCRATCH_BYTES (8u << 20)
+#define COLL_RING_NOALLOC_MAX_COUNT (COLL_RING_NOALLOC_SCRATCH_BYTES / 4u)
+COLL_API int coll_all_reduce_ring_noalloc(const void* const* send, void* const* recv, int nranks, size_t count,
+                                          coll_dtype_t dtype, coll_op_t op, coll_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 COLL_API const char* coll_strerror(int status);
 COLL_API int coll_version(void); /* major*10000 + minor*100 + patch */

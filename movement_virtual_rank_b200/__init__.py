@@ -68,6 +68,7 @@ _SIGS = {
     "coll_moe_route_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "coll_moe_dispatch": (_I, [_PP, _PP, _PP, _PP, _I, _I, _I, _I, _SZ, _I, _I64, _VP, _VP]),
     "coll_moe_combine": (_I, [_PP, _PP, _PP, _PP, _PP, _I, _I, _I, _I, _SZ, _I, _I64, _VP, _VP]),
+    "coll_all_reduce_ring_noalloc": (_I, [_PP, _PP, _I, _SZ, _I, _I, _VP]),
     "coll_strerror": (ctypes.c_char_p, [_I]),
     "coll_version": (_I, []),
 }
@@ -256,6 +257,29 @@ def coll_all_reduce(send, recv, op="sum", algo=TWOSHOT, workspace: torch.Tensor 
     with torch.cuda.device(send[0].device):
         _check("coll_all_reduce", lib().coll_all_reduce(ps, pr, len(send), n, _dt(send[0]), _op(op), algo,
                                                         ws_ptr, ws_bytes, _stream(stream)))
+
+
+RING_NOALLOC_MAX_COUNT = (8 << 20) // 4
+
+
+def coll_all_reduce_ring_noalloc(send, recv, op="sum", stream=None):
+    """Ring all-reduce that takes no workspace and allocates nothing, for
+    callers that may not allocate device memory: its partial sums live in a
+    fixed 8 MiB array inside the library (at most RING_NOALLOC_MAX_COUNT
+    elements per rank).  Same result as coll_all_reduce(..., algo=RING).
+    Calls that overlap on the GPU share that array and race."""
+    send = _ranks(send, "send", send[0].dtype)
+    recv = _ranks(recv, "recv", send[0].dtype)
+    if len(send) != len(recv):
+        raise ValueError("send and recv must list the same ranks")
+    n = _same_numel(send, "send")
+    if _same_numel(recv, "recv") != n:
+        raise ValueError("send and recv sizes differ")
+    ps, _k1 = _ptrs(send)
+    pr, _k2 = _ptrs(recv)
+    with torch.cuda.device(send[0].device):
+        _check("coll_all_reduce_ring_noalloc",
+               lib().coll_all_reduce_ring_noalloc(ps, pr, len(send), n, _dt(send[0]), _op(op), _stream(stream)))
 
 
 def coll_all_gather(send, recv, stream=None):
