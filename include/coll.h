@@ -78,7 +78,8 @@ typedef enum {
   COLL_ALGO_AUTO = 0,    /* currently TWOSHOT */
   COLL_ALGO_ONESHOT = 1, /* every rank reads all N inputs itself            */
   COLL_ALGO_TWOSHOT = 2, /* owner s reduces segment s, sends it to everyone */
-  COLL_ALGO_RING = 3     /* 2(N-1) neighbour steps                          */
+  COLL_ALGO_RING = 3,    /* 2(N-1) neighbour steps, one launch per step     */
+  COLL_ALGO_RING_LL = 4  /* the same ring in one launch, LL packets between ranks */
 } coll_algo_t;
 typedef enum { COLL_PROTO_SIMPLE = 0, COLL_PROTO_LL = 1, COLL_PROTO_LL128 = 2 } coll_proto_t;
 
@@ -154,8 +155,21 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    travel in fp32 (int32 for int32) through `workspace`
  *    (coll_all_reduce_workspace_size() bytes, 256-byte aligned); the result
  *    may differ from the rank-order reduction by rounding only.
+ *  RING_LL ([RLL] "Traditional LL Protocols", "Pro5000 ?": NCCL's Ring LL
+ *    kernel): the RING schedule, chunk order and rounding (bit-identical
+ *    result) in ONE cooperative launch.  Virtual rank r is a set of CTAs; it
+ *    sends each step's values to rank r+1 as LL lines [4 B value | 4 B flag]
+ *    in a FIFO in `workspace`, and rank r+1 re-reads each 16-byte group until
+ *    both flags match before using it.  Waits are bounded (about 1 s); a wait
+ *    that runs out makes every CTA stop and raises COLL_DEV_TIMEOUT in the
+ *    status pair at byte offset 16 of the workspace (int[2], cleared by the
+ *    caller).  The workspace (coll_all_reduce_workspace_size() bytes,
+ *    256-byte aligned) must be zero-filled once before its first use and
+ *    serves one call at a time; the library keeps a call counter in it.
+ *    Buffers that are not 16-byte aligned take the RING path.
  *  AUTO picks TWOSHOT.  ONESHOT and TWOSHOT ignore `workspace`.
- * In place (recv[r] == send[r]) is allowed for TWOSHOT, RING and AUTO. */
+ * In place (recv[r] == send[r]) is allowed for TWOSHOT, RING, RING_LL and
+ * AUTO. */
 COLL_API int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size_t count,
                     coll_dtype_t dtype, coll_op_t op, coll_algo_t algo, void* workspace,
                     size_t workspace_bytes, coll_stream_t stream);
@@ -297,6 +311,17 @@ COLL_API int coll_moe_combine(const void* const* y, const int32_t* const* topk_i
 #define COLL_RING_NOALLOC_MAX_COUNT (COLL_RING_NOALLOC_SCRATCH_BYTES / 4u)
 COLL_API int coll_all_reduce_ring_noalloc(const void* const* send, void* const* recv, int nranks, size_t count,
                                           coll_dtype_t dtype, coll_op_t op, coll_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Bounded wait on a device word (diagnostic).  Enqueues a one-thread kernel
+ * that re-reads *flag until it equals `expect`, for at most `budget_us`
+ * microseconds of GPU time; if the budget runs out it raises
+ * COLL_DEV_TIMEOUT in d_status (required) and returns normally.  It is the
+ * same bounded poll every waiting kernel of this library uses, exposed so that
+ * the time-out path can be exercised on purpose with a flag that nothing
+ * sets.  budget_us must be in [1, 10,000,000]. */
+COLL_API int coll_wait_flag(const uint32_t* flag, uint32_t expect, uint32_t budget_us, int* d_status,
+                            coll_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 COLL_API const char* coll_strerror(int status);

@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libmvrcoll.so")
 
 BF16, FP16, FP32, INT32 = 0, 1, 2, 3
 SUM, MAX, MIN, PROD = 0, 1, 2, 3
-ALGO_AUTO, ONESHOT, TWOSHOT, RING = 0, 1, 2, 3
+ALGO_AUTO, ONESHOT, TWOSHOT, RING, RING_LL = 0, 1, 2, 3, 4
 SIMPLE, LL, LL128 = 0, 1, 2
 DEV_OK, DEV_FLAG_MISMATCH, DEV_TIMEOUT, DEV_SPLIT_OVERFLOW, DEV_BAD_ROUTE = 0, 1, 2, 3, 4
 MAX_RANKS = 64
@@ -30,7 +30,7 @@ MAX_RANKS = 64
 _DTYPES = {torch.bfloat16: BF16, torch.float16: FP16, torch.float32: FP32, torch.int32: INT32}
 _ESIZE = {BF16: 2, FP16: 2, FP32: 4, INT32: 4}
 OPS = {"sum": SUM, "max": MAX, "min": MIN, "prod": PROD}
-ALGOS = {"auto": ALGO_AUTO, "oneshot": ONESHOT, "twoshot": TWOSHOT, "ring": RING}
+ALGOS = {"auto": ALGO_AUTO, "oneshot": ONESHOT, "twoshot": TWOSHOT, "ring": RING, "ring_ll": RING_LL}
 PROTOS = {"simple": SIMPLE, "ll": LL, "ll128": LL128}
 
 
@@ -69,6 +69,7 @@ _SIGS = {
     "coll_moe_dispatch": (_I, [_PP, _PP, _PP, _PP, _I, _I, _I, _I, _SZ, _I, _I64, _VP, _VP]),
     "coll_moe_combine": (_I, [_PP, _PP, _PP, _PP, _PP, _I, _I, _I, _I, _SZ, _I, _I64, _VP, _VP]),
     "coll_all_reduce_ring_noalloc": (_I, [_PP, _PP, _I, _SZ, _I, _I, _VP]),
+    "coll_wait_flag": (_I, [_VP, ctypes.c_uint32, ctypes.c_uint32, _VP, _VP]),
     "coll_strerror": (ctypes.c_char_p, [_I]),
     "coll_version": (_I, []),
 }
@@ -236,8 +237,9 @@ def coll_all_reduce_workspace_size(nranks: int, count: int, dtype: torch.dtype, 
 
 
 def coll_all_reduce(send, recv, op="sum", algo=TWOSHOT, workspace: torch.Tensor | None = None, stream=None):
-    """``workspace`` (RING only): a CUDA tensor of at least
-    coll_all_reduce_workspace_size() bytes; allocated here when omitted."""
+    """``workspace`` (RING and RING_LL): a CUDA tensor of at least
+    coll_all_reduce_workspace_size() bytes, zero-filled before its first
+    RING_LL use; allocated (zeroed) here when omitted."""
     algo = ALGOS[algo] if isinstance(algo, str) else int(algo)
     send = _ranks(send, "send", send[0].dtype)
     recv = _ranks(recv, "recv", send[0].dtype)
@@ -247,10 +249,10 @@ def coll_all_reduce(send, recv, op="sum", algo=TWOSHOT, workspace: torch.Tensor 
     if _same_numel(recv, "recv") != n:
         raise ValueError("send and recv sizes differ")
     ws_ptr, ws_bytes = None, 0
-    if algo == RING:
-        need = coll_all_reduce_workspace_size(len(send), n, send[0].dtype, RING)
+    if algo in (RING, RING_LL):
+        need = coll_all_reduce_workspace_size(len(send), n, send[0].dtype, algo)
         if workspace is None:
-            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=send[0].device)
+            workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=send[0].device)
         ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     ps, _k1 = _ptrs(send)
     pr, _k2 = _ptrs(recv)
@@ -458,6 +460,15 @@ def coll_moe_combine(y, topk_ids, pos, topk_w, out, n_experts: int, status: torc
     with torch.cuda.device(y[0].device):
         _check("coll_moe_combine", lib().coll_moe_combine(py, pi, pp, pw, po, n, tokens, topk, n_experts, hidden,
                                                           _dt(y[0]), cap, st, _stream(stream)))
+
+
+def coll_wait_flag(flag: torch.Tensor, expect: int, budget_us: int, status: torch.Tensor, stream=None):
+    """Bounded wait on a device word (flag: int32/uint32 CUDA tensor, first element)."""
+    _cuda(flag, "flag")
+    _cuda(status, "status")
+    with torch.cuda.device(flag.device):
+        _check("coll_wait_flag", lib().coll_wait_flag(flag.data_ptr(), expect & 0xFFFFFFFF, budget_us,
+                                                      status.data_ptr(), _stream(stream)))
 
 
 def coll_strerror(code: int) -> str:

@@ -286,15 +286,17 @@ int coll_reduce_scatter(const void* const* send, void* const* recv, int nranks, 
 
 // ------------------------------------------------------------- AllReduce ----
 size_t coll_all_reduce_workspace_size(int nranks, size_t count, coll_dtype_t dtype, coll_algo_t algo) {
-  if (algo != COLL_ALGO_RING || !valid_n(nranks) || !elem_size(dtype)) return 0;
-  return ring_ws(count);
+  if (!valid_n(nranks) || !elem_size(dtype)) return 0;
+  if (algo == COLL_ALGO_RING) return ring_ws(count);
+  if (algo == COLL_ALGO_RING_LL) return std::max(ring_ll_workspace(nranks, count, elem_size(dtype)), 256 + ring_ws(count));
+  return 0;
 }
 
 int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size_t count, coll_dtype_t dtype,
                     coll_op_t op, coll_algo_t algo, void* workspace, size_t workspace_bytes, coll_stream_t stream) {
   const int es = elem_size(dtype);
   if (!es) return COLL_ERR_UNSUPPORTED;
-  if (!valid_op(op) || algo < COLL_ALGO_AUTO || algo > COLL_ALGO_RING) return COLL_ERR_UNSUPPORTED;
+  if (!valid_op(op) || algo < COLL_ALGO_AUTO || algo > COLL_ALGO_RING_LL) return COLL_ERR_UNSUPPORTED;
   if (!valid_n(nranks) || !all_nonnull(send, nranks) || !all_nonnull(recv, nranks)) return COLL_ERR_INVALID_ARG;
   const size_t bytes = count * es;
   if (bytes == 0) return COLL_OK;
@@ -304,20 +306,33 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
     for (int r = 0; r < nranks; ++r)
       if (overlap(recv[q], bytes, send[r], bytes) && !(q == r && recv[q] == send[r] && algo != COLL_ALGO_ONESHOT))
         return COLL_ERR_ALIAS;
-  if (algo == COLL_ALGO_RING && nranks > 1) {
-    if (workspace == nullptr || workspace_bytes < ring_ws(count) || !al16(workspace)) return COLL_ERR_WORKSPACE;
-    if (overlap(workspace, ring_ws(count), recv[0], bytes)) {
-      // the partials must not live inside any rank's buffer
-      return COLL_ERR_ALIAS;
-    }
+  if ((algo == COLL_ALGO_RING || algo == COLL_ALGO_RING_LL) && nranks > 1) {
+    const size_t need = coll_all_reduce_workspace_size(nranks, count, dtype, algo);
+    if (workspace == nullptr || workspace_bytes < need || (U(workspace) & (algo == COLL_ALGO_RING_LL ? 255 : 15)))
+      return COLL_ERR_WORKSPACE;
+    // the partials / FIFOs must not live inside any rank's buffer
     for (int r = 0; r < nranks; ++r)
-      if (overlap(workspace, ring_ws(count), send[r], bytes) || overlap(workspace, ring_ws(count), recv[r], bytes))
-        return COLL_ERR_ALIAS;
+      if (overlap(workspace, need, send[r], bytes) || overlap(workspace, need, recv[r], bytes)) return COLL_ERR_ALIAS;
   }
   if (nranks == 1) return copy_one(send[0], recv[0], bytes, S(stream));
   bool vec = true;
   for (int r = 0; r < nranks; ++r) vec = vec && al16(send[r]) && al16(recv[r]);
   const size_t seg = seg_elems(count, nranks, es);
+  if (algo == COLL_ALGO_RING_LL) {
+    if (vec) {
+      const char* in[COLL_MAX_RANKS];
+      char* out[COLL_MAX_RANKS];
+      for (int r = 0; r < nranks; ++r) {
+        in[r] = static_cast<const char*>(send[r]);
+        out[r] = static_cast<char*>(recv[r]);
+      }
+      int* status = reinterpret_cast<int*>(static_cast<char*>(workspace) + 16);
+      return launch_ring_ll(in, out, nranks, count, dtype, op, workspace, status, S(stream));
+    }
+    // unaligned buffers: the stream-ordered ring, its partials after the header
+    workspace = static_cast<char*>(workspace) + 256;
+    algo = COLL_ALGO_RING;
+  }
   if (algo == COLL_ALGO_RING) {
     RingStepArgs a{};
     for (int r = 0; r < nranks; ++r) {
@@ -464,6 +479,11 @@ int coll_all_to_all_v(const void* const* send, void* const* recv, int nranks, co
                       static_cast<size_t>(c) * row});
     }
   return launch_copy_jobs(jobs.data(), static_cast<int>(jobs.size()), S(stream));
+}
+
+int coll_wait_flag(const uint32_t* flag, uint32_t expect, uint32_t budget_us, int* d_status, coll_stream_t stream) {
+  if (flag == nullptr || d_status == nullptr || budget_us == 0 || budget_us > 10000000u) return COLL_ERR_INVALID_ARG;
+  return launch_wait_flag(flag, expect, budget_us, d_status, S(stream));
 }
 
 // --------------------------------------------------------------- packets ----

@@ -15,8 +15,16 @@
 #include <algorithm>
 #include <vector>
 
+#include "bulk.cuh"
 #include "common.cuh"
 #include "internal.h"
+
+// The fan-out uses bulk copies when every CTA gets at least this many tiles
+// to pipeline (below that a CTA waits for one load, then one store round,
+// and the element path is faster); compile-time tunable.
+#ifndef MVR_FANOUT_TMA_MIN_TILES_PER_CTA
+#define MVR_FANOUT_TMA_MIN_TILES_PER_CTA 4
+#endif
 
 namespace mvr {
 
@@ -69,11 +77,77 @@ __global__ void __launch_bounds__(kThreads) k_fanout(const __grid_constant__ Fan
   }
 }
 
+// Bulk-copy fan-out: one thread per CTA streams tiles of a source into a ring
+// of shared-memory stages with cp.async.bulk and writes each landed tile to
+// every destination with bulk stores; a stage is refilled once its stores
+// have finished reading it.  Tiles of all sources are interleaved over the
+// grid so that every source progresses at once.
+constexpr int kTmaTile = 8192;
+constexpr int kTmaStages = 4;
+
+__global__ void __launch_bounds__(32) k_fanout_tma(const __grid_constant__ FanoutArgs a) {
+  extern __shared__ __align__(128) unsigned char stage_buf[];
+  __shared__ __align__(8) uint64_t bar[kTmaStages];
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x != 0) return;
+  for (int st = 0; st < kTmaStages; ++st) mbar_init(&bar[st], 1);
+  fence_barrier_init();
+  const uint64_t pieces = (a.bytes + kTmaTile - 1) / kTmaTile;
+  const uint64_t total = pieces * static_cast<uint64_t>(a.ns);
+  const uint64_t stride = gridDim.x;
+  auto issue = [&](uint64_t t, int st) {
+    const int r = static_cast<int>(t % a.ns);
+    const uint64_t off = (t / a.ns) * kTmaTile;
+    const uint32_t len = static_cast<uint32_t>(a.bytes - off < kTmaTile ? a.bytes - off : kTmaTile);
+    mbar_arrive_expect_tx(&bar[st], len);
+    bulk_load(stage_buf + st * kTmaTile, a.src[r] + off, len, &bar[st]);
+  };
+  int inflight = 0;
+  for (int st = 0; st < kTmaStages && blockIdx.x + st * stride < total; ++st, ++inflight) issue(blockIdx.x + st * stride, st);
+  int i = 0;
+  for (uint64_t t = blockIdx.x; t < total; t += stride, ++i) {
+    const int st = i % kTmaStages;
+    if (!mbar_wait_bounded(&bar[st], (i / kTmaStages) & 1)) {
+      report(a.status, COLL_DEV_TIMEOUT, 1);
+      bulk_wait_all();
+      for (int k = 1; k < inflight; ++k)  // the loads still in flight, bounded again
+        mbar_wait_bounded(&bar[(i + k) % kTmaStages], ((i + k) / kTmaStages) & 1);
+      return;
+    }
+    --inflight;
+    const int r = static_cast<int>(t % a.ns);
+    const uint64_t off = (t / a.ns) * kTmaTile;
+    const uint32_t len = static_cast<uint32_t>(a.bytes - off < kTmaTile ? a.bytes - off : kTmaTile);
+    const unsigned char* src = stage_buf + st * kTmaTile;
+    const uint64_t roff = static_cast<uint64_t>(r) * a.dst_stride + off;
+    for (int q = 0; q < a.nd; ++q) {
+      if (a.skip_diag && q == r) continue;
+      bulk_store(a.dst[q] + roff, src, len);
+    }
+    bulk_commit();
+    const uint64_t nxt = t + kTmaStages * stride;
+    if (nxt < total) {
+      bulk_wait_read<0>();
+      issue(nxt, st);
+      ++inflight;
+    }
+  }
+  bulk_wait_all();
+}
+
 int launch_fanout(const FanoutArgs& a, cudaStream_t s) {
   if (a.bytes == 0 || a.ns == 0 || a.nd == 0) return COLL_OK;
   uint64_t bits = a.dst_stride;
   for (int r = 0; r < a.ns; ++r) bits |= reinterpret_cast<uintptr_t>(a.src[r]);
   for (int q = 0; q < a.nd; ++q) bits |= reinterpret_cast<uintptr_t>(a.dst[q]);
+  const uint64_t tiles = (a.bytes + kTmaTile - 1) / kTmaTile * a.ns;
+  const uint64_t tma_grid = static_cast<uint64_t>(num_sms()) * 6;  // 6 x 32 KB of stages per SM
+  if ((bits & 15) == 0 && (a.bytes & 15) == 0 && tiles >= MVR_FANOUT_TMA_MIN_TILES_PER_CTA * tma_grid) {
+    const uint64_t grid = tma_grid;
+    launch_pdl(k_fanout_tma, dim3(static_cast<unsigned>(grid)), dim3(32), kTmaStages * kTmaTile, s, a);
+    return launch_status(cudaGetLastError());
+  }
   const int U = pick_unit(bits);
   const unsigned grid = grid_for(a.bytes / U, a.ns);
   switch (U) {

@@ -41,6 +41,11 @@ struct RingStepArgs {
 int launch_ring_rs_step(const RingStepArgs& a, coll_dtype_t dt, coll_op_t op, bool vec,
                         cudaStream_t s);
 
+size_t ring_ll_workspace(int n, size_t count, int es);
+int launch_ring_ll(const char* const* in, char* const* out, int n, size_t count, coll_dtype_t dt, coll_op_t op,
+                   void* workspace, int* status, cudaStream_t s);
+int launch_wait_flag(const uint32_t* flag, uint32_t expect, uint32_t budget_us, int* status, cudaStream_t s);
+
 // ---------------------------------------------------------------- copies ----
 struct FanoutArgs {
   const char* src[kMaxRanksH];
@@ -49,6 +54,7 @@ struct FanoutArgs {
   uint64_t dst_stride;  // dst for (source r, destination q) = dst[q] + r * dst_stride
   int ns, nd;
   int skip_diag;        // skip q == r (in-place all-gather)
+  int* status;          // optional device status pair (bounded-wait timeouts)
 };
 int launch_fanout(const FanoutArgs& a, cudaStream_t s);
 

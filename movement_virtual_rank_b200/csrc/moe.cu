@@ -281,7 +281,7 @@ int launch_moe_dispatch(const MoeMoveArgs& a, cudaStream_t s) {
 
 // ---------------------------------------------------------------- combine ----
 
-template <int DT, bool VEC>
+template <int DT, bool VEC, int TK>  // TK: top-k known at compile time (0 = runtime)
 __global__ void __launch_bounds__(kMoveThreads) k_moe_combine(const __grid_constant__ MoeMoveArgs a) {
   pdl_wait();
   pdl_trigger();
@@ -291,14 +291,15 @@ __global__ void __launch_bounds__(kMoveThreads) k_moe_combine(const __grid_const
   __shared__ const char* src[kMaxTopk];
   __shared__ float wk[kMaxTopk];
   __shared__ int nbad;
+  const int topk = TK > 0 ? TK : a.topk;
   const int64_t rows = static_cast<int64_t>(a.n) * a.tokens;
   const uint64_t relems = a.row_bytes / ES;
   int bad = 0;
   for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
     const int s = static_cast<int>(row / a.tokens);
     const int t = static_cast<int>(row % a.tokens);
-    if (threadIdx.x < a.topk) {
-      const int64_t j = static_cast<int64_t>(t) * a.topk + threadIdx.x;
+    if (threadIdx.x < topk) {
+      const int64_t j = static_cast<int64_t>(t) * topk + threadIdx.x;
       const int e = a.ids[s][j];
       const int64_t p = a.pos[s][j];
       const int d = e / a.epr;
@@ -312,10 +313,35 @@ __global__ void __launch_bounds__(kMoveThreads) k_moe_combine(const __grid_const
     }
     __syncthreads();
     char* out = a.y[s] + static_cast<uint64_t>(t) * a.row_bytes;
-    if constexpr (VEC) {
+    if constexpr (VEC && TK > 0) {
+      const char* sp[TK];
+      float w[TK];
+#pragma unroll
+      for (int k = 0; k < TK; ++k) {
+        sp[k] = src[k];
+        w[k] = wk[k];
+      }
+      for (uint64_t u = threadIdx.x; u < relems / VN; u += blockDim.x) {
+        uint4 x[TK];
+#pragma unroll
+        for (int k = 0; k < TK; ++k) x[k] = sp[k] != nullptr ? ld16(sp[k] + u * 16) : make_uint4(0, 0, 0, 0);
+        Vec<DT> acc;
+#pragma unroll
+        for (int k = 0; k < TK; ++k) {
+          Vec<DT> v;
+          widen16<DT>(x[k], v);
+#pragma unroll
+          for (int i = 0; i < VN; ++i) {
+            const float prod = __fmul_rn(w[k], v.v[i]);
+            acc.v[i] = k == 0 ? prod : __fadd_rn(acc.v[i], prod);
+          }
+        }
+        st16(out + u * 16, narrow16<DT>(acc));
+      }
+    } else if constexpr (VEC) {
       for (uint64_t u = threadIdx.x; u < relems / VN; u += blockDim.x) {
         Vec<DT> acc;
-        for (int k = 0; k < a.topk; ++k) {
+        for (int k = 0; k < topk; ++k) {
           Vec<DT> v;
           if (src[k] != nullptr) widen16<DT>(ld16(src[k] + u * 16), v);
           else widen16<DT>(make_uint4(0, 0, 0, 0), v);
@@ -331,7 +357,7 @@ __global__ void __launch_bounds__(kMoveThreads) k_moe_combine(const __grid_const
     } else {
       for (uint64_t e = threadIdx.x; e < relems; e += blockDim.x) {
         float acc = 0.f;
-        for (int k = 0; k < a.topk; ++k) {
+        for (int k = 0; k < topk; ++k) {
           const float v = src[k] != nullptr ? widen1<DT>(*reinterpret_cast<const S*>(src[k] + e * ES)) : 0.f;
           const float prod = __fmul_rn(wk[k], v);
           acc = k == 0 ? prod : __fadd_rn(acc, prod);
@@ -354,8 +380,9 @@ static int launch_combine_dt(const MoeMoveArgs& a, cudaStream_t s) {
   uint64_t bits = a.row_bytes;
   for (int r = 0; r < a.n; ++r) bits |= reinterpret_cast<uintptr_t>(a.x[r]) | reinterpret_cast<uintptr_t>(a.y[r]);
   const unsigned grid = move_grid(rows);
-  if ((bits & 15) == 0) launch_pdl(k_moe_combine<DT, true>, dim3(grid), dim3(kMoveThreads), 0, s, a);
-  else launch_pdl(k_moe_combine<DT, false>, dim3(grid), dim3(kMoveThreads), 0, s, a);
+  if ((bits & 15) == 0 && a.topk == 8) launch_pdl(k_moe_combine<DT, true, 8>, dim3(grid), dim3(kMoveThreads), 0, s, a);
+  else if ((bits & 15) == 0) launch_pdl(k_moe_combine<DT, true, 0>, dim3(grid), dim3(kMoveThreads), 0, s, a);
+  else launch_pdl(k_moe_combine<DT, false, 0>, dim3(grid), dim3(kMoveThreads), 0, s, a);
   return launch_status(cudaGetLastError());
 }
 

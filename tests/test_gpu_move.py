@@ -241,3 +241,42 @@ def test_all_to_all_v_many_launches():
     want = oracle.all_to_all_v(xs, [np.full(t.numel(), -1, np.int32) for t in recv], sc, sd, rd, row)
     for d in range(n):
         assert np.array_equal(from_dev(recv[d], "int32"), want[d])
+
+
+@pytest.mark.parametrize("count", [1 << 21, 2000008, 2000003])
+@pytest.mark.parametrize("n", [2, 8])
+def test_all_gather_bulk_copy_sizes(n, count):
+    """Large fan-outs (at least 4 tiles of 8 KB per CTA, about 29 MB in all on
+    148 SMs) take the bulk-copy (TMA) path: a whole number of tiles, a ragged
+    last tile, and a length that is not a multiple of 16 bytes (which must
+    take the element path instead).  The 2-rank cases stay below the
+    threshold and check the element path at the same sizes."""
+    need_gpu()
+    xs = rand(n, count, "bf16", salt=count + 3 * n)
+    send = [to_dev(x, "bf16") for x in xs]
+    recv = [torch.full((n * count,), 3.0, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+    M.coll_all_gather(send, recv)
+    torch.cuda.synchronize()
+    want = np.concatenate(xs)
+    for q in range(n):
+        assert np.array_equal(from_dev(recv[q], "bf16"), want)
+    # in place
+    recv2 = [torch.zeros(n * count, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+    for r in range(n):
+        recv2[r][r * count:(r + 1) * count].copy_(send[r])
+    M.coll_all_gather([recv2[r][r * count:(r + 1) * count] for r in range(n)], recv2)
+    torch.cuda.synchronize()
+    for q in range(n):
+        assert np.array_equal(from_dev(recv2[q], "bf16"), want)
+
+
+@pytest.mark.parametrize("count", [1 << 23, (1 << 23) + 4, 3 * 1000003])
+def test_broadcast_bulk_copy_sizes(count):
+    need_gpu()
+    n = 8
+    xs = rand(n, count, "int32", salt=count)
+    bufs = [to_dev(x, "int32") for x in xs]
+    M.coll_broadcast(bufs, 5)
+    torch.cuda.synchronize()
+    for q in range(n):
+        assert np.array_equal(from_dev(bufs[q], "int32"), xs[5])

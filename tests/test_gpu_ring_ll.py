@@ -1,0 +1,128 @@
+"""GPU parity: the single-launch LL ring all-reduce (COLL_ALGO_RING_LL).
+
+It follows the ring schedule, chunk order and rounding of the stream-ordered
+ring, so its output is compared bit for bit with the oracle's ring; repeated
+calls on one workspace check that the per-call flag epoch keeps earlier
+lines from being taken for new ones.  The bounded wait is checked on its own
+with coll_wait_flag on a flag that nothing sets: the kernel gives up, reports
+COLL_DEV_TIMEOUT and the context stays usable.
+"""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import movement_virtual_rank_b200 as M
+import oracle
+import workloads as W
+from gpu_util import from_dev, need_gpu, status_tensor, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def bits(a):
+    a = np.asarray(a)
+    return a.view(np.uint32) if a.dtype == np.float32 else a
+
+
+def run(xs, dtype, op, ws=None, in_place=False):
+    send = [to_dev(x, dtype) for x in xs]
+    recv = send if in_place else [torch.empty_like(t) for t in send]
+    M.coll_all_reduce(send, recv, op=op, algo=M.RING_LL, workspace=ws)
+    torch.cuda.synchronize()
+    return [from_dev(t, dtype) for t in recv]
+
+
+@pytest.mark.parametrize("n", [2, 3, 4, 8])
+@pytest.mark.parametrize("count", [1, 9, 8 * 37 + 3, 65536 + 24, 300007, 1835008])
+def test_ring_ll_bf16_sum(n, count):
+    need_gpu()
+    xs = W.ranks_values(W.W_MISC, n, count, "bf16", "normal", salt=count + 7 * n)
+    want = oracle.all_reduce_ring(xs, 0, "bf16")
+    got = run(xs, "bf16", 0)
+    for q in range(n):
+        assert np.array_equal(got[q], want[q]), q
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16", "fp32", "int32"])
+@pytest.mark.parametrize("op", [0, 1, 2, 3])
+def test_ring_ll_dtypes_ops(dtype, op):
+    need_gpu()
+    n, count = 5, 12301
+    if dtype == "int32":
+        g = W.rng(W.W_MISC, 0, salt=op + 40)
+        xs = [g.integers(-1000, 1000, count, dtype=np.int64).astype(np.int32) for _ in range(n)]
+    else:
+        xs = W.ranks_values(W.W_MISC, n, count, dtype, "uniform" if op == 3 else "normal", salt=op + 40)
+    want = oracle.all_reduce_ring(xs, op, dtype)
+    got = run(xs, dtype, op)
+    for q in range(n):
+        assert np.array_equal(bits(got[q]), bits(want[q])), q
+
+
+def test_ring_ll_repeated_calls_one_workspace_and_in_place():
+    """Twenty calls on one workspace: every call must use only its own lines."""
+    need_gpu()
+    n, count = 8, 200003
+    need = M.coll_all_reduce_workspace_size(n, count, torch.bfloat16, M.RING_LL)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for call in range(20):
+        xs = W.ranks_values(W.W_MISC, n, count, "bf16", "normal", salt=500 + call)
+        got = run(xs, "bf16", 0, ws=ws, in_place=(call % 2 == 1))
+        want = oracle.all_reduce_ring(xs, 0, "bf16")
+        for q in range(n):
+            assert np.array_equal(got[q], want[q]), (call, q)
+    st = ws[16:24].view(torch.int32)
+    assert st.tolist() == [0, 0]
+
+
+def test_ring_ll_tp_decode_workload():
+    need_gpu()
+    for tokens, hidden in W.tp_decode_shapes():
+        xs = W.tp_decode(tokens, hidden)
+        got = run(xs, "bf16", 0)
+        want = oracle.all_reduce_ring(xs, 0, "bf16")
+        for q in range(8):
+            assert np.array_equal(got[q], want[q]), (tokens, hidden, q)
+
+
+def test_ring_ll_unaligned_takes_the_ring_path():
+    need_gpu()
+    n, count = 4, 5001
+    xs = W.ranks_values(W.W_MISC, n, count, "bf16", "normal", salt=77)
+    raw = [torch.empty(count + 8, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+    send = [raw[r][1:count + 1] for r in range(n)]
+    for r in range(n):
+        send[r].copy_(to_dev(xs[r], "bf16"))
+    recv = [torch.empty(count + 8, dtype=torch.bfloat16, device="cuda")[3:count + 3] for _ in range(n)]
+    M.coll_all_reduce(send, recv, algo=M.RING_LL)
+    torch.cuda.synchronize()
+    want = oracle.all_reduce_ring(xs, 0, "bf16")
+    for q in range(n):
+        assert np.array_equal(from_dev(recv[q], "bf16"), want[q])
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """A flag that nothing sets: the wait gives up after its budget, raises
+    COLL_DEV_TIMEOUT, and later work on the same context is unaffected."""
+    need_gpu()
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = status_tensor()
+    t0 = time.perf_counter()
+    M.coll_wait_flag(flag, 1, 20000, st)  # 20 ms budget
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    assert st.tolist() == [M.DEV_TIMEOUT, 1]
+    assert 0.015 < dt < 5.0
+    # a flag that is already set returns at once with no status
+    st.zero_()
+    flag.fill_(7)
+    M.coll_wait_flag(flag, 7, 20000, st)
+    torch.cuda.synchronize()
+    assert st.tolist() == [0, 0]
+    # the context still works
+    xs = W.ranks_values(W.W_MISC, 3, 999, "bf16", "normal", salt=1)
+    got = run(xs, "bf16", 0)
+    want = oracle.all_reduce_ring(xs, 0, "bf16")
+    assert all(np.array_equal(g, w) for g, w in zip(got, want))
