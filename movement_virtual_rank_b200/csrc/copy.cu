@@ -191,11 +191,95 @@ __global__ void __launch_bounds__(kThreads) k_copy_jobs(const __grid_constant__ 
     else j1 = m - 1;
   }
   int j = j0;
-  for (uint64_t u = lo + threadIdx.x; u < hi; u += blockDim.x) {
-    while (u >= a.job[j + 1].start) ++j;
-    const uint64_t off = (u - a.job[j].start) * U;
-    stu<U>(a.job[j].dst + off, ldu<U>(a.job[j].src + off));
+  // four units per thread per round: all four loads are issued before any store
+  constexpr int kU = 4;
+  for (uint64_t base = lo + threadIdx.x; base < hi; base += kU * blockDim.x) {
+    typename UnitT<U>::T v[kU];
+    char* d[kU];
+#pragma unroll
+    for (int i = 0; i < kU; ++i) {
+      const uint64_t u = base + static_cast<uint64_t>(i) * blockDim.x;
+      d[i] = nullptr;
+      if (u < hi) {
+        while (u >= a.job[j + 1].start) ++j;
+        const uint64_t off = (u - a.job[j].start) * U;
+        v[i] = ldu<U>(a.job[j].src + off);
+        d[i] = a.job[j].dst + off;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kU; ++i)
+      if (d[i] != nullptr) stu<U>(d[i], v[i]);
   }
+}
+
+// Bulk-copy form of the job list for large copies: one thread per CTA
+// streams tiles (each within one job) through a ring of shared-memory stages,
+// loading with cp.async.bulk and storing each landed tile with a bulk store.
+struct TmaJob {
+  const char* src;
+  char* dst;
+  uint64_t bytes;
+  uint64_t tile0;  // first tile of this job in the concatenation of all jobs
+};
+constexpr int kMaxTmaJobs = 900;  // 900 * 32 B + header < 32 KB of kernel parameters
+struct TmaJobsArgs {
+  uint64_t total_tiles;
+  int njobs;
+  int* status;
+  TmaJob job[kMaxTmaJobs + 1];  // job[njobs].tile0 == total_tiles (sentinel)
+};
+
+__global__ void __launch_bounds__(32) k_copy_jobs_tma(const __grid_constant__ TmaJobsArgs a) {
+  extern __shared__ __align__(128) unsigned char stage_buf[];
+  __shared__ __align__(8) uint64_t bar[kTmaStages];
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x != 0) return;
+  for (int st = 0; st < kTmaStages; ++st) mbar_init(&bar[st], 1);
+  fence_barrier_init();
+  const uint64_t stride = gridDim.x;
+  int jl = 0;  // job of the next tile to load (tiles are visited in increasing order)
+  int js = 0;  // job of the next tile to store
+  auto locate = [&](uint64_t t, int& j, uint64_t& off, uint32_t& len) {
+    while (t >= a.job[j + 1].tile0) ++j;
+    off = (t - a.job[j].tile0) * kTmaTile;
+    const uint64_t rest = a.job[j].bytes - off;
+    len = static_cast<uint32_t>(rest < kTmaTile ? rest : kTmaTile);
+  };
+  auto issue = [&](uint64_t t, int st) {
+    uint64_t off;
+    uint32_t len;
+    locate(t, jl, off, len);
+    mbar_arrive_expect_tx(&bar[st], len);
+    bulk_load(stage_buf + st * kTmaTile, a.job[jl].src + off, len, &bar[st]);
+  };
+  int inflight = 0;
+  for (int st = 0; st < kTmaStages && blockIdx.x + st * stride < a.total_tiles; ++st, ++inflight)
+    issue(blockIdx.x + st * stride, st);
+  int i = 0;
+  for (uint64_t t = blockIdx.x; t < a.total_tiles; t += stride, ++i) {
+    const int st = i % kTmaStages;
+    if (!mbar_wait_bounded(&bar[st], (i / kTmaStages) & 1)) {
+      report(a.status, COLL_DEV_TIMEOUT, 1);
+      bulk_wait_all();
+      for (int k = 1; k < inflight; ++k) mbar_wait_bounded(&bar[(i + k) % kTmaStages], ((i + k) / kTmaStages) & 1);
+      return;
+    }
+    --inflight;
+    uint64_t off;
+    uint32_t len;
+    locate(t, js, off, len);
+    bulk_store(a.job[js].dst + off, stage_buf + st * kTmaTile, len);
+    bulk_commit();
+    const uint64_t nxt = t + kTmaStages * stride;
+    if (nxt < a.total_tiles) {
+      bulk_wait_read<0>();
+      issue(nxt, st);
+      ++inflight;
+    }
+  }
+  bulk_wait_all();
 }
 
 int launch_copy_jobs(const CopyJob* jobs, int njobs, cudaStream_t s) {
@@ -210,6 +294,33 @@ int launch_copy_jobs(const CopyJob* jobs, int njobs, cudaStream_t s) {
   }
   if (v.empty()) return COLL_OK;
   const int U = pick_unit(bits);
+  // large, 16-byte aligned job lists go through the bulk-copy path
+  if (U == 16) {
+    uint64_t tiles = 0;
+    for (const CopyJob& j : v) tiles += (j.bytes + kTmaTile - 1) / kTmaTile;
+    const uint64_t tma_grid = static_cast<uint64_t>(num_sms()) * 6;
+    if (tiles >= MVR_FANOUT_TMA_MIN_TILES_PER_CTA * tma_grid) {
+      static thread_local TmaJobsArgs targs;  // ~29 KB: keep it off the stack
+      for (size_t first = 0; first < v.size(); first += kMaxTmaJobs) {
+        const int nj = static_cast<int>(std::min<size_t>(kMaxTmaJobs, v.size() - first));
+        uint64_t acc = 0;
+        for (int i = 0; i < nj; ++i) {
+          const CopyJob& j = v[first + i];
+          targs.job[i] = TmaJob{j.src, j.dst, j.bytes, acc};
+          acc += (j.bytes + kTmaTile - 1) / kTmaTile;
+        }
+        targs.job[nj] = TmaJob{nullptr, nullptr, 0, acc};
+        targs.total_tiles = acc;
+        targs.njobs = nj;
+        targs.status = nullptr;
+        const uint64_t grid = std::min<uint64_t>(acc, tma_grid);
+        launch_pdl(k_copy_jobs_tma, dim3(static_cast<unsigned>(grid)), dim3(32), kTmaStages * kTmaTile, s, targs);
+        const int st = launch_status(cudaGetLastError());
+        if (st != COLL_OK) return st;
+      }
+      return COLL_OK;
+    }
+  }
   static thread_local CopyJobsArgs args;  // ~23 KB: keep it off the stack
   for (size_t first = 0; first < v.size(); first += kMaxJobs) {
     const int nj = static_cast<int>(std::min<size_t>(kMaxJobs, v.size() - first));

@@ -20,6 +20,7 @@
 // expert rows and forms acc = fl32(w0*y0), acc = fl32(acc + fl32(wk*yk)).
 #include <algorithm>
 
+#include "bulk.cuh"
 #include "common.cuh"
 #include "internal.h"
 
@@ -250,6 +251,88 @@ __global__ void __launch_bounds__(kMoveThreads) k_moe_dispatch(const __grid_cons
   if (threadIdx.x == 0) report(a.status, COLL_DEV_SPLIT_OVERFLOW, nbad);
 }
 
+// Bulk-copy dispatch: one warp per CTA.  Each token row is loaded once into
+// a shared-memory stage with cp.async.bulk and written to its topk receive
+// rows with bulk stores; when a row's load is issued, lanes 0..topk-1 also
+// look up where it goes, so the stores never wait on those lookups.
+constexpr int kDispStages = 4;
+constexpr uint32_t kDispMaxRow = 32768;  // bytes of one row in a stage
+
+__global__ void __launch_bounds__(32) k_moe_dispatch_tma(const __grid_constant__ MoeMoveArgs a, uint32_t stage_bytes) {
+  extern __shared__ __align__(128) unsigned char stage_buf[];
+  __shared__ __align__(8) uint64_t bar[kDispStages];
+  __shared__ char* dst[kDispStages][kMaxTopk];
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x;
+  const uint32_t rb = static_cast<uint32_t>(a.row_bytes);
+  if (lane == 0) {
+    for (int st = 0; st < kDispStages; ++st) mbar_init(&bar[st], 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  const uint64_t rows = static_cast<uint64_t>(a.n) * a.tokens;
+  const uint64_t stride = gridDim.x;
+  int bad = 0;
+  auto issue = [&](uint64_t row, int st) {
+    const int s = static_cast<int>(row / a.tokens);
+    const int t = static_cast<int>(row % a.tokens);
+    if (lane < a.topk) {
+      const int64_t j = static_cast<int64_t>(t) * a.topk + lane;
+      const int e = a.ids[s][j];
+      const int64_t p = a.pos[s][j];
+      const int d = e / a.epr;
+      if (e < 0 || d >= a.n || p < 0 || p >= a.capacity) {
+        dst[st][lane] = nullptr;
+        ++bad;
+      } else {
+        dst[st][lane] = a.y[d] + static_cast<uint64_t>(p) * rb;
+      }
+    }
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bar[st], rb);
+      bulk_load(stage_buf + st * stage_bytes, a.x[s] + static_cast<uint64_t>(t) * rb, rb, &bar[st]);
+    }
+  };
+  int inflight = 0;
+  for (int st = 0; st < kDispStages && blockIdx.x + st * stride < rows; ++st, ++inflight) issue(blockIdx.x + st * stride, st);
+  __syncwarp();
+  int i = 0;
+  for (uint64_t row = blockIdx.x; row < rows; row += stride, ++i) {
+    const int st = i % kDispStages;
+    int ok = 1;
+    if (lane == 0) {
+      ok = mbar_wait_bounded(&bar[st], (i / kDispStages) & 1) ? 1 : 0;
+      if (ok) {
+        for (int k = 0; k < a.topk; ++k)
+          if (dst[st][k] != nullptr) bulk_store(dst[st][k], stage_buf + st * stage_bytes, rb);
+        bulk_commit();
+      }
+    }
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    if (!ok) {
+      if (lane == 0) {
+        report(a.status, COLL_DEV_TIMEOUT, 1);
+        bulk_wait_all();
+        for (int k = 1; k < inflight; ++k)
+          mbar_wait_bounded(&bar[(i + k) % kDispStages], ((i + k) / kDispStages) & 1);
+      }
+      return;
+    }
+    --inflight;
+    const uint64_t nxt = row + kDispStages * stride;
+    if (nxt < rows) {
+      if (lane == 0) bulk_wait_read<0>();
+      __syncwarp();  // the stage and its destination list are free again
+      issue(nxt, st);
+      ++inflight;
+      __syncwarp();
+    }
+  }
+  if (lane == 0) bulk_wait_all();
+  report_warp(a.status, COLL_DEV_SPLIT_OVERFLOW, bad);
+}
+
 static int pick_unit(uint64_t bits) {
   if ((bits & 15) == 0) return 16;
   if ((bits & 7) == 0) return 8;
@@ -268,6 +351,26 @@ int launch_moe_dispatch(const MoeMoveArgs& a, cudaStream_t s) {
   if (rows == 0 || a.row_bytes == 0) return COLL_OK;
   uint64_t bits = a.row_bytes;
   for (int r = 0; r < a.n; ++r) bits |= reinterpret_cast<uintptr_t>(a.x[r]) | reinterpret_cast<uintptr_t>(a.y[r]);
+  // whole rows through shared memory once there are enough of them
+  const uint32_t stage_bytes = static_cast<uint32_t>((a.row_bytes + 127) / 128 * 128);
+  const int64_t per_sm = std::max<int64_t>(1, (200 * 1024) / (kDispStages * static_cast<int64_t>(stage_bytes)));
+  const int64_t tma_grid = static_cast<int64_t>(num_sms()) * per_sm;
+  if ((bits & 15) == 0 && a.row_bytes <= kDispMaxRow && rows >= 4 * tma_grid) {
+    const size_t smem = static_cast<size_t>(kDispStages) * stage_bytes;
+    static int smem_set[COLL_MAX_RANKS] = {0};  // per device: largest size enabled so far
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= COLL_MAX_RANKS) dev = 0;
+    if (smem > 48 * 1024 && smem_set[dev] < static_cast<int>(smem)) {
+      const cudaError_t e =
+          cudaFuncSetAttribute(k_moe_dispatch_tma, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e != cudaSuccess) return launch_status(e);
+      smem_set[dev] = static_cast<int>(smem);
+    }
+    launch_pdl(k_moe_dispatch_tma, dim3(static_cast<unsigned>(std::min<int64_t>(rows, tma_grid))), dim3(32), smem, s, a,
+               stage_bytes);
+    return launch_status(cudaGetLastError());
+  }
   const unsigned grid = move_grid(rows);
   switch (pick_unit(bits)) {
     case 16: launch_pdl(k_moe_dispatch<16>, dim3(grid), dim3(kMoveThreads), 0, s, a); break;
@@ -295,23 +398,37 @@ __global__ void __launch_bounds__(kMoveThreads) k_moe_combine(const __grid_const
   const int64_t rows = static_cast<int64_t>(a.n) * a.tokens;
   const uint64_t relems = a.row_bytes / ES;
   int bad = 0;
+  // (expert, row, weight) of row `row`, choice threadIdx.x; fetched one row
+  // ahead so that their latency overlaps the streaming of the current row
+  int m_e = 0;
+  int64_t m_p = 0;
+  float m_w = 0.f;
+  auto fetch = [&](int64_t row) {
+    if (threadIdx.x < topk && row < rows) {
+      const int s = static_cast<int>(row / a.tokens);
+      const int t = static_cast<int>(row % a.tokens);
+      const int64_t j = static_cast<int64_t>(t) * topk + threadIdx.x;
+      m_e = a.ids[s][j];
+      m_p = a.pos[s][j];
+      m_w = a.w[s][j];
+    }
+  };
+  fetch(blockIdx.x);
   for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
     const int s = static_cast<int>(row / a.tokens);
     const int t = static_cast<int>(row % a.tokens);
     if (threadIdx.x < topk) {
-      const int64_t j = static_cast<int64_t>(t) * topk + threadIdx.x;
-      const int e = a.ids[s][j];
-      const int64_t p = a.pos[s][j];
-      const int d = e / a.epr;
-      wk[threadIdx.x] = a.w[s][j];
-      if (e < 0 || d >= a.n || p < 0 || p >= a.capacity) {
+      const int d = m_e / a.epr;
+      wk[threadIdx.x] = m_w;
+      if (m_e < 0 || d >= a.n || m_p < 0 || m_p >= a.capacity) {
         src[threadIdx.x] = nullptr;
         ++bad;
       } else {
-        src[threadIdx.x] = a.x[d] + static_cast<uint64_t>(p) * a.row_bytes;
+        src[threadIdx.x] = a.x[d] + static_cast<uint64_t>(m_p) * a.row_bytes;
       }
     }
     __syncthreads();
+    fetch(row + gridDim.x);
     char* out = a.y[s] + static_cast<uint64_t>(t) * a.row_bytes;
     if constexpr (VEC && TK > 0) {
       const char* sp[TK];

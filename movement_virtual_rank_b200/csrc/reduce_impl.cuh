@@ -124,8 +124,6 @@ __global__ void __launch_bounds__(kThreads) k_reduce_scalar(const __grid_constan
 // writes the finished chunk to rank c's output.
 template <int DT, int OP, bool VEC>
 __global__ void __launch_bounds__(kThreads) k_ring_rs(const __grid_constant__ RingStepArgs a) {
-  pdl_wait();
-  pdl_trigger();
   using A = typename Elem<DT>::A;
   using S = typename Elem<DT>::S;
   constexpr int VN = Vec<DT>::kN;
@@ -143,10 +141,13 @@ __global__ void __launch_bounds__(kThreads) k_ring_rs(const __grid_constant__ Ri
   const bool last = a.k == a.n - 1;
   A* part_buf = reinterpret_cast<A*>(a.partial);
   const uint64_t stride = static_cast<uint64_t>(parts) * blockDim.x;
+  const uint64_t v0 = static_cast<uint64_t>(part) * blockDim.x + threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   uint64_t scalar_from = lo;
   if constexpr (VEC) {
     const uint64_t nv = (hi - lo) / VN;
-    for (uint64_t v = static_cast<uint64_t>(part) * blockDim.x + threadIdx.x; v < nv; v += stride) {
+    for (uint64_t v = v0; v < nv; v += stride) {
       const uint64_t e = lo + v * VN;
       Vec<DT> acc;
       if (first) {

@@ -121,9 +121,6 @@ __global__ void __launch_bounds__(kRingLLThreads) k_ring_ll(const __grid_constan
           return false;
         }
       }
-      // back off before re-reading: thousands of pollers must not crowd out
-      // the lines they are waiting for in L2
-      __nanosleep(it < 4 ? 32u : 256u);
 #pragma unroll
       for (int i = 0; i < NG; ++i)
         if (!(x[i].y == f && x[i].w == f)) x[i] = ld_volatile16(p + i);
@@ -167,21 +164,44 @@ __global__ void __launch_bounds__(kRingLLThreads) k_ring_ll(const __grid_constan
     }
   };
 
+  // The rank's own inputs are final before the kernel starts, so the values
+  // it adds at the first kPreload reduce-scatter steps are fetched up front:
+  // each hop then costs only the LL hand-off, not an extra trip to DRAM after
+  // the poll succeeds.  (The steps are unrolled so the values stay in
+  // registers.)
+  constexpr int kPreload = 8;
   const uint64_t stride = static_cast<uint64_t>(a.groups) * blockDim.x * VN;
   for (uint64_t e = (static_cast<uint64_t>(g) * blockDim.x + threadIdx.x) * VN; alive && e < a.seg; e += stride) {
-    A p[VN], x[VN];
-    // reduce-scatter phase
-    own((r - 1 + n) % n, e, p);
-    send(0, e, p);
-    for (int k = 1; k < n && alive; ++k) {
-      const int c = ((r - 1 - k) % n + n) % n;
-      if (!recv(k - 1, e, p)) {
-        alive = false;
-        break;
-      }
-      own(c, e, x);
+    A p[VN];
+    uint4 pre[kPreload];
 #pragma unroll
-      for (int i = 0; i < VN; ++i) p[i] = op_step<OP>(p[i], x[i]);
+    for (int k = 0; k < kPreload; ++k) {
+      pre[k] = make_uint4(0, 0, 0, 0);
+      if (k < n) {
+        const int c = ((r - 1 - k) % n + n) % n;
+        const uint64_t gi = static_cast<uint64_t>(c) * a.seg + e;
+        const uint64_t end = min(static_cast<uint64_t>(c) * a.seg + a.seg, a.count);
+        if (gi + VN <= end) pre[k] = ld16(a.in[r] + gi * ES);
+      }
+    }
+    // the values rank r adds at step k (chunk c): preloaded, or read now
+    auto own_at = [&](const uint4& v, int c, A (&out)[VN]) {
+      const uint64_t gi = static_cast<uint64_t>(c) * a.seg + e;
+      const uint64_t end = min(static_cast<uint64_t>(c) * a.seg + a.seg, a.count);
+      if (gi + VN <= end) {
+        Vec<DT> w;
+        widen16<DT>(v, w);
+#pragma unroll
+        for (int i = 0; i < VN; ++i) out[i] = w.v[i];
+      } else {
+        own(c, e, out);
+      }
+    };
+    // one reduce-scatter step k >= 1: receive, add my values, (round,) send
+    auto rs_step = [&](int k, const A (&xv)[VN]) -> bool {
+      if (!recv(k - 1, e, p)) return false;
+#pragma unroll
+      for (int i = 0; i < VN; ++i) p[i] = op_step<OP>(p[i], xv[i]);
       if (k == n - 1) {
         // complete on rank r: round once; what travels on is the rounded value
         Vec<DT> w;
@@ -194,6 +214,22 @@ __global__ void __launch_bounds__(kRingLLThreads) k_ring_ll(const __grid_constan
         put(r, e, p);
       }
       send(k, e, p);
+      return true;
+    };
+    // reduce-scatter phase
+    own_at(pre[0], (r - 1 + n) % n, p);
+    send(0, e, p);
+#pragma unroll
+    for (int k = 1; k < kPreload; ++k) {
+      if (k >= n || !alive) break;
+      A xv[VN];
+      own_at(pre[k], ((r - 1 - k) % n + n) % n, xv);
+      alive = rs_step(k, xv);
+    }
+    for (int k = kPreload; k < n && alive; ++k) {
+      A xv[VN];
+      own(((r - 1 - k) % n + n) % n, e, xv);
+      alive = rs_step(k, xv);
     }
     // all-gather phase
     for (int j = 1; j < n && alive; ++j) {

@@ -192,3 +192,43 @@ def test_moe_workload():
     for s in range(n):
         got = from_dev(out[s], "bf16").reshape(tokens, hidden)[sel[s]].reshape(-1)
         assert np.array_equal(got, wc[s]), s
+
+
+@pytest.mark.parametrize("dtype,n,tokens,topk,experts,hidden", [
+    ("bf16", 4, 1024, 4, 16, 4096), ("fp32", 3, 700, 3, 9, 4000)])
+def test_dispatch_bulk_copy_path(dtype, n, tokens, topk, experts, hidden):
+    """Enough rows per CTA for the bulk-copy dispatch: rows land exactly where
+    the oracle puts them; a receive buffer a few rows short reports exactly
+    the rows that do not fit and writes nothing outside it."""
+    need_gpu()
+    ids, ws = W.moe_routing(tokens, experts, topk, n)
+    xs = W.ranks_values(W.W_MISC, n, tokens * hidden, dtype, "normal", salt=hidden + n)
+    dids, pos, wsc, wpos = check_route(ids, experts)
+    per_dest = wsc.sum(axis=0)
+    cap = int(per_dest.max())
+    xd = [to_dev(x, dtype) for x in xs]
+    recv = [torch.zeros(cap * hidden, dtype=xd[0].dtype, device="cuda") for _ in range(n)]
+    st = status_tensor()
+    M.coll_moe_dispatch(xd, dids, pos, recv, experts, status=st)
+    torch.cuda.synchronize()
+    assert st.tolist() == [0, 0]
+    want = oracle.moe_dispatch(xs, ids, wpos, [np.zeros(cap * hidden, dtype=xs[0].dtype) for _ in range(n)],
+                               experts, hidden)
+    for d in range(n):
+        assert np.array_equal(from_dev(recv[d], dtype), want[d]), d
+    short = cap - 5
+    guard = [torch.full(((short + 2) * hidden,), 7.0, dtype=xd[0].dtype, device="cuda") for _ in range(n)]
+    small = [g[:short * hidden] for g in guard]
+    st.zero_()
+    M.coll_moe_dispatch(xd, dids, pos, small, experts, status=st)
+    torch.cuda.synchronize()
+    lost = int(sum(max(0, int(c) - short) for c in per_dest))
+    assert st.tolist() == [M.DEV_SPLIT_OVERFLOW, lost]
+    fill = from_dev(torch.full(((short + 2) * hidden,), 7.0, dtype=xd[0].dtype, device="cuda"), dtype)
+    for d in range(n):
+        # rows the destination receives and that fit are written; every other
+        # row of the buffer and its guard rows keep the fill value
+        k = min(int(per_dest[d]), short) * hidden
+        expect = fill.copy()
+        expect[:k] = want[d][:k]
+        assert np.array_equal(from_dev(guard[d], dtype), expect), d

@@ -280,3 +280,44 @@ def test_broadcast_bulk_copy_sizes(count):
     torch.cuda.synchronize()
     for q in range(n):
         assert np.array_equal(from_dev(bufs[q], "int32"), xs[5])
+
+
+def test_copy_jobs_bulk_copy_path():
+    """Copy lists of 29 MB and more take the bulk-copy path: scatter of
+    8 x 4 MiB, all-to-all of 8 x 8 MiB, and an all-to-all-v with ragged row
+    counts, all checked on the device against their definitions."""
+    need_gpu()
+    n = 8
+    c = 2 << 20  # bf16 elements per rank block (4 MiB)
+    full = torch.randn(n * c, device="cuda").to(torch.bfloat16)
+    recv = [torch.empty(c, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+    M.coll_scatter(full, recv, 3)
+    torch.cuda.synchronize()
+    for r in range(n):
+        assert torch.equal(recv[r].view(torch.int16), full[r * c:(r + 1) * c].view(torch.int16))
+    blk = 1 << 19
+    send = [torch.randn(n * blk, device="cuda").to(torch.bfloat16) for _ in range(n)]
+    out = [torch.empty_like(t) for t in send]
+    M.coll_all_to_all(send, out)
+    torch.cuda.synchronize()
+    for d in range(n):
+        for s in range(n):
+            assert torch.equal(out[d][s * blk:(s + 1) * blk].view(torch.int16),
+                               send[s][d * blk:(d + 1) * blk].view(torch.int16))
+    row = 1024
+    sc = W.random_splits(n, 600, salt=99)
+    sd = np.zeros_like(sc)
+    sd[:, 1:] = np.cumsum(sc, axis=1)[:, :-1]
+    rc = sc.T.copy()
+    rd = np.zeros_like(rc)
+    rd[:, 1:] = np.cumsum(rc, axis=1)[:, :-1]
+    vs = [torch.randn(max(1, int(sc[s].sum())) * row, device="cuda").to(torch.bfloat16) for s in range(n)]
+    vr = [torch.zeros(max(1, int(rc[d].sum())) * row, dtype=torch.bfloat16, device="cuda") for d in range(n)]
+    assert int(sc.sum()) * row * 2 >= 29 << 20
+    M.coll_all_to_all_v(vs, vr, sc, sd, rd, row)
+    torch.cuda.synchronize()
+    for s in range(n):
+        for d in range(n):
+            k = int(sc[s, d]) * row
+            a, b = int(sd[s, d]) * row, int(rd[d, s]) * row
+            assert torch.equal(vr[d][b:b + k].view(torch.int16), vs[s][a:a + k].view(torch.int16)), (s, d)
