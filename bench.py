@@ -262,10 +262,12 @@ def build_ll_sweep(M, oracle, sizes=None):
 
 
 def build_ring_compare(M, oracle):
-    """The ring all-reduce three ways on the TP-decode shapes (8 virtual ranks,
+    """The ring all-reduce four ways on the TP-decode shapes (8 virtual ranks,
     bf16): one launch per ring step (RING), one cooperative launch with LL
-    packets between ranks (RING_LL), and the stream-ordered packet path of the
-    LL sweep (per-rank LL pack, packetised two-shot, per-rank unpack)."""
+    packets between ranks (RING_LL), one launch of 8-CTA clusters with the
+    hops over distributed shared memory (RING_CLUSTER), and the
+    stream-ordered packet path of the LL sweep (per-rank LL pack, packetised
+    two-shot, per-rank unpack)."""
     import torch
     n = 8
     ops = []
@@ -274,8 +276,9 @@ def build_ring_compare(M, oracle):
         count = tokens * hidden
         S = count * 2
         send = [_dev(x, torch.bfloat16) for x in xs]
-        for algo, aname, launches in ((M.RING, "ring", 2 * (n - 1)), (M.RING_LL, "ring_ll", 1)):
-            need = M.coll_all_reduce_workspace_size(n, count, torch.bfloat16, algo)
+        for algo, aname, launches in ((M.RING, "ring", 2 * (n - 1)), (M.RING_LL, "ring_ll", 1),
+                                      (M.RING_CLUSTER, "ring_cluster", 1)):
+            need = max(64, M.coll_all_reduce_workspace_size(n, count, torch.bfloat16, algo))
             ops.append(Op(f"all_reduce/{aname}",
                           lambda b, algo=algo: (lambda: M.coll_all_reduce(b["send"], b["recv"], algo=algo,
                                                                            workspace=b["ws"])),
@@ -304,6 +307,7 @@ def build_ring_compare(M, oracle):
                       inputs=["send"], outputs=["recv"], kernel="all_reduce/ll_pack_ar_unpack"))
     return ops, {"workload": "ring_compare_8vr", "virtual_ranks": n, "shapes": W.tp_decode_shapes(),
                  "variants": ["ring (launch per step)", "ring_ll (one launch, LL packets)",
+                              "ring_cluster (one launch, cluster DSMEM hops)",
                               "LL pack + packetised two-shot + unpack (stream-ordered)"]}
 
 
@@ -485,15 +489,25 @@ def lib_digest():
     return h.hexdigest()[:16]
 
 
+def sources_digest(files) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for fn in sorted(files):
+        with open(os.path.join(ROOT, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
 def traffic_for(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, if taken on this exact source."""
+    """DRAM bytes per call from profiles/traffic.json, if the counters were
+    taken on the kernel's current source (its files' digest still matches)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
     e = d.get(workload, {}).get(kernel)
-    if e and e.get("source_digest") == lib_digest():
-        return e.get("dram_bytes_per_launch")
+    if e and e.get("digest") == sources_digest(e.get("sources", [])):
+        return e.get("dram_bytes_per_call")
     return None
 
 

@@ -79,7 +79,8 @@ typedef enum {
   COLL_ALGO_ONESHOT = 1, /* every rank reads all N inputs itself            */
   COLL_ALGO_TWOSHOT = 2, /* owner s reduces segment s, sends it to everyone */
   COLL_ALGO_RING = 3,    /* 2(N-1) neighbour steps, one launch per step     */
-  COLL_ALGO_RING_LL = 4  /* the same ring in one launch, LL packets between ranks */
+  COLL_ALGO_RING_LL = 4, /* the same ring in one launch, LL packets between ranks */
+  COLL_ALGO_RING_CLUSTER = 5 /* the same ring, ranks = CTAs of a cluster, hops over DSMEM */
 } coll_algo_t;
 typedef enum { COLL_PROTO_SIMPLE = 0, COLL_PROTO_LL = 1, COLL_PROTO_LL128 = 2 } coll_proto_t;
 
@@ -167,9 +168,20 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    256-byte aligned) must be zero-filled once before its first use and
  *    serves one call at a time; the library keeps a call counter in it.
  *    Buffers that are not 16-byte aligned take the RING path.
+ *  RING_CLUSTER: the RING schedule, chunk order and rounding (bit-identical
+ *    result) in one launch of thread-block clusters of N CTAs, CTA r playing
+ *    virtual rank r: each hop is an asynchronous store into the next CTA's
+ *    shared memory over the SM-to-SM network that completes that CTA's
+ *    mbarrier, so the partials never touch HBM.  The clusters are about as
+ *    many as fit on the GPU at once and walk the message tile by tile, two
+ *    tiles in flight.  Needs 2 <= N <= 8 and 16-byte aligned buffers;
+ *    otherwise, if a RING-sized `workspace` is given, the call takes the RING
+ *    path, else it returns COLL_ERR_UNSUPPORTED.  `workspace` is optional:
+ *    when at least 24 bytes are given, bytes 16..23 receive the status pair
+ *    (COLL_DEV_TIMEOUT if a bounded wait ran out).
  *  AUTO picks TWOSHOT.  ONESHOT and TWOSHOT ignore `workspace`.
- * In place (recv[r] == send[r]) is allowed for TWOSHOT, RING, RING_LL and
- * AUTO. */
+ * In place (recv[r] == send[r]) is allowed for TWOSHOT, RING, RING_LL,
+ * RING_CLUSTER and AUTO. */
 COLL_API int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size_t count,
                     coll_dtype_t dtype, coll_op_t op, coll_algo_t algo, void* workspace,
                     size_t workspace_bytes, coll_stream_t stream);

@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libmvrcoll.so")
 
 BF16, FP16, FP32, INT32 = 0, 1, 2, 3
 SUM, MAX, MIN, PROD = 0, 1, 2, 3
-ALGO_AUTO, ONESHOT, TWOSHOT, RING, RING_LL = 0, 1, 2, 3, 4
+ALGO_AUTO, ONESHOT, TWOSHOT, RING, RING_LL, RING_CLUSTER = 0, 1, 2, 3, 4, 5
 SIMPLE, LL, LL128 = 0, 1, 2
 DEV_OK, DEV_FLAG_MISMATCH, DEV_TIMEOUT, DEV_SPLIT_OVERFLOW, DEV_BAD_ROUTE = 0, 1, 2, 3, 4
 MAX_RANKS = 64
@@ -30,7 +30,8 @@ MAX_RANKS = 64
 _DTYPES = {torch.bfloat16: BF16, torch.float16: FP16, torch.float32: FP32, torch.int32: INT32}
 _ESIZE = {BF16: 2, FP16: 2, FP32: 4, INT32: 4}
 OPS = {"sum": SUM, "max": MAX, "min": MIN, "prod": PROD}
-ALGOS = {"auto": ALGO_AUTO, "oneshot": ONESHOT, "twoshot": TWOSHOT, "ring": RING, "ring_ll": RING_LL}
+ALGOS = {"auto": ALGO_AUTO, "oneshot": ONESHOT, "twoshot": TWOSHOT, "ring": RING, "ring_ll": RING_LL,
+         "ring_cluster": RING_CLUSTER}
 PROTOS = {"simple": SIMPLE, "ll": LL, "ll128": LL128}
 
 
@@ -237,9 +238,11 @@ def coll_all_reduce_workspace_size(nranks: int, count: int, dtype: torch.dtype, 
 
 
 def coll_all_reduce(send, recv, op="sum", algo=TWOSHOT, workspace: torch.Tensor | None = None, stream=None):
-    """``workspace`` (RING and RING_LL): a CUDA tensor of at least
-    coll_all_reduce_workspace_size() bytes, zero-filled before its first
-    RING_LL use; allocated (zeroed) here when omitted."""
+    """``workspace``: a CUDA tensor passed through to the library when given.
+    RING and RING_LL need one of at least coll_all_reduce_workspace_size()
+    bytes (zero-filled before its first RING_LL use) and get a zeroed one
+    allocated here when it is omitted; RING_CLUSTER uses one, when given, for
+    its status pair and its fallback to RING."""
     algo = ALGOS[algo] if isinstance(algo, str) else int(algo)
     send = _ranks(send, "send", send[0].dtype)
     recv = _ranks(recv, "recv", send[0].dtype)
@@ -249,10 +252,10 @@ def coll_all_reduce(send, recv, op="sum", algo=TWOSHOT, workspace: torch.Tensor 
     if _same_numel(recv, "recv") != n:
         raise ValueError("send and recv sizes differ")
     ws_ptr, ws_bytes = None, 0
-    if algo in (RING, RING_LL):
+    if workspace is None and algo in (RING, RING_LL):
         need = coll_all_reduce_workspace_size(len(send), n, send[0].dtype, algo)
-        if workspace is None:
-            workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=send[0].device)
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=send[0].device)
+    if workspace is not None:
         ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     ps, _k1 = _ptrs(send)
     pr, _k2 = _ptrs(recv)

@@ -32,6 +32,19 @@ int launch_status(cudaError_t e) {
   return COLL_ERR_CUDA;
 }
 
+int allow_dynamic_smem(const void* fn, size_t bytes, int* done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= COLL_MAX_RANKS) dev = 0;
+  if (done[dev] >= static_cast<int>(bytes)) return COLL_OK;
+  const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();  // reported here; keep it from surfacing in a later call
+    return launch_status(e);
+  }
+  done[dev] = static_cast<int>(bytes);
+  return COLL_OK;
+}
+
 int num_sms() {
   static std::atomic<int> cache[COLL_MAX_RANKS];
   int dev = 0;
@@ -296,7 +309,7 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
                     coll_op_t op, coll_algo_t algo, void* workspace, size_t workspace_bytes, coll_stream_t stream) {
   const int es = elem_size(dtype);
   if (!es) return COLL_ERR_UNSUPPORTED;
-  if (!valid_op(op) || algo < COLL_ALGO_AUTO || algo > COLL_ALGO_RING_LL) return COLL_ERR_UNSUPPORTED;
+  if (!valid_op(op) || algo < COLL_ALGO_AUTO || algo > COLL_ALGO_RING_CLUSTER) return COLL_ERR_UNSUPPORTED;
   if (!valid_n(nranks) || !all_nonnull(send, nranks) || !all_nonnull(recv, nranks)) return COLL_ERR_INVALID_ARG;
   const size_t bytes = count * es;
   if (bytes == 0) return COLL_OK;
@@ -318,6 +331,30 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
   bool vec = true;
   for (int r = 0; r < nranks; ++r) vec = vec && al16(send[r]) && al16(recv[r]);
   const size_t seg = seg_elems(count, nranks, es);
+  if (algo == COLL_ALGO_RING_CLUSTER) {
+    if (vec && ring_cluster_supported(nranks)) {
+      if (workspace != nullptr && workspace_bytes >= 24 && !al16(workspace)) return COLL_ERR_WORKSPACE;
+      for (int r = 0; r < nranks; ++r)
+        if (workspace != nullptr && workspace_bytes >= 24 &&
+            (overlap(workspace, 24, send[r], bytes) || overlap(workspace, 24, recv[r], bytes)))
+          return COLL_ERR_ALIAS;
+      const char* in[COLL_MAX_RANKS];
+      char* out[COLL_MAX_RANKS];
+      for (int r = 0; r < nranks; ++r) {
+        in[r] = static_cast<const char*>(send[r]);
+        out[r] = static_cast<char*>(recv[r]);
+      }
+      int* status = (workspace != nullptr && workspace_bytes >= 24)
+                        ? reinterpret_cast<int*>(static_cast<char*>(workspace) + 16)
+                        : nullptr;
+      return launch_ring_cluster(in, out, nranks, count, dtype, op, status, S(stream));
+    }
+    const size_t need = ring_ws(count);
+    if (workspace == nullptr || workspace_bytes < need || !al16(workspace)) return COLL_ERR_UNSUPPORTED;
+    for (int r = 0; r < nranks; ++r)
+      if (overlap(workspace, need, send[r], bytes) || overlap(workspace, need, recv[r], bytes)) return COLL_ERR_ALIAS;
+    algo = COLL_ALGO_RING;
+  }
   if (algo == COLL_ALGO_RING_LL) {
     if (vec) {
       const char* in[COLL_MAX_RANKS];

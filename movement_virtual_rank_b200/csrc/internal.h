@@ -16,6 +16,11 @@ constexpr int kBlockThreads = 256;  // threads per CTA of the element-wise kerne
 int num_sms();                      // SM count of the current device (cached)
 int elem_size(coll_dtype_t dt);     // 2 or 4, 0 for an unknown dtype
 int launch_status(cudaError_t e);   // COLL_OK or COLL_ERR_CUDA (remembers the error text)
+// Raise `fn`'s dynamic shared memory limit to at least `bytes` on the current
+// device (`done` holds one entry per device ordinal, the largest limit set so
+// far).  Called before every launch that uses dynamic shared memory, whatever
+// its size: the 48 KB default counts the kernel's static shared memory too.
+int allow_dynamic_smem(const void* fn, size_t bytes, int* done);
 
 // ----------------------------------------------------------- reductions ----
 struct ReduceArgs {
@@ -44,6 +49,9 @@ int launch_ring_rs_step(const RingStepArgs& a, coll_dtype_t dt, coll_op_t op, bo
 size_t ring_ll_workspace(int n, size_t count, int es);
 int launch_ring_ll(const char* const* in, char* const* out, int n, size_t count, coll_dtype_t dt, coll_op_t op,
                    void* workspace, int* status, cudaStream_t s);
+bool ring_cluster_supported(int n);
+int launch_ring_cluster(const char* const* in, char* const* out, int n, size_t count, coll_dtype_t dt, coll_op_t op,
+                        int* status, cudaStream_t s);
 int launch_wait_flag(const uint32_t* flag, uint32_t expect, uint32_t budget_us, int* status, cudaStream_t s);
 
 // ---------------------------------------------------------------- copies ----

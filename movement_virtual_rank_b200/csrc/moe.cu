@@ -188,11 +188,9 @@ __global__ void __launch_bounds__(kTile) k_moe_pos(const __grid_constant__ MoeRo
 int launch_moe_route(const MoeRouteArgs& a, cudaStream_t s) {
   const unsigned grid = static_cast<unsigned>(a.n * a.tiles);
   const size_t smem = static_cast<size_t>(a.n_experts) * kWords * sizeof(uint32_t);
-  if (smem > 48 * 1024) {
-    const cudaError_t e = cudaFuncSetAttribute(k_moe_count, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(smem));
-    if (e != cudaSuccess) return launch_status(e);
-  }
+  static int smem_set[COLL_MAX_RANKS] = {0};  // per device ordinal: largest limit set so far
+  const int ok = allow_dynamic_smem(reinterpret_cast<const void*>(k_moe_count), smem, smem_set);
+  if (ok != COLL_OK) return ok;
   launch_pdl(k_moe_count, dim3(grid), dim3(kTile), smem, s, a);  // tokens == 0 still zeroes the counts
   int st = launch_status(cudaGetLastError());
   if (st != COLL_OK) return st;
@@ -357,16 +355,9 @@ int launch_moe_dispatch(const MoeMoveArgs& a, cudaStream_t s) {
   const int64_t tma_grid = static_cast<int64_t>(num_sms()) * per_sm;
   if ((bits & 15) == 0 && a.row_bytes <= kDispMaxRow && rows >= 4 * tma_grid) {
     const size_t smem = static_cast<size_t>(kDispStages) * stage_bytes;
-    static int smem_set[COLL_MAX_RANKS] = {0};  // per device: largest size enabled so far
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= COLL_MAX_RANKS) dev = 0;
-    if (smem > 48 * 1024 && smem_set[dev] < static_cast<int>(smem)) {
-      const cudaError_t e =
-          cudaFuncSetAttribute(k_moe_dispatch_tma, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      if (e != cudaSuccess) return launch_status(e);
-      smem_set[dev] = static_cast<int>(smem);
-    }
+    static int smem_set[COLL_MAX_RANKS] = {0};  // per device ordinal: largest limit set so far
+    const int ok = allow_dynamic_smem(reinterpret_cast<const void*>(k_moe_dispatch_tma), smem, smem_set);
+    if (ok != COLL_OK) return ok;
     launch_pdl(k_moe_dispatch_tma, dim3(static_cast<unsigned>(std::min<int64_t>(rows, tma_grid))), dim3(32), smem, s, a,
                stage_bytes);
     return launch_status(cudaGetLastError());
@@ -398,37 +389,23 @@ __global__ void __launch_bounds__(kMoveThreads) k_moe_combine(const __grid_const
   const int64_t rows = static_cast<int64_t>(a.n) * a.tokens;
   const uint64_t relems = a.row_bytes / ES;
   int bad = 0;
-  // (expert, row, weight) of row `row`, choice threadIdx.x; fetched one row
-  // ahead so that their latency overlaps the streaming of the current row
-  int m_e = 0;
-  int64_t m_p = 0;
-  float m_w = 0.f;
-  auto fetch = [&](int64_t row) {
-    if (threadIdx.x < topk && row < rows) {
-      const int s = static_cast<int>(row / a.tokens);
-      const int t = static_cast<int>(row % a.tokens);
-      const int64_t j = static_cast<int64_t>(t) * topk + threadIdx.x;
-      m_e = a.ids[s][j];
-      m_p = a.pos[s][j];
-      m_w = a.w[s][j];
-    }
-  };
-  fetch(blockIdx.x);
   for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
     const int s = static_cast<int>(row / a.tokens);
     const int t = static_cast<int>(row % a.tokens);
     if (threadIdx.x < topk) {
-      const int d = m_e / a.epr;
-      wk[threadIdx.x] = m_w;
-      if (m_e < 0 || d >= a.n || m_p < 0 || m_p >= a.capacity) {
+      const int64_t j = static_cast<int64_t>(t) * topk + threadIdx.x;
+      const int e = a.ids[s][j];
+      const int64_t p = a.pos[s][j];
+      const int d = e / a.epr;
+      wk[threadIdx.x] = a.w[s][j];
+      if (e < 0 || d >= a.n || p < 0 || p >= a.capacity) {
         src[threadIdx.x] = nullptr;
         ++bad;
       } else {
-        src[threadIdx.x] = a.x[d] + static_cast<uint64_t>(m_p) * a.row_bytes;
+        src[threadIdx.x] = a.x[d] + static_cast<uint64_t>(p) * a.row_bytes;
       }
     }
     __syncthreads();
-    fetch(row + gridDim.x);
     char* out = a.y[s] + static_cast<uint64_t>(t) * a.row_bytes;
     if constexpr (VEC && TK > 0) {
       const char* sp[TK];

@@ -1,0 +1,423 @@
+// Ring all-reduce with the virtual ranks as the CTAs of one thread-block
+// cluster: the hop from rank r to rank r+1 goes over distributed shared
+// memory (the SM-to-SM network), not through HBM or a kernel boundary.
+//
+// The schedule, chunk order, fp32 partials and the single rounding are those
+// of coll_all_reduce(RING) (TP communication essay; NCCL's ring kernel named
+// in "From NCCL Ring LL to PCIe IPC AllReduce"), so the result is
+// bit-identical.  CTA r of a cluster of N plays virtual rank r; the segment
+// is cut into tiles of kRcThreads x VN elements per chunk, and the clusters
+// walk the tiles with a stride (persistent: about as many clusters as fit on
+// the GPU at once).  Thread t owns VN elements of each chunk of a tile.
+//
+// Hop transport.  For each of the 2N-2 hops of a tile the sender stores its
+// values straight into a slot of the receiver's shared memory with
+// st.async ... mbarrier::complete_tx, so the store itself completes the
+// receiver's mbarrier for that slot (release at cluster scope, no separate
+// fence or arrive).  The receiver armed that mbarrier with the slot's byte
+// count and waits on it (acquire at cluster scope).  Every slot is written
+// once per tile; two slot sets alternate between consecutive tiles, and a
+// split cluster barrier (arrive after a tile, wait one tile later) keeps a
+// sender from refilling a set before every receiver has read it.
+//
+// All of a ring's dependencies stay inside one cluster, whose CTAs the
+// hardware schedules together, so clusters may run in any order and in
+// waves.  Every wait is bounded: a CTA whose wait runs out raises
+// COLL_DEV_TIMEOUT, sets an abort word in every CTA of its cluster, stops
+// sending and receiving, still takes every cluster barrier, and before it
+// exits polls (bounded) the slots it still expects, so that no store is in
+// flight into it.  Only st.async stores and mbarrier updates cross CTAs;
+// there is no bulk copy and no multicast.
+#include <algorithm>
+
+#include "bulk.cuh"
+#include "common.cuh"
+#include "internal.h"
+
+namespace mvr {
+
+constexpr int kRcThreads = 128;
+constexpr int kRcMaxRanks = 8;                    // portable cluster size
+constexpr int kRcSlots = 2 * kRcMaxRanks - 2;     // hops per tile
+constexpr long long kRcBudgetCycles = 1ll << 28;  // about 0.14 s per wait
+constexpr long long kRcDrainCycles = 1ll << 17;   // about 70 us per slot, abort path only
+
+struct RingClusterArgs {
+  const char* in[kMaxRanks];
+  char* out[kMaxRanks];
+  uint64_t count, seg, tiles;
+  int n;
+  int* status;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_idx() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_count() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
+// shared::cluster address of my shared variable at `p` in CTA `rank`
+__device__ __forceinline__ uint32_t map_to(const void* p, uint32_t rank) {
+  uint32_t local = static_cast<uint32_t>(__cvta_generic_to_shared(p)), remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
+  return remote;
+}
+// 16 bytes into another CTA's shared memory, completing 16 bytes of the
+// transaction count of that CTA's mbarrier at `bar_addr`
+__device__ __forceinline__ void st_async16(uint32_t addr, const uint4& v, uint32_t bar_addr) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
+      "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar_addr)
+      : "memory");
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_volatile_smem(const uint32_t* p) {
+  return *reinterpret_cast<const volatile uint32_t*>(p);
+}
+__device__ __forceinline__ bool try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar))), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+template <int DT, int OP>
+__global__ void __launch_bounds__(kRcThreads) k_ring_cluster(const __grid_constant__ RingClusterArgs a) {
+  using A = typename Elem<DT>::A;
+  using S = typename Elem<DT>::S;
+  constexpr int VN = Vec<DT>::kN;  // elements per thread (16 bytes of input)
+  constexpr int NQ = VN / 4;       // 16-byte pieces of fp32 / int32 payload per thread
+  constexpr int ES = Elem<DT>::kSize;
+  constexpr uint64_t TE = static_cast<uint64_t>(kRcThreads) * VN;  // elements of a chunk per tile
+  constexpr uint32_t kSlotBytes = kRcThreads * NQ * 16;
+  extern __shared__ __align__(16) uint4 slot_buf[];  // [set][slot][thread][NQ]
+  __shared__ __align__(8) uint64_t bar[2][kRcSlots];
+  __shared__ uint32_t abort_word;
+  const int n = a.n;
+  const int slots = 2 * n - 2;
+  const int r = static_cast<int>(cluster_rank());
+  const uint64_t g = cluster_idx();
+  const uint64_t G = cluster_count();
+  const int tid = threadIdx.x;
+  // thread 0's record of the slots it armed and has not yet seen complete
+  // (bit 16*b + s), and the phase parity each set was last armed for (bit b);
+  // read only by the abort drain
+  uint32_t pending = 0, pending_par = 0;
+  if (tid == 0) {
+    abort_word = 0;
+    for (int b = 0; b < 2; ++b)
+      for (int s = 0; s < slots; ++s) mbar_init(&bar[b][s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int b = 0; b < 2; ++b)  // arm the slots of this cluster's first two tiles
+      if (g + b * G < a.tiles) {
+        for (int s = 0; s < slots; ++s) mbar_arrive_expect_tx(&bar[b][s], kSlotBytes);
+        pending |= ((1u << slots) - 1) << (16 * b);
+      }
+  }
+  cluster_sync_all();  // every CTA's barriers are armed before anyone stores into them
+  pdl_wait();
+  pdl_trigger();
+
+  const int nxt = (r + 1) % n;
+  const uint32_t next_slot0 = map_to(slot_buf, nxt);
+  const uint32_t next_bar0 = map_to(&bar[0][0], nxt);
+  bool alive = true;
+
+  auto chunk_lo = [&](int c) { return static_cast<uint64_t>(c) * a.seg; };
+  auto chunk_end = [&](int c) { return min(chunk_lo(c) + a.seg, a.count); };
+  auto own = [&](int c, uint64_t e, A (&v)[VN]) {
+    const uint64_t gi = chunk_lo(c) + e;
+    const uint64_t end = chunk_end(c);
+#pragma unroll
+    for (int i = 0; i < VN; ++i)
+      v[i] = gi + i < end ? widen1<DT>(*reinterpret_cast<const S*>(a.in[r] + (gi + i) * ES)) : A(0);
+  };
+  auto put = [&](int c, uint64_t e, const A (&v)[VN]) {
+    const uint64_t gi = chunk_lo(c) + e;
+    const uint64_t end = chunk_end(c);
+    if (gi + VN <= end) {
+      Vec<DT> w;
+#pragma unroll
+      for (int i = 0; i < VN; ++i) w.v[i] = v[i];
+      st16(a.out[r] + gi * ES, narrow16<DT>(w));
+    } else {
+#pragma unroll
+      for (int i = 0; i < VN; ++i)
+        if (gi + i < end) *reinterpret_cast<S*>(a.out[r] + (gi + i) * ES) = narrow1<DT>(v[i]);
+    }
+  };
+  auto to_bits = [](A x) -> uint32_t {
+    if constexpr (std::is_same<A, float>::value) return __float_as_uint(x);
+    else return static_cast<uint32_t>(x);
+  };
+  auto from_bits = [](uint32_t u) -> A {
+    if constexpr (std::is_same<A, float>::value) return __uint_as_float(u);
+    else return static_cast<A>(static_cast<int32_t>(u));
+  };
+  auto raise_abort = [&]() {
+    report(a.status, COLL_DEV_TIMEOUT, 1);
+    for (int q = 0; q < n; ++q) st_cluster_u32(map_to(&abort_word, q), 1u);
+  };
+  auto send = [&](int b, int s, const A (&v)[VN]) {
+    if (ld_volatile_smem(&abort_word) != 0) {
+      alive = false;
+      return;
+    }
+    const int si = b * slots + s;
+    const uint32_t base = next_slot0 + static_cast<uint32_t>((si * kRcThreads + tid) * NQ * 16);
+    const uint32_t bar_addr = next_bar0 + static_cast<uint32_t>((b * kRcSlots + s) * 8);
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+      st_async16(base + q * 16,
+                 make_uint4(to_bits(v[4 * q]), to_bits(v[4 * q + 1]), to_bits(v[4 * q + 2]), to_bits(v[4 * q + 3])),
+                 bar_addr);
+  };
+  // wait for slot s of set b (phase parity par) and read my part of it; thread 0
+  // then re-arms the slot for the tile two ahead when this cluster has one
+  auto recv = [&](int b, int s, uint32_t par, bool rearm, A (&v)[VN]) -> bool {
+    if (!try_wait_cluster(&bar[b][s], par)) {
+      const long long t0 = clock64();
+      while (!try_wait_cluster(&bar[b][s], par)) {
+        if (ld_volatile_smem(&abort_word) != 0) return false;
+        if (clock64() - t0 > kRcBudgetCycles) {
+          raise_abort();
+          return false;
+        }
+      }
+    }
+    const uint4* p = slot_buf + ((b * slots + s) * kRcThreads + tid) * NQ;
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      const uint4 x = p[q];
+      v[4 * q] = from_bits(x.x);
+      v[4 * q + 1] = from_bits(x.y);
+      v[4 * q + 2] = from_bits(x.z);
+      v[4 * q + 3] = from_bits(x.w);
+    }
+    if (tid == 0) {
+      pending &= ~(1u << (16 * b + s));
+      if (rearm) {
+        mbar_arrive_expect_tx(&bar[b][s], kSlotBytes);
+        pending |= 1u << (16 * b + s);
+        pending_par = (pending_par & ~(1u << b)) | ((par ^ 1u) << b);
+      }
+    }
+    return true;
+  };
+  // the 16-byte input vectors this rank adds at each reduce-scatter step of tile t
+  auto fetch = [&](uint64_t t, uint4 (&dst)[kRcMaxRanks]) {
+    const uint64_t e = t * TE + static_cast<uint64_t>(tid) * VN;
+#pragma unroll
+    for (int k = 0; k < kRcMaxRanks; ++k) {
+      dst[k] = make_uint4(0, 0, 0, 0);
+      if (k < n) {
+        const int c = ((r - 1 - k) % n + n) % n;
+        const uint64_t gi = chunk_lo(c) + e;
+        if (gi + VN <= chunk_end(c)) dst[k] = ld16(a.in[r] + gi * ES);
+      }
+    }
+  };
+
+  uint4 pre[kRcMaxRanks];
+  if (g < a.tiles) fetch(g, pre);
+  uint32_t it = 0;
+  for (uint64_t t = g; t < a.tiles; t += G, ++it) {
+    const int b = static_cast<int>(it & 1);
+    const uint32_t par = (it >> 1) & 1;
+    const bool rearm = t + 2 * G < a.tiles;
+    const uint64_t e = t * TE + static_cast<uint64_t>(tid) * VN;
+    uint4 nx[kRcMaxRanks];
+    if (t + G < a.tiles) fetch(t + G, nx);  // next tile's inputs, in flight during this one
+    else
+#pragma unroll
+      for (int k = 0; k < kRcMaxRanks; ++k) nx[k] = make_uint4(0, 0, 0, 0);
+
+    auto mine = [&](int k, A (&v)[VN]) {
+      const int c = ((r - 1 - k) % n + n) % n;
+      if (chunk_lo(c) + e + VN <= chunk_end(c)) {
+        Vec<DT> w;
+        widen16<DT>(pre[k], w);
+#pragma unroll
+        for (int i = 0; i < VN; ++i) v[i] = w.v[i];
+      } else {
+        own(c, e, v);
+      }
+    };
+
+    if (alive) {
+      A p[VN];
+      mine(0, p);
+      send(b, 0, p);
+#pragma unroll
+      for (int k = 1; k < kRcMaxRanks; ++k) {
+        if (k >= n || !alive) break;
+        A x[VN];
+        mine(k, x);
+        if (!recv(b, k - 1, par, rearm, p)) {
+          alive = false;
+          break;
+        }
+#pragma unroll
+        for (int i = 0; i < VN; ++i) p[i] = op_step<OP>(p[i], x[i]);
+        if (k == n - 1) {  // complete on this rank: one rounding, the rounded value travels on
+          Vec<DT> w;
+#pragma unroll
+          for (int i = 0; i < VN; ++i) w.v[i] = p[i];
+          Vec<DT> back;
+          widen16<DT>(narrow16<DT>(w), back);
+#pragma unroll
+          for (int i = 0; i < VN; ++i) p[i] = back.v[i];
+          put(r, e, p);
+        }
+        send(b, k, p);
+      }
+      for (int j = 1; j < n && alive; ++j) {  // all-gather hops
+        if (!recv(b, n - 2 + j, par, rearm, p)) {
+          alive = false;
+          break;
+        }
+        put(((r - j) % n + n) % n, e, p);
+        if (j < n - 1) send(b, n - 1 + j, p);
+      }
+    }
+    // this CTA has read set b of this tile; before the next tile refills the
+    // other set, every CTA must have read that one (their arrive one tile ago)
+    if (it > 0) cluster_wait();
+    cluster_arrive();
+#pragma unroll
+    for (int k = 0; k < kRcMaxRanks; ++k) pre[k] = nx[k];
+  }
+  if (it > 0) cluster_wait();
+  if (tid == 0 && ld_volatile_smem(&abort_word) != 0) {
+    // abort path: let any store still in flight into this CTA land first
+    for (int b = 0; b < 2; ++b)
+      for (int s = 0; s < slots; ++s)
+        if (pending & (1u << (16 * b + s))) {
+          const long long t0 = clock64();
+          while (!try_wait_cluster(&bar[b][s], (pending_par >> b) & 1u) && clock64() - t0 < kRcDrainCycles) {
+          }
+        }
+  }
+}
+
+// clusters of n CTAs that fit on the device at once (cached per device and n)
+template <int DT, int OP>
+static uint64_t resident_clusters(int n, size_t smem, int dev) {
+  static int cache[COLL_MAX_RANKS][kRcMaxRanks + 1] = {};
+  const bool cached = dev >= 0 && dev < COLL_MAX_RANKS;
+  if (cached && cache[dev][n] > 0) return static_cast<uint64_t>(cache[dev][n]);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(n));
+  cfg.blockDim = dim3(kRcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(n);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int v = 0;
+  if (cudaOccupancyMaxActiveClusters(&v, k_ring_cluster<DT, OP>, &cfg) != cudaSuccess || v <= 0) {
+    (void)cudaGetLastError();
+    v = std::max(1, num_sms() / n);
+  }
+  if (cached) cache[dev][n] = v;
+  return static_cast<uint64_t>(v);
+}
+
+template <int DT, int OP>
+static int launch_ring_cluster_t(RingClusterArgs a, cudaStream_t s) {
+  constexpr int VN = Vec<DT>::kN;
+  const uint64_t per_tile = static_cast<uint64_t>(kRcThreads) * VN;
+  a.tiles = std::max<uint64_t>(1, (a.seg + per_tile - 1) / per_tile);
+  const size_t smem = static_cast<size_t>(2) * (2 * a.n - 2) * kRcThreads * VN * 4;
+  static int smem_set[COLL_MAX_RANKS] = {0};  // per device ordinal: largest limit set so far
+  const int st = allow_dynamic_smem(reinterpret_cast<const void*>(k_ring_cluster<DT, OP>), smem, smem_set);
+  if (st != COLL_OK) return st;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  static bool carveout_set[COLL_MAX_RANKS] = {};  // two CTAs of up to 112 KB share an SM
+  if (dev >= 0 && dev < COLL_MAX_RANKS && !carveout_set[dev]) {
+    if (cudaFuncSetAttribute(k_ring_cluster<DT, OP>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+      (void)cudaGetLastError();  // a preference only
+    carveout_set[dev] = true;
+  }
+  const uint64_t clusters = std::min<uint64_t>(a.tiles, resident_clusters<DT, OP>(a.n, smem, dev));
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(clusters * a.n));
+  cfg.blockDim = dim3(kRcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(a.n);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_ring_cluster<DT, OP>, a);
+  if (e != cudaSuccess) (void)cudaGetLastError();  // reported here; keep it from surfacing in a later call
+  return launch_status(e);
+}
+
+template <int DT>
+static int launch_ring_cluster_dt(const RingClusterArgs& a, coll_op_t op, cudaStream_t s) {
+  switch (op) {
+    case COLL_SUM: return launch_ring_cluster_t<DT, COLL_SUM>(a, s);
+    case COLL_MAX: return launch_ring_cluster_t<DT, COLL_MAX>(a, s);
+    case COLL_MIN: return launch_ring_cluster_t<DT, COLL_MIN>(a, s);
+    case COLL_PROD: return launch_ring_cluster_t<DT, COLL_PROD>(a, s);
+  }
+  return COLL_ERR_UNSUPPORTED;
+}
+
+bool ring_cluster_supported(int n) { return n >= 2 && n <= kRcMaxRanks; }
+
+int launch_ring_cluster(const char* const* in, char* const* out, int n, size_t count, coll_dtype_t dt, coll_op_t op,
+                        int* status, cudaStream_t s) {
+  RingClusterArgs a{};
+  for (int r = 0; r < n; ++r) {
+    a.in[r] = in[r];
+    a.out[r] = out[r];
+  }
+  const int es = elem_size(dt);
+  const size_t g = 16 / es;
+  a.seg = ((count + n - 1) / n + g - 1) / g * g;
+  a.count = count;
+  a.n = n;
+  a.status = status;
+  switch (dt) {
+    case COLL_BF16: return launch_ring_cluster_dt<COLL_BF16>(a, op, s);
+    case COLL_FP16: return launch_ring_cluster_dt<COLL_FP16>(a, op, s);
+    case COLL_FP32: return launch_ring_cluster_dt<COLL_FP32>(a, op, s);
+    case COLL_INT32: return launch_ring_cluster_dt<COLL_INT32>(a, op, s);
+  }
+  return COLL_ERR_UNSUPPORTED;
+}
+
+}  // namespace mvr
