@@ -106,6 +106,9 @@ def _dev(a: np.ndarray, dtype):
     return torch.from_numpy(np.ascontiguousarray(a).view(view).copy()).view(dtype).cuda()
 
 
+FORM_NAMES = {1: "oneshot", 2: "twoshot", 4: "ring_ll", 5: "ring_cluster", 6: "ring_steps"}
+
+
 def build_tp_decode(M, oracle):
     import torch
     ops = []
@@ -114,9 +117,11 @@ def build_tp_decode(M, oracle):
         xs = W.tp_decode(tokens, hidden, n)
         S = tokens * hidden * 2
         send = [_dev(x, torch.bfloat16) for x in xs]
-        for algo, aname, ref, launches in ((M.ONESHOT, "oneshot", oracle.all_reduce_one_shot, 1),
-                                           (M.TWOSHOT, "twoshot", oracle.all_reduce_two_shot, 1),
-                                           (M.RING, "ring", oracle.all_reduce_ring, 2 * (n - 1))):
+        for algo, aname, ref in ((M.ONESHOT, "oneshot", oracle.all_reduce_one_shot),
+                                 (M.TWOSHOT, "twoshot", oracle.all_reduce_two_shot),
+                                 (M.RING, "ring", oracle.all_reduce_ring)):
+            form = M.coll_all_reduce_form(n, tokens * hidden, torch.bfloat16, algo)
+            launches = 2 * (n - 1) if form == M.RING_STEPS else 1
             bufs = {"send": send, "recv": [torch.empty_like(t) for t in send]}
             if algo in (M.RING, M.RING_LL):
                 need = M.coll_all_reduce_workspace_size(n, tokens * hidden, torch.bfloat16, algo)
@@ -128,7 +133,7 @@ def build_tp_decode(M, oracle):
 
             ops.append(Op(f"all_reduce/{aname}", bind, bufs, 2 * n * S, launches,
                           {"op": "all_reduce", "algo": aname, "ranks": n, "shape": [tokens, hidden],
-                           "bytes_per_rank": S},
+                           "bytes_per_rank": S, "form": FORM_NAMES[form]},
                           inputs=["send"], outputs=["recv"],
                           ref=(lambda xs=xs, ref=ref: ref(xs, 0, "bf16")), kernel=f"all_reduce/{aname}"))
     ids = W.sampled_token_ids(n)
@@ -263,7 +268,7 @@ def build_ll_sweep(M, oracle, sizes=None):
 
 def build_ring_compare(M, oracle):
     """The ring all-reduce four ways on the TP-decode shapes (8 virtual ranks,
-    bf16): one launch per ring step (RING), one cooperative launch with LL
+    bf16): one launch per ring step (RING_STEPS), one cooperative launch with LL
     packets between ranks (RING_LL), one launch of 8-CTA clusters with the
     hops over distributed shared memory (RING_CLUSTER), and the
     stream-ordered packet path of the LL sweep (per-rank LL pack, packetised
@@ -276,7 +281,7 @@ def build_ring_compare(M, oracle):
         count = tokens * hidden
         S = count * 2
         send = [_dev(x, torch.bfloat16) for x in xs]
-        for algo, aname, launches in ((M.RING, "ring", 2 * (n - 1)), (M.RING_LL, "ring_ll", 1),
+        for algo, aname, launches in ((M.RING_STEPS, "ring_steps", 2 * (n - 1)), (M.RING_LL, "ring_ll", 1),
                                       (M.RING_CLUSTER, "ring_cluster", 1)):
             need = max(64, M.coll_all_reduce_workspace_size(n, count, torch.bfloat16, algo))
             ops.append(Op(f"all_reduce/{aname}",
@@ -306,7 +311,7 @@ def build_ring_compare(M, oracle):
                                              "shape": [tokens, hidden], "bytes_per_rank": S},
                       inputs=["send"], outputs=["recv"], kernel="all_reduce/ll_pack_ar_unpack"))
     return ops, {"workload": "ring_compare_8vr", "virtual_ranks": n, "shapes": W.tp_decode_shapes(),
-                 "variants": ["ring (launch per step)", "ring_ll (one launch, LL packets)",
+                 "variants": ["ring_steps (launch per step)", "ring_ll (one launch, LL packets)",
                               "ring_cluster (one launch, cluster DSMEM hops)",
                               "LL pack + packetised two-shot + unpack (stream-ordered)"]}
 

@@ -78,9 +78,10 @@ typedef enum {
   COLL_ALGO_AUTO = 0,    /* currently TWOSHOT */
   COLL_ALGO_ONESHOT = 1, /* every rank reads all N inputs itself            */
   COLL_ALGO_TWOSHOT = 2, /* owner s reduces segment s, sends it to everyone */
-  COLL_ALGO_RING = 3,    /* 2(N-1) neighbour steps, one launch per step     */
+  COLL_ALGO_RING = 3,    /* 2(N-1) neighbour steps: RING_CLUSTER or RING_STEPS by size */
   COLL_ALGO_RING_LL = 4, /* the same ring in one launch, LL packets between ranks */
-  COLL_ALGO_RING_CLUSTER = 5 /* the same ring, ranks = CTAs of a cluster, hops over DSMEM */
+  COLL_ALGO_RING_CLUSTER = 5, /* the same ring, ranks = CTAs of a cluster, hops over DSMEM */
+  COLL_ALGO_RING_STEPS = 6    /* the same ring, one stream-ordered launch per step */
 } coll_algo_t;
 typedef enum { COLL_PROTO_SIMPLE = 0, COLL_PROTO_LL = 1, COLL_PROTO_LL128 = 2 } coll_proto_t;
 
@@ -148,14 +149,23 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    into N owner segments of ceil(count/N) elements rounded up to 16 bytes
  *    (the last ones may be short or empty); owner s reduces segment s across
  *    all ranks and writes it to every rank.  One fused kernel.
- *  RING ([TPC]; NCCL's ring kernel named in [RLL]): 2(N-1) stream-ordered
- *    steps on the ring r -> r+1 over the same N chunks: chunk c starts on rank
- *    c+1, every step moves it one rank on where that rank adds its own values
- *    (so chunk c is accumulated in the order c+1, ..., N-1, 0, ..., c), and
- *    the N-1 all-gather steps pass the finished chunks round.  Partials
- *    travel in fp32 (int32 for int32) through `workspace`
- *    (coll_all_reduce_workspace_size() bytes, 256-byte aligned); the result
- *    may differ from the rank-order reduction by rounding only.
+ *  RING ([TPC]; NCCL's ring kernel named in [RLL]): 2(N-1) steps on the
+ *    ring r -> r+1 over the same N chunks: chunk c starts on rank c+1, every
+ *    step moves it one rank on where that rank adds its own values (so chunk
+ *    c is accumulated in the order c+1, ..., N-1, 0, ..., c), and the N-1
+ *    all-gather steps pass the finished chunks round.  Partials travel in
+ *    fp32 (int32 for int32); the result may differ from the rank-order
+ *    reduction by rounding only.  Runs as RING_CLUSTER (one launch) when
+ *    2 <= N <= 8, every buffer is 16-byte aligned and a rank holds at most
+ *    1 MiB, and as RING_STEPS otherwise: the same result bit for bit.
+ *    coll_all_reduce_form() tells which.  `workspace`:
+ *    coll_all_reduce_workspace_size() bytes, 16-byte aligned: a 256-byte
+ *    header whose bytes 16..23 receive the status pair of the one-launch
+ *    form (int[2], cleared by the caller; COLL_DEV_TIMEOUT if a bounded wait
+ *    ran out), then the partials of the stream-ordered form.
+ *  RING_STEPS: the RING schedule as 2(N-1) stream-ordered launches, one per
+ *    step (the launch boundary is the step's synchronisation); partials in
+ *    the workspace after its header.  Nothing waits, so it cannot time out.
  *  RING_LL ([RLL] "Traditional LL Protocols", "Pro5000 ?": NCCL's Ring LL
  *    kernel): the RING schedule, chunk order and rounding (bit-identical
  *    result) in ONE cooperative launch.  Virtual rank r is a set of CTAs; it
@@ -167,26 +177,34 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    caller).  The workspace (coll_all_reduce_workspace_size() bytes,
  *    256-byte aligned) must be zero-filled once before its first use and
  *    serves one call at a time; the library keeps a call counter in it.
- *    Buffers that are not 16-byte aligned take the RING path.
+ *    Buffers that are not 16-byte aligned take the RING_STEPS path.
  *  RING_CLUSTER: the RING schedule, chunk order and rounding (bit-identical
  *    result) in one launch of thread-block clusters of N CTAs, CTA r playing
  *    virtual rank r: each hop is an asynchronous store into the next CTA's
  *    shared memory over the SM-to-SM network that completes that CTA's
  *    mbarrier, so the partials never touch HBM.  The clusters are about as
- *    many as fit on the GPU at once and walk the message tile by tile, two
- *    tiles in flight.  Needs 2 <= N <= 8 and 16-byte aligned buffers;
- *    otherwise, if a RING-sized `workspace` is given, the call takes the RING
- *    path, else it returns COLL_ERR_UNSUPPORTED.  `workspace` is optional:
+ *    many as fit on the GPU at once and walk the message tile by tile.
+ *    Needs 2 <= N <= 8 and 16-byte aligned buffers; otherwise, if a
+ *    RING-sized `workspace` is given, the call takes the RING_STEPS path,
+ *    else it returns COLL_ERR_UNSUPPORTED.  `workspace` is optional:
  *    when at least 24 bytes are given, bytes 16..23 receive the status pair
  *    (COLL_DEV_TIMEOUT if a bounded wait ran out).
  *  AUTO picks TWOSHOT.  ONESHOT and TWOSHOT ignore `workspace`.
  * In place (recv[r] == send[r]) is allowed for TWOSHOT, RING, RING_LL,
- * RING_CLUSTER and AUTO. */
+ * RING_CLUSTER, RING_STEPS and AUTO. */
 COLL_API int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size_t count,
                     coll_dtype_t dtype, coll_op_t op, coll_algo_t algo, void* workspace,
                     size_t workspace_bytes, coll_stream_t stream);
 COLL_API size_t coll_all_reduce_workspace_size(int nranks, size_t count, coll_dtype_t dtype,
                                       coll_algo_t algo);
+/* The form coll_all_reduce() runs for these arguments when nranks >= 2 and
+ * count >= 1: ONESHOT, TWOSHOT, RING_LL, RING_CLUSTER or RING_STEPS (AUTO
+ * and RING resolved; `aligned` != 0 when every buffer is 16-byte aligned).
+ * RING_CLUSTER launches one kernel, RING_STEPS 2(N-1), the others one.
+ * Returns a negative COLL_ERR_* for an invalid rank count, dtype or algo.
+ * Library introspection; the sources have no counterpart. */
+COLL_API int coll_all_reduce_form(int nranks, size_t count, coll_dtype_t dtype, coll_algo_t algo,
+                                  int aligned);
 
 /* AllGather ([TUT] 7.1, 7.3): every recv[q] (N * send_count elements) gets
  * recv[q][r * send_count + i] = send[r][i]: the slices are concatenated, not

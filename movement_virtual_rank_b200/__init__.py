@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libmvrcoll.so")
 
 BF16, FP16, FP32, INT32 = 0, 1, 2, 3
 SUM, MAX, MIN, PROD = 0, 1, 2, 3
-ALGO_AUTO, ONESHOT, TWOSHOT, RING, RING_LL, RING_CLUSTER = 0, 1, 2, 3, 4, 5
+ALGO_AUTO, ONESHOT, TWOSHOT, RING, RING_LL, RING_CLUSTER, RING_STEPS = 0, 1, 2, 3, 4, 5, 6
 SIMPLE, LL, LL128 = 0, 1, 2
 DEV_OK, DEV_FLAG_MISMATCH, DEV_TIMEOUT, DEV_SPLIT_OVERFLOW, DEV_BAD_ROUTE = 0, 1, 2, 3, 4
 MAX_RANKS = 64
@@ -31,7 +31,7 @@ _DTYPES = {torch.bfloat16: BF16, torch.float16: FP16, torch.float32: FP32, torch
 _ESIZE = {BF16: 2, FP16: 2, FP32: 4, INT32: 4}
 OPS = {"sum": SUM, "max": MAX, "min": MIN, "prod": PROD}
 ALGOS = {"auto": ALGO_AUTO, "oneshot": ONESHOT, "twoshot": TWOSHOT, "ring": RING, "ring_ll": RING_LL,
-         "ring_cluster": RING_CLUSTER}
+         "ring_cluster": RING_CLUSTER, "ring_steps": RING_STEPS}
 PROTOS = {"simple": SIMPLE, "ll": LL, "ll128": LL128}
 
 
@@ -58,6 +58,7 @@ _SIGS = {
     "coll_reduce_scatter": (_I, [_PP, _PP, _I, _SZ, _I, _I, _VP]),
     "coll_all_reduce": (_I, [_PP, _PP, _I, _SZ, _I, _I, _I, _VP, _SZ, _VP]),
     "coll_all_reduce_workspace_size": (_SZ, [_I, _SZ, _I, _I]),
+    "coll_all_reduce_form": (_I, [_I, _SZ, _I, _I, _I]),
     "coll_all_gather": (_I, [_PP, _PP, _I, _SZ, _I, _VP]),
     "coll_all_to_all": (_I, [_PP, _PP, _I, _SZ, _I, _VP]),
     "coll_all_to_all_v": (_I, [_PP, _PP, _I, _PI64, _PI64, _PI64, _PI64, _PI64, _SZ, _I, _VP]),
@@ -237,12 +238,23 @@ def coll_all_reduce_workspace_size(nranks: int, count: int, dtype: torch.dtype, 
     return int(lib().coll_all_reduce_workspace_size(nranks, count, _DTYPES[dtype], algo))
 
 
+def coll_all_reduce_form(nranks: int, count: int, dtype: torch.dtype, algo=TWOSHOT, aligned: bool = True) -> int:
+    """The form coll_all_reduce() runs: ONESHOT, TWOSHOT, RING_LL,
+    RING_CLUSTER (one launch) or RING_STEPS (2(N-1) launches)."""
+    algo = ALGOS[algo] if isinstance(algo, str) else int(algo)
+    rc = int(lib().coll_all_reduce_form(nranks, count, _DTYPES[dtype], algo, 1 if aligned else 0))
+    if rc < 0:
+        _check("coll_all_reduce_form", rc)
+    return rc
+
+
 def coll_all_reduce(send, recv, op="sum", algo=TWOSHOT, workspace: torch.Tensor | None = None, stream=None):
     """``workspace``: a CUDA tensor passed through to the library when given.
-    RING and RING_LL need one of at least coll_all_reduce_workspace_size()
-    bytes (zero-filled before its first RING_LL use) and get a zeroed one
-    allocated here when it is omitted; RING_CLUSTER uses one, when given, for
-    its status pair and its fallback to RING."""
+    RING, RING_STEPS and RING_LL need one of at least
+    coll_all_reduce_workspace_size() bytes (zero-filled before its first
+    RING_LL use) and get a zeroed one allocated here when it is omitted;
+    RING_CLUSTER uses one, when given, for its status pair and its fallback
+    to RING_STEPS."""
     algo = ALGOS[algo] if isinstance(algo, str) else int(algo)
     send = _ranks(send, "send", send[0].dtype)
     recv = _ranks(recv, "recv", send[0].dtype)
@@ -252,7 +264,7 @@ def coll_all_reduce(send, recv, op="sum", algo=TWOSHOT, workspace: torch.Tensor 
     if _same_numel(recv, "recv") != n:
         raise ValueError("send and recv sizes differ")
     ws_ptr, ws_bytes = None, 0
-    if workspace is None and algo in (RING, RING_LL):
+    if workspace is None and algo in (RING, RING_LL, RING_STEPS):
         need = coll_all_reduce_workspace_size(len(send), n, send[0].dtype, algo)
         workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=send[0].device)
     if workspace is not None:

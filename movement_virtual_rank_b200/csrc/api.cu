@@ -298,18 +298,43 @@ int coll_reduce_scatter(const void* const* send, void* const* recv, int nranks, 
 }
 
 // ------------------------------------------------------------- AllReduce ----
+// RING runs as one cluster launch up to this many bytes per rank (where it
+// measured faster on B200 than the stream-ordered steps), as steps above it
+constexpr size_t kRingClusterMaxBytes = size_t(1) << 20;
+
+static coll_algo_t ring_form(int nranks, size_t bytes, bool vec) {
+  return (vec && ring_cluster_supported(nranks) && bytes <= kRingClusterMaxBytes) ? COLL_ALGO_RING_CLUSTER
+                                                                                  : COLL_ALGO_RING_STEPS;
+}
+
 size_t coll_all_reduce_workspace_size(int nranks, size_t count, coll_dtype_t dtype, coll_algo_t algo) {
   if (!valid_n(nranks) || !elem_size(dtype)) return 0;
-  if (algo == COLL_ALGO_RING) return ring_ws(count);
+  // 256-byte header (status pair at bytes 16..23), then the fp32 / int32 partials
+  if (algo == COLL_ALGO_RING || algo == COLL_ALGO_RING_STEPS) return 256 + ring_ws(count);
   if (algo == COLL_ALGO_RING_LL) return std::max(ring_ll_workspace(nranks, count, elem_size(dtype)), 256 + ring_ws(count));
   return 0;
+}
+
+int coll_all_reduce_form(int nranks, size_t count, coll_dtype_t dtype, coll_algo_t algo, int aligned) {
+  const int es = elem_size(dtype);
+  if (!es || !valid_n(nranks)) return COLL_ERR_INVALID_ARG;
+  if (algo < COLL_ALGO_AUTO || algo > COLL_ALGO_RING_STEPS) return COLL_ERR_UNSUPPORTED;
+  const bool vec = aligned != 0;
+  switch (algo) {
+    case COLL_ALGO_AUTO: return COLL_ALGO_TWOSHOT;
+    case COLL_ALGO_RING: return ring_form(nranks, count * es, vec);
+    case COLL_ALGO_RING_LL: return vec ? COLL_ALGO_RING_LL : COLL_ALGO_RING_STEPS;
+    case COLL_ALGO_RING_CLUSTER:
+      return vec && ring_cluster_supported(nranks) ? COLL_ALGO_RING_CLUSTER : COLL_ALGO_RING_STEPS;
+    default: return algo;
+  }
 }
 
 int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size_t count, coll_dtype_t dtype,
                     coll_op_t op, coll_algo_t algo, void* workspace, size_t workspace_bytes, coll_stream_t stream) {
   const int es = elem_size(dtype);
   if (!es) return COLL_ERR_UNSUPPORTED;
-  if (!valid_op(op) || algo < COLL_ALGO_AUTO || algo > COLL_ALGO_RING_CLUSTER) return COLL_ERR_UNSUPPORTED;
+  if (!valid_op(op) || algo < COLL_ALGO_AUTO || algo > COLL_ALGO_RING_STEPS) return COLL_ERR_UNSUPPORTED;
   if (!valid_n(nranks) || !all_nonnull(send, nranks) || !all_nonnull(recv, nranks)) return COLL_ERR_INVALID_ARG;
   const size_t bytes = count * es;
   if (bytes == 0) return COLL_OK;
@@ -319,7 +344,8 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
     for (int r = 0; r < nranks; ++r)
       if (overlap(recv[q], bytes, send[r], bytes) && !(q == r && recv[q] == send[r] && algo != COLL_ALGO_ONESHOT))
         return COLL_ERR_ALIAS;
-  if ((algo == COLL_ALGO_RING || algo == COLL_ALGO_RING_LL) && nranks > 1) {
+  const bool ring_ws_needed = algo == COLL_ALGO_RING || algo == COLL_ALGO_RING_LL || algo == COLL_ALGO_RING_STEPS;
+  if (ring_ws_needed && nranks > 1) {
     const size_t need = coll_all_reduce_workspace_size(nranks, count, dtype, algo);
     if (workspace == nullptr || workspace_bytes < need || (U(workspace) & (algo == COLL_ALGO_RING_LL ? 255 : 15)))
       return COLL_ERR_WORKSPACE;
@@ -331,29 +357,28 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
   bool vec = true;
   for (int r = 0; r < nranks; ++r) vec = vec && al16(send[r]) && al16(recv[r]);
   const size_t seg = seg_elems(count, nranks, es);
+  if (algo == COLL_ALGO_RING) algo = ring_form(nranks, bytes, vec);  // workspace checked above
   if (algo == COLL_ALGO_RING_CLUSTER) {
+    const bool has_ws = workspace != nullptr && workspace_bytes >= 24;
     if (vec && ring_cluster_supported(nranks)) {
-      if (workspace != nullptr && workspace_bytes >= 24 && !al16(workspace)) return COLL_ERR_WORKSPACE;
-      for (int r = 0; r < nranks; ++r)
-        if (workspace != nullptr && workspace_bytes >= 24 &&
-            (overlap(workspace, 24, send[r], bytes) || overlap(workspace, 24, recv[r], bytes)))
-          return COLL_ERR_ALIAS;
+      if (has_ws && !al16(workspace)) return COLL_ERR_WORKSPACE;
+      for (int r = 0; r < nranks && has_ws; ++r)
+        if (overlap(workspace, 24, send[r], bytes) || overlap(workspace, 24, recv[r], bytes)) return COLL_ERR_ALIAS;
       const char* in[COLL_MAX_RANKS];
       char* out[COLL_MAX_RANKS];
       for (int r = 0; r < nranks; ++r) {
         in[r] = static_cast<const char*>(send[r]);
         out[r] = static_cast<char*>(recv[r]);
       }
-      int* status = (workspace != nullptr && workspace_bytes >= 24)
-                        ? reinterpret_cast<int*>(static_cast<char*>(workspace) + 16)
-                        : nullptr;
+      int* status = has_ws ? reinterpret_cast<int*>(static_cast<char*>(workspace) + 16) : nullptr;
       return launch_ring_cluster(in, out, nranks, count, dtype, op, status, S(stream));
     }
-    const size_t need = ring_ws(count);
+    // no cluster form: the stream-ordered steps, given a RING-sized workspace
+    const size_t need = 256 + ring_ws(count);
     if (workspace == nullptr || workspace_bytes < need || !al16(workspace)) return COLL_ERR_UNSUPPORTED;
     for (int r = 0; r < nranks; ++r)
       if (overlap(workspace, need, send[r], bytes) || overlap(workspace, need, recv[r], bytes)) return COLL_ERR_ALIAS;
-    algo = COLL_ALGO_RING;
+    algo = COLL_ALGO_RING_STEPS;
   }
   if (algo == COLL_ALGO_RING_LL) {
     if (vec) {
@@ -366,17 +391,15 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
       int* status = reinterpret_cast<int*>(static_cast<char*>(workspace) + 16);
       return launch_ring_ll(in, out, nranks, count, dtype, op, workspace, status, S(stream));
     }
-    // unaligned buffers: the stream-ordered ring, its partials after the header
-    workspace = static_cast<char*>(workspace) + 256;
-    algo = COLL_ALGO_RING;
+    algo = COLL_ALGO_RING_STEPS;  // unaligned buffers: the stream-ordered steps, partials after the header
   }
-  if (algo == COLL_ALGO_RING) {
+  if (algo == COLL_ALGO_RING_STEPS) {
     RingStepArgs a{};
     for (int r = 0; r < nranks; ++r) {
       a.in[r] = static_cast<const char*>(send[r]);
       a.out[r] = static_cast<char*>(recv[r]);
     }
-    a.partial = static_cast<char*>(workspace);
+    a.partial = static_cast<char*>(workspace) + 256;  // after the header
     a.count = count;
     a.seg = seg;
     a.n = nranks;

@@ -15,19 +15,19 @@
 // st.async ... mbarrier::complete_tx, so the store itself completes the
 // receiver's mbarrier for that slot (release at cluster scope, no separate
 // fence or arrive).  The receiver armed that mbarrier with the slot's byte
-// count and waits on it (acquire at cluster scope).  Every slot is written
-// once per tile; two slot sets alternate between consecutive tiles, and a
-// split cluster barrier (arrive after a tile, wait one tile later) keeps a
-// sender from refilling a set before every receiver has read it.
+// count and waits on it (acquire at cluster scope).  Hops are numbered
+// without a break from tile to tile and hop h uses slot h mod N: the ring's
+// own dependencies keep a sender within N-1 hops of its receiver, so N slots
+// per CTA are enough and need neither credits nor a barrier between tiles.
 //
 // All of a ring's dependencies stay inside one cluster, whose CTAs the
 // hardware schedules together, so clusters may run in any order and in
 // waves.  Every wait is bounded: a CTA whose wait runs out raises
-// COLL_DEV_TIMEOUT, sets an abort word in every CTA of its cluster, stops
-// sending and receiving, still takes every cluster barrier, and before it
-// exits polls (bounded) the slots it still expects, so that no store is in
-// flight into it.  Only st.async stores and mbarrier updates cross CTAs;
-// there is no bulk copy and no multicast.
+// COLL_DEV_TIMEOUT and sets an abort word in every CTA of its cluster; all
+// of them stop sending and receiving, meet at the final cluster barrier, and
+// before leaving poll (bounded) the slots they still expect, so that no
+// store is in flight into a CTA that has left.  Only st.async stores and
+// mbarrier updates cross CTAs; there is no bulk copy and no multicast.
 #include <algorithm>
 
 #include "bulk.cuh"
@@ -38,7 +38,6 @@ namespace mvr {
 
 constexpr int kRcThreads = 128;
 constexpr int kRcMaxRanks = 8;                    // portable cluster size
-constexpr int kRcSlots = 2 * kRcMaxRanks - 2;     // hops per tile
 constexpr long long kRcBudgetCycles = 1ll << 28;  // about 0.14 s per wait
 constexpr long long kRcDrainCycles = 1ll << 17;   // about 70 us per slot, abort path only
 
@@ -111,29 +110,26 @@ __global__ void __launch_bounds__(kRcThreads) k_ring_cluster(const __grid_consta
   constexpr int ES = Elem<DT>::kSize;
   constexpr uint64_t TE = static_cast<uint64_t>(kRcThreads) * VN;  // elements of a chunk per tile
   constexpr uint32_t kSlotBytes = kRcThreads * NQ * 16;
-  extern __shared__ __align__(16) uint4 slot_buf[];  // [set][slot][thread][NQ]
-  __shared__ __align__(8) uint64_t bar[2][kRcSlots];
+  extern __shared__ __align__(16) uint4 slot_buf[];  // [slot][thread][NQ]
+  __shared__ __align__(8) uint64_t bar[kRcMaxRanks];
   __shared__ uint32_t abort_word;
   const int n = a.n;
-  const int slots = 2 * n - 2;
+  const uint32_t H = 2 * n - 2;  // hops per tile
   const int r = static_cast<int>(cluster_rank());
   const uint64_t g = cluster_idx();
   const uint64_t G = cluster_count();
   const int tid = threadIdx.x;
-  // thread 0's record of the slots it armed and has not yet seen complete
-  // (bit 16*b + s), and the phase parity each set was last armed for (bit b);
-  // read only by the abort drain
+  // hop h of this cluster (tile after tile) lands in slot h % n, phase h / n
+  const uint32_t total_hops = static_cast<uint32_t>((a.tiles - g + G - 1) / G) * H;
+  // thread 0's record of the slots armed and not yet seen complete, and the
+  // parity each was last armed for (bit j); read only by the abort drain
   uint32_t pending = 0, pending_par = 0;
   if (tid == 0) {
     abort_word = 0;
-    for (int b = 0; b < 2; ++b)
-      for (int s = 0; s < slots; ++s) mbar_init(&bar[b][s], 1);
+    for (int j = 0; j < n; ++j) mbar_init(&bar[j], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    for (int b = 0; b < 2; ++b)  // arm the slots of this cluster's first two tiles
-      if (g + b * G < a.tiles) {
-        for (int s = 0; s < slots; ++s) mbar_arrive_expect_tx(&bar[b][s], kSlotBytes);
-        pending |= ((1u << slots) - 1) << (16 * b);
-      }
+    for (int j = 0; j < n; ++j) mbar_arrive_expect_tx(&bar[j], kSlotBytes);
+    pending = (1u << n) - 1;
   }
   cluster_sync_all();  // every CTA's barriers are armed before anyone stores into them
   pdl_wait();
@@ -141,7 +137,7 @@ __global__ void __launch_bounds__(kRcThreads) k_ring_cluster(const __grid_consta
 
   const int nxt = (r + 1) % n;
   const uint32_t next_slot0 = map_to(slot_buf, nxt);
-  const uint32_t next_bar0 = map_to(&bar[0][0], nxt);
+  const uint32_t next_bar0 = map_to(bar, nxt);
   bool alive = true;
 
   auto chunk_lo = [&](int c) { return static_cast<uint64_t>(c) * a.seg; };
@@ -179,26 +175,27 @@ __global__ void __launch_bounds__(kRcThreads) k_ring_cluster(const __grid_consta
     report(a.status, COLL_DEV_TIMEOUT, 1);
     for (int q = 0; q < n; ++q) st_cluster_u32(map_to(&abort_word, q), 1u);
   };
-  auto send = [&](int b, int s, const A (&v)[VN]) {
+  auto send = [&](uint32_t h, const A (&v)[VN]) {
     if (ld_volatile_smem(&abort_word) != 0) {
       alive = false;
       return;
     }
-    const int si = b * slots + s;
-    const uint32_t base = next_slot0 + static_cast<uint32_t>((si * kRcThreads + tid) * NQ * 16);
-    const uint32_t bar_addr = next_bar0 + static_cast<uint32_t>((b * kRcSlots + s) * 8);
+    const uint32_t j = h % n;
+    const uint32_t base = next_slot0 + (j * kRcThreads + tid) * NQ * 16;
 #pragma unroll
     for (int q = 0; q < NQ; ++q)
       st_async16(base + q * 16,
                  make_uint4(to_bits(v[4 * q]), to_bits(v[4 * q + 1]), to_bits(v[4 * q + 2]), to_bits(v[4 * q + 3])),
-                 bar_addr);
+                 next_bar0 + j * 8);
   };
-  // wait for slot s of set b (phase parity par) and read my part of it; thread 0
-  // then re-arms the slot for the tile two ahead when this cluster has one
-  auto recv = [&](int b, int s, uint32_t par, bool rearm, A (&v)[VN]) -> bool {
-    if (!try_wait_cluster(&bar[b][s], par)) {
+  // wait for hop h and read my part of its slot; thread 0 then re-arms the
+  // slot for hop h + n when this cluster has one
+  auto recv = [&](uint32_t h, A (&v)[VN]) -> bool {
+    const uint32_t j = h % n;
+    const uint32_t par = (h / n) & 1;
+    if (!try_wait_cluster(&bar[j], par)) {
       const long long t0 = clock64();
-      while (!try_wait_cluster(&bar[b][s], par)) {
+      while (!try_wait_cluster(&bar[j], par)) {
         if (ld_volatile_smem(&abort_word) != 0) return false;
         if (clock64() - t0 > kRcBudgetCycles) {
           raise_abort();
@@ -206,7 +203,7 @@ __global__ void __launch_bounds__(kRcThreads) k_ring_cluster(const __grid_consta
         }
       }
     }
-    const uint4* p = slot_buf + ((b * slots + s) * kRcThreads + tid) * NQ;
+    const uint4* p = slot_buf + (j * kRcThreads + tid) * NQ;
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
       const uint4 x = p[q];
@@ -216,11 +213,11 @@ __global__ void __launch_bounds__(kRcThreads) k_ring_cluster(const __grid_consta
       v[4 * q + 3] = from_bits(x.w);
     }
     if (tid == 0) {
-      pending &= ~(1u << (16 * b + s));
-      if (rearm) {
-        mbar_arrive_expect_tx(&bar[b][s], kSlotBytes);
-        pending |= 1u << (16 * b + s);
-        pending_par = (pending_par & ~(1u << b)) | ((par ^ 1u) << b);
+      pending &= ~(1u << j);
+      if (h + n < total_hops) {
+        mbar_arrive_expect_tx(&bar[j], kSlotBytes);
+        pending |= 1u << j;
+        pending_par ^= 1u << j;
       }
     }
     return true;
@@ -239,13 +236,13 @@ __global__ void __launch_bounds__(kRcThreads) k_ring_cluster(const __grid_consta
     }
   };
 
+  // A slot is refilled only after its previous hop was read: the sender's
+  // hop h depends, thread by thread, on this rank's hop h - n + 1, which this
+  // rank sends only after reading hop h - n.  So n slots need no credits.
   uint4 pre[kRcMaxRanks];
-  if (g < a.tiles) fetch(g, pre);
-  uint32_t it = 0;
-  for (uint64_t t = g; t < a.tiles; t += G, ++it) {
-    const int b = static_cast<int>(it & 1);
-    const uint32_t par = (it >> 1) & 1;
-    const bool rearm = t + 2 * G < a.tiles;
+  fetch(g, pre);
+  uint32_t h0 = 0;  // this tile's first hop
+  for (uint64_t t = g; t < a.tiles && alive; t += G, h0 += H) {
     const uint64_t e = t * TE + static_cast<uint64_t>(tid) * VN;
     uint4 nx[kRcMaxRanks];
     if (t + G < a.tiles) fetch(t + G, nx);  // next tile's inputs, in flight during this one
@@ -265,59 +262,52 @@ __global__ void __launch_bounds__(kRcThreads) k_ring_cluster(const __grid_consta
       }
     };
 
-    if (alive) {
-      A p[VN];
-      mine(0, p);
-      send(b, 0, p);
+    A p[VN];
+    mine(0, p);
+    send(h0, p);
 #pragma unroll
-      for (int k = 1; k < kRcMaxRanks; ++k) {
-        if (k >= n || !alive) break;
-        A x[VN];
-        mine(k, x);
-        if (!recv(b, k - 1, par, rearm, p)) {
-          alive = false;
-          break;
-        }
-#pragma unroll
-        for (int i = 0; i < VN; ++i) p[i] = op_step<OP>(p[i], x[i]);
-        if (k == n - 1) {  // complete on this rank: one rounding, the rounded value travels on
-          Vec<DT> w;
-#pragma unroll
-          for (int i = 0; i < VN; ++i) w.v[i] = p[i];
-          Vec<DT> back;
-          widen16<DT>(narrow16<DT>(w), back);
-#pragma unroll
-          for (int i = 0; i < VN; ++i) p[i] = back.v[i];
-          put(r, e, p);
-        }
-        send(b, k, p);
+    for (int k = 1; k < kRcMaxRanks; ++k) {
+      if (k >= n || !alive) break;
+      A x[VN];
+      mine(k, x);
+      if (!recv(h0 + k - 1, p)) {
+        alive = false;
+        break;
       }
-      for (int j = 1; j < n && alive; ++j) {  // all-gather hops
-        if (!recv(b, n - 2 + j, par, rearm, p)) {
-          alive = false;
-          break;
-        }
-        put(((r - j) % n + n) % n, e, p);
-        if (j < n - 1) send(b, n - 1 + j, p);
+#pragma unroll
+      for (int i = 0; i < VN; ++i) p[i] = op_step<OP>(p[i], x[i]);
+      if (k == n - 1) {  // complete on this rank: one rounding, the rounded value travels on
+        Vec<DT> w;
+#pragma unroll
+        for (int i = 0; i < VN; ++i) w.v[i] = p[i];
+        Vec<DT> back;
+        widen16<DT>(narrow16<DT>(w), back);
+#pragma unroll
+        for (int i = 0; i < VN; ++i) p[i] = back.v[i];
+        put(r, e, p);
       }
+      send(h0 + k, p);
     }
-    // this CTA has read set b of this tile; before the next tile refills the
-    // other set, every CTA must have read that one (their arrive one tile ago)
-    if (it > 0) cluster_wait();
-    cluster_arrive();
+    for (int j = 1; j < n && alive; ++j) {  // all-gather hops
+      if (!recv(h0 + n - 2 + j, p)) {
+        alive = false;
+        break;
+      }
+      put(((r - j) % n + n) % n, e, p);
+      if (j < n - 1) send(h0 + n - 1 + j, p);
+    }
 #pragma unroll
     for (int k = 0; k < kRcMaxRanks; ++k) pre[k] = nx[k];
   }
-  if (it > 0) cluster_wait();
+  cluster_sync_all();  // no CTA leaves while a neighbour may still store into it
   if (tid == 0 && ld_volatile_smem(&abort_word) != 0) {
     // abort path: let any store still in flight into this CTA land first
-    for (int b = 0; b < 2; ++b)
-      for (int s = 0; s < slots; ++s)
-        if (pending & (1u << (16 * b + s))) {
-          const long long t0 = clock64();
-          while (!try_wait_cluster(&bar[b][s], (pending_par >> b) & 1u) && clock64() - t0 < kRcDrainCycles) {
-          }
+    for (int j = 0; j < n; ++j)
+      if (pending & (1u << j)) {
+        const long long t0 = clock64();
+        while (!try_wait_cluster(&bar[j], (pending_par >> j) & 1u) && clock64() - t0 < kRcDrainCycles) {
         }
+      }
   }
 }
 
@@ -352,13 +342,13 @@ static int launch_ring_cluster_t(RingClusterArgs a, cudaStream_t s) {
   constexpr int VN = Vec<DT>::kN;
   const uint64_t per_tile = static_cast<uint64_t>(kRcThreads) * VN;
   a.tiles = std::max<uint64_t>(1, (a.seg + per_tile - 1) / per_tile);
-  const size_t smem = static_cast<size_t>(2) * (2 * a.n - 2) * kRcThreads * VN * 4;
+  const size_t smem = static_cast<size_t>(a.n) * kRcThreads * VN * 4;
   static int smem_set[COLL_MAX_RANKS] = {0};  // per device ordinal: largest limit set so far
   const int st = allow_dynamic_smem(reinterpret_cast<const void*>(k_ring_cluster<DT, OP>), smem, smem_set);
   if (st != COLL_OK) return st;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
-  static bool carveout_set[COLL_MAX_RANKS] = {};  // two CTAs of up to 112 KB share an SM
+  static bool carveout_set[COLL_MAX_RANKS] = {};  // as many CTAs per SM as shared memory allows
   if (dev >= 0 && dev < COLL_MAX_RANKS && !carveout_set[dev]) {
     if (cudaFuncSetAttribute(k_ring_cluster<DT, OP>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess)

@@ -66,6 +66,30 @@ def test_workspace_sizes():
     assert L.coll_moe_route_workspace_size(8, 4096, 8, 2048) == 0  # too many experts
 
 
+def test_all_reduce_form():
+    """Which form coll_all_reduce runs (host logic only, no device call)."""
+    L = M.lib()
+    mib = 1 << 20
+    assert L.coll_all_reduce_form(8, mib // 2, M.BF16, M.RING, 1) == M.RING_CLUSTER
+    assert L.coll_all_reduce_form(8, mib // 2 + 1, M.BF16, M.RING, 1) == M.RING_STEPS
+    assert L.coll_all_reduce_form(8, mib // 4, M.FP32, M.RING, 1) == M.RING_CLUSTER
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING, 0) == M.RING_STEPS  # unaligned
+    assert L.coll_all_reduce_form(9, 1000, M.BF16, M.RING, 1) == M.RING_STEPS  # beyond a portable cluster
+    assert L.coll_all_reduce_form(2, 1000, M.BF16, M.RING, 1) == M.RING_CLUSTER
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING_CLUSTER, 0) == M.RING_STEPS
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING_LL, 1) == M.RING_LL
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING_LL, 0) == M.RING_STEPS
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, M.ALGO_AUTO, 1) == M.TWOSHOT
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, M.ONESHOT, 1) == M.ONESHOT
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING_STEPS, 1) == M.RING_STEPS
+    assert L.coll_all_reduce_form(0, 1000, M.BF16, M.RING, 1) == -1
+    assert L.coll_all_reduce_form(8, 1000, 9, M.RING, 1) == -1
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, 7, 1) == -2
+    # RING and RING_STEPS: a 256-byte header, then 4 bytes of partial per element
+    for algo in (M.RING, M.RING_STEPS):
+        assert L.coll_all_reduce_workspace_size(8, 1000, M.BF16, algo) == 256 + 4096
+
+
 def _arr(vals):
     a = (ctypes.c_void_p * len(vals))(*vals)
     return ctypes.cast(a, ctypes.POINTER(ctypes.c_void_p)), a

@@ -17,7 +17,8 @@ from gpu_util import ESIZE, Guarded, need_gpu
 pytestmark = pytest.mark.gpu
 
 ALGOS = {M.ONESHOT: oracle.all_reduce_one_shot, M.TWOSHOT: oracle.all_reduce_two_shot,
-         M.RING: oracle.all_reduce_ring, M.RING_LL: oracle.all_reduce_ring}
+         M.RING: oracle.all_reduce_ring, M.RING_LL: oracle.all_reduce_ring, M.RING_STEPS: oracle.all_reduce_ring,
+         M.RING_CLUSTER: oracle.all_reduce_ring}
 
 
 def bits(a):
@@ -47,7 +48,11 @@ def test_fuzz_all_reduce(seed):
     send = [Guarded(count, dtype, offset=off * (r % 2), fill=xs[r]) for r in range(n)]
     in_place = algo != M.ONESHOT and bool(g.integers(0, 2))
     recv = send if in_place else [Guarded(count, dtype, offset=off * ((r + 1) % 2)) for r in range(n)]
-    M.coll_all_reduce([b.t for b in send], [b.t for b in recv], op=op, algo=algo)
+    ws = None
+    if algo == M.RING_CLUSTER:  # a RING-sized workspace: the fallback for unaligned buffers or N > 8
+        need = M.coll_all_reduce_workspace_size(n, count, send[0].t.dtype, M.RING)
+        ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    M.coll_all_reduce([b.t for b in send], [b.t for b in recv], op=op, algo=algo, workspace=ws)
     torch.cuda.synchronize()
     want = ALGOS[algo](xs, op, dtype)
     for q in range(n):

@@ -21,6 +21,7 @@ ALGO_FN = {
     M.TWOSHOT: oracle.all_reduce_two_shot,
     M.ONESHOT: oracle.all_reduce_one_shot,
     M.RING: oracle.all_reduce_ring,
+    M.RING_STEPS: oracle.all_reduce_ring,
 }
 OPNAME = {0: "sum", 1: "max", 2: "min", 3: "prod"}
 
@@ -57,7 +58,7 @@ def assert_ranks_equal(got, want, what=""):
                                  f"got {g[bad[:5]]} want {w[bad[:5]]}")
 
 
-@pytest.mark.parametrize("algo", [M.TWOSHOT, M.ONESHOT, M.RING])
+@pytest.mark.parametrize("algo", [M.TWOSHOT, M.ONESHOT, M.RING, M.RING_STEPS])
 @pytest.mark.parametrize("n", [1, 2, 3, 4, 5, 8])
 @pytest.mark.parametrize("count", [1, 7, 8 * 37 + 3, 65536 + 24, 300007])
 def test_all_reduce_bf16_sum(algo, n, count):
@@ -69,7 +70,7 @@ def test_all_reduce_bf16_sum(algo, n, count):
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp16", "fp32", "int32"])
 @pytest.mark.parametrize("op", [0, 1, 2, 3])
-@pytest.mark.parametrize("algo", [M.TWOSHOT, M.ONESHOT, M.RING])
+@pytest.mark.parametrize("algo", [M.TWOSHOT, M.ONESHOT, M.RING, M.RING_STEPS])
 @pytest.mark.parametrize("n", [3, 8, 13])
 def test_all_reduce_dtypes_ops(dtype, op, algo, n):
     need_gpu()
@@ -79,7 +80,7 @@ def test_all_reduce_dtypes_ops(dtype, op, algo, n):
     assert_ranks_equal(got, ALGO_FN[algo](xs, op, dtype), f"{dtype} {OPNAME[op]} algo {algo}")
 
 
-@pytest.mark.parametrize("algo", [M.TWOSHOT, M.RING])
+@pytest.mark.parametrize("algo", [M.TWOSHOT, M.RING, M.RING_STEPS])
 def test_all_reduce_in_place(algo):
     need_gpu()
     xs = inputs(8, 50001, "bf16", salt=3)
@@ -87,7 +88,7 @@ def test_all_reduce_in_place(algo):
     assert_ranks_equal(got, ALGO_FN[algo](xs, 0, "bf16"))
 
 
-@pytest.mark.parametrize("algo", [M.TWOSHOT, M.ONESHOT, M.RING])
+@pytest.mark.parametrize("algo", [M.TWOSHOT, M.ONESHOT, M.RING, M.RING_STEPS])
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
 def test_all_reduce_unaligned_and_guards(algo, dtype):
     need_gpu()
@@ -123,7 +124,7 @@ def test_special_values(dtype, op):
     k = v.size
     idx = np.array(np.meshgrid(np.arange(k), np.arange(k), np.arange(k), indexing="ij")).reshape(3, -1)
     xs = [v[idx[r]] for r in range(3)]
-    for algo in (M.TWOSHOT, M.ONESHOT, M.RING):
+    for algo in (M.TWOSHOT, M.ONESHOT, M.RING, M.RING_STEPS):
         got = run_all_reduce(xs, dtype, op, algo)
         assert_ranks_equal(got, ALGO_FN[algo](xs, op, dtype), f"{dtype} {OPNAME[op]} algo {algo}")
 
@@ -144,7 +145,7 @@ def test_tp_decode_workload(tokens, hidden):
     need_gpu()
     xs = W.tp_decode(tokens, hidden)
     ref = oracle.all_reduce(xs, 0, "bf16")
-    for algo in (M.ONESHOT, M.TWOSHOT, M.RING):
+    for algo in (M.ONESHOT, M.TWOSHOT, M.RING, M.RING_STEPS):
         got = run_all_reduce(xs, "bf16", M.SUM, algo)
         assert_ranks_equal(got, ALGO_FN[algo](xs, 0, "bf16"), f"algo {algo}")
         if algo == M.RING:
