@@ -157,7 +157,7 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    fp32 (int32 for int32); the result may differ from the rank-order
  *    reduction by rounding only.  Runs as RING_CLUSTER (one launch) when
  *    2 <= N <= 8, every buffer is 16-byte aligned and a rank holds at most
- *    1 MiB, and as RING_STEPS otherwise: the same result bit for bit.
+ *    2.5 MiB, and as RING_STEPS otherwise: the same result bit for bit.
  *    coll_all_reduce_form() tells which.  `workspace`:
  *    coll_all_reduce_workspace_size() bytes, 16-byte aligned: a 256-byte
  *    header whose bytes 16..23 receive the status pair of the one-launch

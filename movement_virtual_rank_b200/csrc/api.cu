@@ -300,7 +300,7 @@ int coll_reduce_scatter(const void* const* send, void* const* recv, int nranks, 
 // ------------------------------------------------------------- AllReduce ----
 // RING runs as one cluster launch up to this many bytes per rank (where it
 // measured faster on B200 than the stream-ordered steps), as steps above it
-constexpr size_t kRingClusterMaxBytes = size_t(1) << 20;
+constexpr size_t kRingClusterMaxBytes = size_t(5) << 19;  // 2.5 MiB
 
 static coll_algo_t ring_form(int nranks, size_t bytes, bool vec) {
   return (vec && ring_cluster_supported(nranks) && bytes <= kRingClusterMaxBytes) ? COLL_ALGO_RING_CLUSTER

@@ -106,21 +106,26 @@ __global__ void __launch_bounds__(kRcThreads) k_ring_cluster(const __grid_consta
   using A = typename Elem<DT>::A;
   using S = typename Elem<DT>::S;
   constexpr int VN = Vec<DT>::kN;  // elements per thread (16 bytes of input)
-  constexpr int NQ = VN / 4;       // 16-byte pieces of fp32 / int32 payload per thread
+  constexpr int NQ = VN / 4;       // 16-byte pieces of fp32 / int32 partials per thread
   constexpr int ES = Elem<DT>::kSize;
   constexpr uint64_t TE = static_cast<uint64_t>(kRcThreads) * VN;  // elements of a chunk per tile
-  constexpr uint32_t kSlotBytes = kRcThreads * NQ * 16;
-  extern __shared__ __align__(16) uint4 slot_buf[];  // [slot][thread][NQ]
+  // reduce-scatter hops carry fp32 / int32 partials, all-gather hops the
+  // rounded values in the storage type (16 bytes per thread)
+  constexpr uint32_t kWideBytes = kRcThreads * NQ * 16;
+  constexpr uint32_t kNarrowBytes = kRcThreads * 16;
+  constexpr uint32_t kSlotU4 = kRcThreads * NQ;  // slot size in 16-byte units
+  extern __shared__ __align__(16) uint4 slot_buf[];  // [slot][kSlotU4]
   __shared__ __align__(8) uint64_t bar[kRcMaxRanks];
   __shared__ uint32_t abort_word;
   const int n = a.n;
-  const uint32_t H = 2 * n - 2;  // hops per tile
+  const uint32_t H = 2 * n - 2;  // hops per tile: n-1 reduce-scatter, then n-1 all-gather
   const int r = static_cast<int>(cluster_rank());
   const uint64_t g = cluster_idx();
   const uint64_t G = cluster_count();
   const int tid = threadIdx.x;
   // hop h of this cluster (tile after tile) lands in slot h % n, phase h / n
   const uint32_t total_hops = static_cast<uint32_t>((a.tiles - g + G - 1) / G) * H;
+  auto hop_bytes = [&](uint32_t k) { return k < static_cast<uint32_t>(n - 1) ? kWideBytes : kNarrowBytes; };
   // thread 0's record of the slots armed and not yet seen complete, and the
   // parity each was last armed for (bit j); read only by the abort drain
   uint32_t pending = 0, pending_par = 0;
@@ -128,7 +133,7 @@ __global__ void __launch_bounds__(kRcThreads) k_ring_cluster(const __grid_consta
     abort_word = 0;
     for (int j = 0; j < n; ++j) mbar_init(&bar[j], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    for (int j = 0; j < n; ++j) mbar_arrive_expect_tx(&bar[j], kSlotBytes);
+    for (int j = 0; j < n; ++j) mbar_arrive_expect_tx(&bar[j], hop_bytes(j));
     pending = (1u << n) - 1;
   }
   cluster_sync_all();  // every CTA's barriers are armed before anyone stores into them
@@ -142,27 +147,6 @@ __global__ void __launch_bounds__(kRcThreads) k_ring_cluster(const __grid_consta
 
   auto chunk_lo = [&](int c) { return static_cast<uint64_t>(c) * a.seg; };
   auto chunk_end = [&](int c) { return min(chunk_lo(c) + a.seg, a.count); };
-  auto own = [&](int c, uint64_t e, A (&v)[VN]) {
-    const uint64_t gi = chunk_lo(c) + e;
-    const uint64_t end = chunk_end(c);
-#pragma unroll
-    for (int i = 0; i < VN; ++i)
-      v[i] = gi + i < end ? widen1<DT>(*reinterpret_cast<const S*>(a.in[r] + (gi + i) * ES)) : A(0);
-  };
-  auto put = [&](int c, uint64_t e, const A (&v)[VN]) {
-    const uint64_t gi = chunk_lo(c) + e;
-    const uint64_t end = chunk_end(c);
-    if (gi + VN <= end) {
-      Vec<DT> w;
-#pragma unroll
-      for (int i = 0; i < VN; ++i) w.v[i] = v[i];
-      st16(a.out[r] + gi * ES, narrow16<DT>(w));
-    } else {
-#pragma unroll
-      for (int i = 0; i < VN; ++i)
-        if (gi + i < end) *reinterpret_cast<S*>(a.out[r] + (gi + i) * ES) = narrow1<DT>(v[i]);
-    }
-  };
   auto to_bits = [](A x) -> uint32_t {
     if constexpr (std::is_same<A, float>::value) return __float_as_uint(x);
     else return static_cast<uint32_t>(x);
@@ -171,39 +155,74 @@ __global__ void __launch_bounds__(kRcThreads) k_ring_cluster(const __grid_consta
     if constexpr (std::is_same<A, float>::value) return __uint_as_float(u);
     else return static_cast<A>(static_cast<int32_t>(u));
   };
-  auto raise_abort = [&]() {
-    report(a.status, COLL_DEV_TIMEOUT, 1);
-    for (int q = 0; q < n; ++q) st_cluster_u32(map_to(&abort_word, q), 1u);
-  };
-  auto send = [&](uint32_t h, const A (&v)[VN]) {
-    if (ld_volatile_smem(&abort_word) != 0) {
-      alive = false;
-      return;
+  // store a rounded 16-byte vector (storage type) of chunk c to my output
+  auto put = [&](int c, uint64_t e, const uint4& w) {
+    const uint64_t gi = chunk_lo(c) + e;
+    const uint64_t end = chunk_end(c);
+    if (gi + VN <= end) {
+      st16(a.out[r] + gi * ES, w);
+    } else {
+      const S* sv = reinterpret_cast<const S*>(&w);
+#pragma unroll
+      for (int i = 0; i < VN; ++i)
+        if (gi + i < end) *reinterpret_cast<S*>(a.out[r] + (gi + i) * ES) = sv[i];
     }
-    const uint32_t j = h % n;
-    const uint32_t base = next_slot0 + (j * kRcThreads + tid) * NQ * 16;
+  };
+
+  // Hops are sent and received in the same order 0, 1, 2, ...: the send side
+  // keeps its slot, the receive side its slot, phase parity and in-tile index.
+  uint32_t js = 0;                          // slot of the next hop to send
+  uint32_t hr = 0, jr = 0, pr = 0, kr = 0;  // next hop to receive: index, slot, parity, index in tile
+  auto send_wide = [&](const A (&v)[VN]) {
+    const uint32_t base = next_slot0 + (js * kSlotU4 + tid * NQ) * 16;
+    const uint32_t bar_addr = next_bar0 + js * 8;
 #pragma unroll
     for (int q = 0; q < NQ; ++q)
       st_async16(base + q * 16,
                  make_uint4(to_bits(v[4 * q]), to_bits(v[4 * q + 1]), to_bits(v[4 * q + 2]), to_bits(v[4 * q + 3])),
-                 next_bar0 + j * 8);
+                 bar_addr);
+    js = js + 1 == static_cast<uint32_t>(n) ? 0 : js + 1;
   };
-  // wait for hop h and read my part of its slot; thread 0 then re-arms the
-  // slot for hop h + n when this cluster has one
-  auto recv = [&](uint32_t h, A (&v)[VN]) -> bool {
-    const uint32_t j = h % n;
-    const uint32_t par = (h / n) & 1;
-    if (!try_wait_cluster(&bar[j], par)) {
+  auto send_narrow = [&](const uint4& w) {
+    st_async16(next_slot0 + (js * kSlotU4 + tid) * 16, w, next_bar0 + js * 8);
+    js = js + 1 == static_cast<uint32_t>(n) ? 0 : js + 1;
+  };
+  // wait for the next hop; thread 0 then re-arms its slot for hop + n
+  auto wait_next = [&]() -> bool {
+    if (!try_wait_cluster(&bar[jr], pr)) {
       const long long t0 = clock64();
-      while (!try_wait_cluster(&bar[j], par)) {
+      while (!try_wait_cluster(&bar[jr], pr)) {
         if (ld_volatile_smem(&abort_word) != 0) return false;
         if (clock64() - t0 > kRcBudgetCycles) {
-          raise_abort();
+          report(a.status, COLL_DEV_TIMEOUT, 1);
+          for (int q = 0; q < n; ++q) st_cluster_u32(map_to(&abort_word, q), 1u);
           return false;
         }
       }
     }
-    const uint4* p = slot_buf + (j * kRcThreads + tid) * NQ;
+    return true;
+  };
+  auto advance = [&]() {
+    if (tid == 0) {
+      pending &= ~(1u << jr);
+      if (hr + n < total_hops) {
+        uint32_t k2 = kr + n;
+        if (k2 >= H) k2 -= H;
+        mbar_arrive_expect_tx(&bar[jr], hop_bytes(k2));
+        pending |= 1u << jr;
+        pending_par ^= 1u << jr;
+      }
+    }
+    ++hr;
+    kr = kr + 1 == H ? 0 : kr + 1;
+    if (++jr == static_cast<uint32_t>(n)) {
+      jr = 0;
+      pr ^= 1;
+    }
+  };
+  auto recv_wide = [&](A (&v)[VN]) -> bool {
+    if (!wait_next()) return false;
+    const uint4* p = slot_buf + jr * kSlotU4 + tid * NQ;
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
       const uint4 x = p[q];
@@ -212,14 +231,13 @@ __global__ void __launch_bounds__(kRcThreads) k_ring_cluster(const __grid_consta
       v[4 * q + 2] = from_bits(x.z);
       v[4 * q + 3] = from_bits(x.w);
     }
-    if (tid == 0) {
-      pending &= ~(1u << j);
-      if (h + n < total_hops) {
-        mbar_arrive_expect_tx(&bar[j], kSlotBytes);
-        pending |= 1u << j;
-        pending_par ^= 1u << j;
-      }
-    }
+    advance();
+    return true;
+  };
+  auto recv_narrow = [&](uint4& w) -> bool {
+    if (!wait_next()) return false;
+    w = slot_buf[jr * kSlotU4 + tid];
+    advance();
     return true;
   };
   // the 16-byte input vectors this rank adds at each reduce-scatter step of tile t
@@ -241,8 +259,8 @@ __global__ void __launch_bounds__(kRcThreads) k_ring_cluster(const __grid_consta
   // rank sends only after reading hop h - n.  So n slots need no credits.
   uint4 pre[kRcMaxRanks];
   fetch(g, pre);
-  uint32_t h0 = 0;  // this tile's first hop
-  for (uint64_t t = g; t < a.tiles && alive; t += G, h0 += H) {
+  const int c0 = r == 0 ? n - 1 : r - 1;  // chunk of reduce-scatter step 0
+  for (uint64_t t = g; t < a.tiles && alive; t += G) {
     const uint64_t e = t * TE + static_cast<uint64_t>(tid) * VN;
     uint4 nx[kRcMaxRanks];
     if (t + G < a.tiles) fetch(t + G, nx);  // next tile's inputs, in flight during this one
@@ -250,51 +268,59 @@ __global__ void __launch_bounds__(kRcThreads) k_ring_cluster(const __grid_consta
 #pragma unroll
       for (int k = 0; k < kRcMaxRanks; ++k) nx[k] = make_uint4(0, 0, 0, 0);
 
-    auto mine = [&](int k, A (&v)[VN]) {
-      const int c = ((r - 1 - k) % n + n) % n;
-      if (chunk_lo(c) + e + VN <= chunk_end(c)) {
+    // my values for reduce-scatter step k, chunk c (vector, or ragged tail)
+    auto mine = [&](int k, int c, A (&v)[VN]) {
+      const uint64_t gi = chunk_lo(c) + e;
+      const uint64_t end = chunk_end(c);
+      if (gi + VN <= end) {
         Vec<DT> w;
         widen16<DT>(pre[k], w);
 #pragma unroll
         for (int i = 0; i < VN; ++i) v[i] = w.v[i];
       } else {
-        own(c, e, v);
+#pragma unroll
+        for (int i = 0; i < VN; ++i)
+          v[i] = gi + i < end ? widen1<DT>(*reinterpret_cast<const S*>(a.in[r] + (gi + i) * ES)) : A(0);
       }
     };
 
     A p[VN];
-    mine(0, p);
-    send(h0, p);
+    int c = c0;
+    mine(0, c, p);
+    send_wide(p);
 #pragma unroll
     for (int k = 1; k < kRcMaxRanks; ++k) {
-      if (k >= n || !alive) break;
+      if (k >= n) break;
+      c = c == 0 ? n - 1 : c - 1;
       A x[VN];
-      mine(k, x);
-      if (!recv(h0 + k - 1, p)) {
+      mine(k, c, x);
+      if (!recv_wide(p)) {
         alive = false;
         break;
       }
 #pragma unroll
       for (int i = 0; i < VN; ++i) p[i] = op_step<OP>(p[i], x[i]);
-      if (k == n - 1) {  // complete on this rank: one rounding, the rounded value travels on
+      if (k < n - 1) {
+        send_wide(p);
+      } else {  // complete on this rank (c == r): one rounding; the rounded value travels on
         Vec<DT> w;
 #pragma unroll
         for (int i = 0; i < VN; ++i) w.v[i] = p[i];
-        Vec<DT> back;
-        widen16<DT>(narrow16<DT>(w), back);
-#pragma unroll
-        for (int i = 0; i < VN; ++i) p[i] = back.v[i];
-        put(r, e, p);
+        const uint4 fin = narrow16<DT>(w);
+        put(r, e, fin);
+        send_narrow(fin);
       }
-      send(h0 + k, p);
     }
-    for (int j = 1; j < n && alive; ++j) {  // all-gather hops
-      if (!recv(h0 + n - 2 + j, p)) {
+    int cj = r;
+    for (int j = 1; j < n && alive; ++j) {  // all-gather hops: chunk r - j arrives, is stored and passed on
+      uint4 w;
+      if (!recv_narrow(w)) {
         alive = false;
         break;
       }
-      put(((r - j) % n + n) % n, e, p);
-      if (j < n - 1) send(h0 + n - 1 + j, p);
+      cj = cj == 0 ? n - 1 : cj - 1;
+      put(cj, e, w);
+      if (j < n - 1) send_narrow(w);
     }
 #pragma unroll
     for (int k = 0; k < kRcMaxRanks; ++k) pre[k] = nx[k];
