@@ -267,12 +267,13 @@ def build_ll_sweep(M, oracle, sizes=None):
 
 
 def build_ring_compare(M, oracle):
-    """The ring all-reduce four ways on the TP-decode shapes (8 virtual ranks,
-    bf16): one launch per ring step (RING_STEPS), one cooperative launch with LL
-    packets between ranks (RING_LL), one launch of 8-CTA clusters with the
-    hops over distributed shared memory (RING_CLUSTER), and the
-    stream-ordered packet path of the LL sweep (per-rank LL pack, packetised
-    two-shot, per-rank unpack)."""
+    """Ring and packet all-reduce latency on the TP-decode shapes (8 virtual
+    ranks, bf16): the ring as one launch per step (RING_STEPS), as one
+    cooperative launch with LL packets between ranks (RING_LL) and as one
+    launch of 8-CTA clusters with the hops over distributed shared memory
+    (RING_CLUSTER); the two-shot with LL packets fused into one cooperative
+    launch (TWOSHOT_LL); and the stream-ordered packet path of the LL sweep
+    (per-rank LL pack, packetised two-shot, per-rank unpack)."""
     import torch
     n = 8
     ops = []
@@ -282,7 +283,7 @@ def build_ring_compare(M, oracle):
         S = count * 2
         send = [_dev(x, torch.bfloat16) for x in xs]
         for algo, aname, launches in ((M.RING_STEPS, "ring_steps", 2 * (n - 1)), (M.RING_LL, "ring_ll", 1),
-                                      (M.RING_CLUSTER, "ring_cluster", 1)):
+                                      (M.RING_CLUSTER, "ring_cluster", 1), (M.TWOSHOT_LL, "twoshot_ll", 1)):
             need = max(64, M.coll_all_reduce_workspace_size(n, count, torch.bfloat16, algo))
             ops.append(Op(f"all_reduce/{aname}",
                           lambda b, algo=algo: (lambda: M.coll_all_reduce(b["send"], b["recv"], algo=algo,
@@ -313,6 +314,7 @@ def build_ring_compare(M, oracle):
     return ops, {"workload": "ring_compare_8vr", "virtual_ranks": n, "shapes": W.tp_decode_shapes(),
                  "variants": ["ring_steps (launch per step)", "ring_ll (one launch, LL packets)",
                               "ring_cluster (one launch, cluster DSMEM hops)",
+                              "twoshot_ll (one launch, LL packets, fused)",
                               "LL pack + packetised two-shot + unpack (stream-ordered)"]}
 
 
@@ -614,6 +616,8 @@ def main():
     ap.add_argument("--lead-us", type=float, default=300.0, help="sleep before each timed replay (outside the events)")
     ap.add_argument("--cold-factor", type=float, default=2.5, help="replicas x footprint >= this x L2")
     ap.add_argument("--max-replicas", type=int, default=256)
+    ap.add_argument("--filter", default=None,
+                    help="time only the ops whose 'name shape' (e.g. 'all_reduce/ring 256x7168') matches this regex")
     args = ap.parse_args()
     rank, world, local = dist_env()
 
@@ -630,6 +634,13 @@ def main():
     import oracle
 
     ops, cfg = WORKLOADS[args.workload](M, oracle)
+    if args.filter:
+        import re
+        pat = re.compile(args.filter)
+        ops = [op for op in ops if pat.search(f"{op.name} {'x'.join(map(str, op.meta.get('shape', [])))}")]
+        if not ops:
+            raise SystemExit(f"--filter {args.filter!r} matches no op of workload {args.workload}")
+        cfg = {**cfg, "filter": args.filter}
     prop = torch.cuda.get_device_properties(local)
     l2 = prop.L2_cache_size
     flush = torch.empty(2 * l2 // 4, dtype=torch.int32, device="cuda")
@@ -756,20 +767,23 @@ def main():
                        "us_single": round(statistics.median(op.single) * 1e6, 3), **extra,
                        "replicas": graphs[id(op)][1], "gbs": round(gbs, 1),
                        "frac_measured_hbm": round(gbs / hbm, 4), "frac_8tbs": round(gbs / 8000, 4)})
-        k = by_kernel.setdefault(op.kernel, {"time": 0.0, "bytes": 0, "calls": 0, "launches": op.launches})
+        k = by_kernel.setdefault(op.kernel, {"time": 0.0, "bytes": 0, "calls": 0, "launches": 0})
         k["time"] += sum(op.times)
         k["bytes"] += op.per_launch_bytes * args.steps
         k["calls"] += args.steps
+        k["launches"] += op.launches * args.steps
     dom = max(by_kernel, key=lambda k: by_kernel[k]["time"])
     d = by_kernel[dom]
     avg_call = d["time"] / d["calls"]
     achieved = d["bytes"] / d["calls"] / avg_call / 1e9
-    roof = {"bound": "hbm", "kernel": dom, "launches_per_call": d["launches"], "achieved": round(achieved, 1),
+    launches_per_call = d["launches"] / d["calls"]  # an op whose form depends on size averages over its shapes
+    roof = {"bound": "hbm", "kernel": dom, "launches_per_call": round(launches_per_call, 3),
+            "achieved": round(achieved, 1),
             "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
             "peak_source": f"{hbm_src} (MEASURED_PEAKS.json hbm_gbs, burst)",
             "share_of_step": round(d["time"] / total_s, 4), "traffic": traffic_for(dom, args.workload),
             "avg_call_us": round(avg_call * 1e6, 3),
-            "avg_launch_us": round(avg_call * 1e6 / d["launches"], 3),
+            "avg_launch_us": round(avg_call * 1e6 / launches_per_call, 3),
             "algorithmic_bytes_per_call": round(d["bytes"] / d["calls"]),
             "note": "achieved = the op's algorithmic bytes / its device time; for a multi-launch op both are "
                     "spread evenly over its launches, so per launch the ratio is the same"}

@@ -81,7 +81,8 @@ typedef enum {
   COLL_ALGO_RING = 3,    /* 2(N-1) neighbour steps: RING_CLUSTER or RING_STEPS by size */
   COLL_ALGO_RING_LL = 4, /* the same ring in one launch, LL packets between ranks */
   COLL_ALGO_RING_CLUSTER = 5, /* the same ring, ranks = CTAs of a cluster, hops over DSMEM */
-  COLL_ALGO_RING_STEPS = 6    /* the same ring, one stream-ordered launch per step */
+  COLL_ALGO_RING_STEPS = 6,   /* the same ring, one stream-ordered launch per step */
+  COLL_ALGO_TWOSHOT_LL = 7    /* TWOSHOT in one launch, LL packets between ranks */
 } coll_algo_t;
 typedef enum { COLL_PROTO_SIMPLE = 0, COLL_PROTO_LL = 1, COLL_PROTO_LL128 = 2 } coll_proto_t;
 
@@ -189,18 +190,30 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    else it returns COLL_ERR_UNSUPPORTED.  `workspace` is optional:
  *    when at least 24 bytes are given, bytes 16..23 receive the status pair
  *    (COLL_DEV_TIMEOUT if a bounded wait ran out).
+ *  TWOSHOT_LL ([RLL] "Traditional LL Protocols" and the "Pro5000 ?" two-shot,
+ *    fused): the TWOSHOT segments and arithmetic (bit-identical result) in
+ *    ONE cooperative launch.  Every rank writes each 16-byte group of its
+ *    input as LL lines [4 B value | 4 B flag] into its owner's receive area;
+ *    the owner polls until every line's flag is current, reduces in rank
+ *    order, rounds once and writes the result as LL lines into every rank's
+ *    receive area; every rank polls those and stores its output.  Workspace:
+ *    coll_all_reduce_workspace_size() bytes (256 + 4 N^2 seg size-of-dtype),
+ *    256-byte aligned, zero-filled once before its first use, one call at a
+ *    time; header as RING_LL (call counter, status pair at byte offset 16,
+ *    COLL_DEV_TIMEOUT if a bounded poll ran out).  Buffers that are not
+ *    16-byte aligned take the TWOSHOT kernel.  Needs N x (CTAs per SM) to
+ *    fit on the GPU at once (COLL_ERR_UNSUPPORTED otherwise).
  *  AUTO picks TWOSHOT.  ONESHOT and TWOSHOT ignore `workspace`.
- * In place (recv[r] == send[r]) is allowed for TWOSHOT, RING, RING_LL,
- * RING_CLUSTER, RING_STEPS and AUTO. */
+ * In place (recv[r] == send[r]) is allowed for every algorithm but ONESHOT. */
 COLL_API int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size_t count,
                     coll_dtype_t dtype, coll_op_t op, coll_algo_t algo, void* workspace,
                     size_t workspace_bytes, coll_stream_t stream);
 COLL_API size_t coll_all_reduce_workspace_size(int nranks, size_t count, coll_dtype_t dtype,
                                       coll_algo_t algo);
 /* The form coll_all_reduce() runs for these arguments when nranks >= 2 and
- * count >= 1: ONESHOT, TWOSHOT, RING_LL, RING_CLUSTER or RING_STEPS (AUTO
- * and RING resolved; `aligned` != 0 when every buffer is 16-byte aligned).
- * RING_CLUSTER launches one kernel, RING_STEPS 2(N-1), the others one.
+ * count >= 1: ONESHOT, TWOSHOT, TWOSHOT_LL, RING_LL, RING_CLUSTER or
+ * RING_STEPS (AUTO and RING resolved; `aligned` != 0 when every buffer is
+ * 16-byte aligned).  RING_STEPS launches 2(N-1) kernels, the others one.
  * Returns a negative COLL_ERR_* for an invalid rank count, dtype or algo.
  * Library introspection; the sources have no counterpart. */
 COLL_API int coll_all_reduce_form(int nranks, size_t count, coll_dtype_t dtype, coll_algo_t algo,

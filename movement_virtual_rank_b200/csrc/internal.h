@@ -46,6 +46,9 @@ struct RingStepArgs {
 int launch_ring_rs_step(const RingStepArgs& a, coll_dtype_t dt, coll_op_t op, bool vec,
                         cudaStream_t s);
 
+size_t twoshot_ll_workspace(int n, size_t count, int es);
+int launch_twoshot_ll(const char* const* in, char* const* out, int n, size_t count, coll_dtype_t dt, coll_op_t op,
+                      void* workspace, int* status, cudaStream_t s);
 size_t ring_ll_workspace(int n, size_t count, int es);
 int launch_ring_ll(const char* const* in, char* const* out, int n, size_t count, coll_dtype_t dt, coll_op_t op,
                    void* workspace, int* status, cudaStream_t s);

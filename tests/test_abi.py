@@ -83,12 +83,16 @@ def test_all_reduce_form():
     assert L.coll_all_reduce_form(8, 1000, M.BF16, M.ALGO_AUTO, 1) == M.TWOSHOT
     assert L.coll_all_reduce_form(8, 1000, M.BF16, M.ONESHOT, 1) == M.ONESHOT
     assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING_STEPS, 1) == M.RING_STEPS
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, M.TWOSHOT_LL, 1) == M.TWOSHOT_LL
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, M.TWOSHOT_LL, 0) == M.TWOSHOT
     assert L.coll_all_reduce_form(0, 1000, M.BF16, M.RING, 1) == -1
     assert L.coll_all_reduce_form(8, 1000, 9, M.RING, 1) == -1
-    assert L.coll_all_reduce_form(8, 1000, M.BF16, 7, 1) == -2
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, 8, 1) == -2
     # RING and RING_STEPS: a 256-byte header, then 4 bytes of partial per element
     for algo in (M.RING, M.RING_STEPS):
         assert L.coll_all_reduce_workspace_size(8, 1000, M.BF16, algo) == 256 + 4096
+    # TWOSHOT_LL: two LL FIFOs of N x N segments (seg = 128 elements here), 8 bytes per 4
+    assert L.coll_all_reduce_workspace_size(8, 1000, M.BF16, M.TWOSHOT_LL) == 256 + 2 * 2 * 64 * 128 * 2
 
 
 def _arr(vals):

@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 
 ALGOS = {M.ONESHOT: oracle.all_reduce_one_shot, M.TWOSHOT: oracle.all_reduce_two_shot,
          M.RING: oracle.all_reduce_ring, M.RING_LL: oracle.all_reduce_ring, M.RING_STEPS: oracle.all_reduce_ring,
-         M.RING_CLUSTER: oracle.all_reduce_ring}
+         M.RING_CLUSTER: oracle.all_reduce_ring, M.TWOSHOT_LL: oracle.all_reduce_two_shot}
 
 
 def bits(a):
@@ -51,6 +51,9 @@ def test_fuzz_all_reduce(seed):
     ws = None
     if algo == M.RING_CLUSTER:  # a RING-sized workspace: the fallback for unaligned buffers or N > 8
         need = M.coll_all_reduce_workspace_size(n, count, send[0].t.dtype, M.RING)
+        ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    elif algo == M.TWOSHOT_LL:
+        need = M.coll_all_reduce_workspace_size(n, count, send[0].t.dtype, M.TWOSHOT_LL)
         ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
     M.coll_all_reduce([b.t for b in send], [b.t for b in recv], op=op, algo=algo, workspace=ws)
     torch.cuda.synchronize()
