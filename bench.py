@@ -195,9 +195,12 @@ def build_sp_prefill(M, oracle):
                  "gather": "fp32 [256,16032] -> dst 0 [256,128256]"}
 
 
+MOE_TOKENS = 4096  # tokens per rank of the MoE workload (and of the all-to-all-v split matrix); --moe-tokens
+
+
 def build_moe(M, oracle):
     import torch
-    n, tokens, topk, experts, hidden = 8, 4096, 8, 256, 7168
+    n, tokens, topk, experts, hidden = 8, MOE_TOKENS, 8, 256, 7168
     ids, ws = W.moe_routing(tokens, experts, topk, n)
     xs = W.moe_tokens(tokens, hidden, n)
     dids = [torch.from_numpy(i).cuda() for i in ids]
@@ -234,10 +237,13 @@ def build_moe(M, oracle):
                  "experts": experts, "topk": topk, "routing": "softmax(N(0,1)+log Zipf(1.1)) top-8, renormalised"}
 
 
+LL_SIZES = None  # bytes per rank of the LL sweep (default 1 KB .. 256 MB, powers of 4); --ll-sizes
+
+
 def build_ll_sweep(M, oracle, sizes=None):
     import torch
     n = 8
-    sizes = sizes or [1 << k for k in range(10, 29, 2)]
+    sizes = sizes or LL_SIZES or [1 << k for k in range(10, 29, 2)]
     ops = []
     for nbytes in sizes:
         count = nbytes // 2
@@ -344,7 +350,7 @@ def build_movement(M, oracle):
            ref=lambda: oracle.all_to_all(xs), kernel="all_to_all"),
     ]
     # all-to-all-v: the MoE workload's split matrix
-    ids, _ = W.moe_routing(4096, 256, 8, n)
+    ids, _ = W.moe_routing(MOE_TOKENS, 256, 8, n)
     sc, sd, rd, _pos = oracle.moe_route(ids, 256)
     row = 7168
     cap_s = [int(sc[s].sum()) for s in range(n)]
@@ -355,7 +361,8 @@ def build_movement(M, oracle):
                   {"send": [torch.randn(k * row, device="cuda").to(torch.bfloat16) for k in cap_s],
                    "recv": [torch.empty(k * row, dtype=torch.bfloat16, device="cuda") for k in cap_r]},
                   2 * moved, 1, {"op": "all_to_all_v", "rows": int(sc.sum()), "row_elems": row,
-                                 "splits": "MoE workload routing (Zipf 1.1, top-8, 256 experts)"},
+                                 "splits": f"MoE workload routing ({MOE_TOKENS} tokens per rank, Zipf 1.1, top-8, "
+                                           "256 experts)"},
                   inputs=["send"], outputs=["recv"], kernel="all_to_all_v"))
     for proto, pname in ((M.LL, "ll"), (M.LL128, "ll128")):
         pb = M.coll_packed_bytes(S, proto)
@@ -616,6 +623,10 @@ def main():
     ap.add_argument("--lead-us", type=float, default=300.0, help="sleep before each timed replay (outside the events)")
     ap.add_argument("--cold-factor", type=float, default=2.5, help="replicas x footprint >= this x L2")
     ap.add_argument("--max-replicas", type=int, default=256)
+    ap.add_argument("--moe-tokens", type=int, default=4096,
+                    help="tokens per rank of the MoE workload and of the all-to-all-v splits (smaller for ncu captures)")
+    ap.add_argument("--ll-sizes", default=None,
+                    help="comma-separated bytes per rank for the LL sweep (smaller for ncu captures)")
     ap.add_argument("--filter", default=None,
                     help="time only the ops whose 'name shape' (e.g. 'all_reduce/ring 256x7168') matches this regex")
     args = ap.parse_args()
@@ -633,6 +644,9 @@ def main():
     import movement_virtual_rank_b200 as M
     import oracle
 
+    global MOE_TOKENS, LL_SIZES
+    MOE_TOKENS = args.moe_tokens
+    LL_SIZES = [int(x) for x in args.ll_sizes.split(",")] if args.ll_sizes else None
     ops, cfg = WORKLOADS[args.workload](M, oracle)
     if args.filter:
         import re
