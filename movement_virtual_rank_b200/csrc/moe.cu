@@ -415,10 +415,8 @@ __global__ void __launch_bounds__(kMoveThreads) k_moe_combine(const __grid_const
         sp[k] = src[k];
         w[k] = wk[k];
       }
-      for (uint64_t u = threadIdx.x; u < relems / VN; u += blockDim.x) {
-        uint4 x[TK];
-#pragma unroll
-        for (int k = 0; k < TK; ++k) x[k] = sp[k] != nullptr ? ld16(sp[k] + u * 16) : make_uint4(0, 0, 0, 0);
+      const uint64_t units = relems / VN;
+      auto one = [&](const uint4 (&x)[TK], uint64_t u) {
         Vec<DT> acc;
 #pragma unroll
         for (int k = 0; k < TK; ++k) {
@@ -431,6 +429,23 @@ __global__ void __launch_bounds__(kMoveThreads) k_moe_combine(const __grid_const
           }
         }
         st16(out + u * 16, narrow16<DT>(acc));
+      };
+      uint64_t u = threadIdx.x;
+      for (; u + blockDim.x < units; u += 2 * blockDim.x) {  // two units per pass: 2 x TK loads in flight
+        uint4 x0[TK], x1[TK];
+#pragma unroll
+        for (int k = 0; k < TK; ++k) {
+          x0[k] = sp[k] != nullptr ? ld16(sp[k] + u * 16) : make_uint4(0, 0, 0, 0);
+          x1[k] = sp[k] != nullptr ? ld16(sp[k] + (u + blockDim.x) * 16) : make_uint4(0, 0, 0, 0);
+        }
+        one(x0, u);
+        one(x1, u + blockDim.x);
+      }
+      if (u < units) {
+        uint4 x0[TK];
+#pragma unroll
+        for (int k = 0; k < TK; ++k) x0[k] = sp[k] != nullptr ? ld16(sp[k] + u * 16) : make_uint4(0, 0, 0, 0);
+        one(x0, u);
       }
     } else if constexpr (VEC) {
       for (uint64_t u = threadIdx.x; u < relems / VN; u += blockDim.x) {
