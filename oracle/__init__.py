@@ -34,7 +34,7 @@ from .collectives import (  # noqa: F401
     all_reduce_one_shot, all_reduce_two_shot, all_reduce_ring, all_gather,
     all_to_all, all_to_all_v, segment_elems,
 )
-from .moe import moe_route, moe_dispatch, moe_combine, moe_permute_send  # noqa: F401
+from .moe import moe_route, moe_route_dedup, moe_dispatch, moe_combine, moe_permute_send  # noqa: F401
 from .packets import (  # noqa: F401
     LL, LL128, packed_bytes, pack, unpack, all_reduce_packed,
 )

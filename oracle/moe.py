@@ -74,6 +74,61 @@ def moe_route(topk_ids, n_experts: int):
     return send_counts, send_displs, recv_displs, pos
 
 
+def moe_route_dedup(topk_ids, n_experts: int):
+    """Route with one dispatched row per (token, destination rank).
+
+    The tutorial (section 8.5.1) only names dispatch designs that send a
+    token once per rank it must reach; the readings taken here:
+
+    * ``send_counts[s][d]`` is the number of tokens of source s with at least
+      one chosen expert on rank d.
+    * Send order on source s: by destination rank, then token ascending;
+      receive order on d: by source rank ascending, then the sender's order.
+    * ``pos[s][t*K + k]`` is the row of (t, rank of expert k) in that rank's
+      receive buffer, the same row for every k whose experts share a rank.
+
+    Same return values as ``moe_route``; ``moe_dispatch`` and ``moe_combine``
+    take the positions unchanged (a row reached twice is written twice with
+    the same bytes, and read once per choice).
+    """
+    n = len(topk_ids)
+    assert n_experts % n == 0
+    epr = n_experts // n
+    send_counts = np.zeros((n, n), dtype=np.int64)
+    dest = []
+    for s in range(n):
+        ids2 = np.asarray(topk_ids[s])
+        assert ids2.size == 0 or (ids2.min() >= 0 and ids2.max() < n_experts)
+        for t in range(ids2.shape[0]):
+            assert len(set(ids2[t].tolist())) == ids2.shape[1], "a token's experts must be distinct"
+        d2 = ids2.astype(np.int64) // epr  # [T, K] destination rank of every choice
+        dest.append(d2)
+        for d in range(n):
+            send_counts[s, d] = int((d2 == d).any(axis=1).sum())
+    send_displs = np.zeros((n, n), dtype=np.int64)
+    for s in range(n):
+        for d in range(1, n):
+            send_displs[s, d] = send_displs[s, d - 1] + send_counts[s, d - 1]
+    recv_displs = np.zeros((n, n), dtype=np.int64)  # [d][s]
+    for d in range(n):
+        for s in range(1, n):
+            recv_displs[d, s] = recv_displs[d, s - 1] + send_counts[s - 1, d]
+    pos = []
+    for s in range(n):
+        d2 = dest[s]
+        t_, k_ = d2.shape
+        p = np.empty(t_ * k_, dtype=np.int64)
+        for d in range(n):
+            reach = (d2 == d).any(axis=1)               # tokens of s that go to d
+            rank = np.cumsum(reach) - 1                 # their order among them
+            for t in np.nonzero(reach)[0]:
+                for k in range(k_):
+                    if d2[t, k] == d:
+                        p[t * k_ + k] = recv_displs[d, s] + rank[t]
+        pos.append(p)
+    return send_counts, send_displs, recv_displs, pos
+
+
 def moe_permute_send(xs, topk_ids, n_experts: int, hidden: int):
     """The sender-side layout: rank s's rows in send order (dest, expert, token)."""
     out = []

@@ -424,6 +424,71 @@ def pin_moe_route_counts_and_layout():
             assert seq == sorted(seq) and (not seq or seq == list(range(seq[0], seq[0] + len(seq))))
 
 
+def pin_moe_route_dedup_hand_example():
+    """Two ranks, experts 0,1 on rank 0 and 2,3 on rank 1 (the tutorial's
+    placement), three tokens, top-2; worked by hand."""
+    ids = [np.array([[0, 1], [2, 0], [3, 2]], np.int32),   # rank 0: t0 -> {0}, t1 -> {1, 0}, t2 -> {1}
+           np.array([[1, 3], [0, 1], [2, 3]], np.int32)]   # rank 1: t0 -> {0, 1}, t1 -> {0}, t2 -> {1}
+    sc, sd, rd, pos = oracle.moe_route_dedup(ids, 4)
+    assert sc.tolist() == [[2, 2], [2, 2]]
+    assert sd.tolist() == [[0, 2], [0, 2]]
+    assert rd.tolist() == [[0, 2], [0, 2]]
+    assert pos[0].tolist() == [0, 0, 0, 1, 1, 1]
+    assert pos[1].tolist() == [2, 2, 3, 3, 3, 3]
+
+
+def pin_moe_route_dedup_layout():
+    n, t, k, e = 4, 64, 4, 16
+    ids, _ = W.moe_routing(t, e, k, n)
+    sc, sd, rd, pos = oracle.moe_route_dedup(ids, e)
+    epr = e // n
+    for d in range(n):
+        got = []
+        for s in range(n):
+            d2 = ids[s] // epr
+            reach = [tt for tt in range(t) if (d2[tt] == d).any()]
+            assert sc[s, d] == len(reach)
+            rows = [int(pos[s][tt * k + kk]) for tt in reach for kk in range(k) if d2[tt, kk] == d]
+            per_tok = [{int(pos[s][tt * k + kk]) for kk in range(k) if d2[tt, kk] == d} for tt in reach]
+            assert all(len(v) == 1 for v in per_tok)  # one row per (token, destination)
+            firsts = [min(v) for v in per_tok]
+            assert firsts == list(range(rd[d, s], rd[d, s] + len(reach)))  # token order, source block
+            got.extend(firsts)
+            assert set(rows) == set(firsts)
+        assert sorted(got) == list(range(int(sc[:, d].sum())))
+    # fewer rows than (token, expert) pairs whenever two experts of a token share a rank
+    assert sc.sum() < n * t * k
+
+
+def pin_moe_route_dedup_reduces_to_route():
+    """With one expert per rank no token reaches a rank twice, and the two
+    routes (expert order inside a destination = token order) coincide."""
+    n, t, k = 8, 40, 3
+    ids, _ = W.moe_routing(t, n, k, n)
+    a = oracle.moe_route(ids, n)
+    b = oracle.moe_route_dedup(ids, n)
+    for x, y in zip(a[:3], b[:3]):
+        assert np.array_equal(x, y)
+    for s in range(n):
+        assert np.array_equal(a[3][s], b[3][s])
+
+
+def pin_moe_dedup_combine_equals_route_combine():
+    """Identity expert: dispatch then combine gives the same bits with either
+    route, since every choice reads a copy of its own token's row."""
+    n, t, k, e, h = 4, 24, 4, 16, 8
+    ids, ws = W.moe_routing(t, e, k, n)
+    xs = [W.ranks_values(W.W_MISC, n, t * h, "bf16", salt=9)[r] for r in range(n)]
+    outs = []
+    for route in (oracle.moe_route, oracle.moe_route_dedup):
+        sc, sd, rd, pos = route(ids, e)
+        bufs = [np.zeros(int(sc[:, d].sum()) * h, np.uint16) for d in range(n)]
+        ys = oracle.moe_dispatch(xs, ids, pos, bufs, e, h)
+        outs.append(oracle.moe_combine(ys, ids, pos, ws, e, h, "bf16"))
+    for s in range(n):
+        assert np.array_equal(outs[0][s], outs[1][s])
+
+
 def pin_moe_dispatch_is_permute_then_all_to_all_v():
     n, t, k, e, h = 4, 48, 4, 16, 8
     ids, ws = W.moe_routing(t, e, k, n)

@@ -132,6 +132,36 @@ def m_route_token_major(mp):
     _patch(mp, "moe_route", f)
 
 
+def m_dedup_route_is_pair_route(mp):
+    _patch(mp, "moe_route_dedup", lambda topk_ids, n_experts: M.moe_route(topk_ids, n_experts))
+
+
+def m_dedup_route_expert_order(mp):
+    """Dedup rows, but ordered inside a destination by the token's smallest
+    expert there, then token."""
+    orig = M.moe_route_dedup
+
+    def f(topk_ids, n_experts):
+        sc, sd, rd, pos = orig(topk_ids, n_experts)
+        n = len(topk_ids)
+        epr = n_experts // n
+        new = []
+        for s in range(n):
+            ids2 = np.asarray(topk_ids[s])
+            t_, k_ = ids2.shape
+            p = np.empty_like(pos[s])
+            for d in range(n):
+                reach = [t for t in range(t_) if (ids2[t] // epr == d).any()]
+                key = sorted(reach, key=lambda t: (int(ids2[t][ids2[t] // epr == d].min()), t))
+                for r, t in enumerate(key):
+                    for k in range(k_):
+                        if ids2[t, k] // epr == d:
+                            p[t * k_ + k] = rd[d, s] + r
+            new.append(p)
+        return sc, sd, rd, new
+    _patch(mp, "moe_route_dedup", f)
+
+
 def m_combine_f64(mp):
     def f(ys, topk_ids, pos, topk_w, n_experts, hidden, dtype):
         n = len(topk_ids)
