@@ -233,6 +233,33 @@ def build_moe(M, oracle):
            {"op": "moe_combine", "ranks": n, "hidden": hidden},
            inputs=["y"], outputs=["out"], kernel="moe_combine"),
     ]
+    # the route deduplicated per (token, destination rank): one row per pair reached
+    dsplit = {k: torch.empty_like(v) for k, v in split.items()}
+    dpos = [torch.empty_like(p) for p in pos]
+    M.coll_moe_route_dedup(dids, experts, dsplit["sc"], dsplit["sd"], dsplit["rd"], dpos, workspace=wsp)
+    torch.cuda.synchronize()
+    uniq = int(dsplit["sc"].sum().item())
+    dcap = int(dsplit["sc"].view(n, n).sum(0).max().item())
+    drecv = [torch.empty(dcap * hidden, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+    ops += [
+        Op("moe_route_dedup",
+           lambda b: (lambda: M.coll_moe_route_dedup(b["ids"], experts, b["sc"], b["sd"], b["rd"], b["pos"],
+                                                     workspace=b["ws"])),
+           {"ids": dids, "pos": dpos, "ws": wsp, **dsplit}, pairs * 4 * 2, 3,
+           {"op": "moe_route_dedup", "ranks": n, "tokens": tokens, "topk": topk, "experts": experts},
+           inputs=["ids"], outputs=["pos"], ref=lambda: oracle.moe_route_dedup(ids, experts), kernel="moe_route"),
+        Op("moe_dispatch_dedup",
+           lambda b: (lambda: M.coll_moe_dispatch(b["x"], b["ids"], b["pos"], b["recv"], experts)),
+           {"x": x, "ids": dids, "pos": dpos, "recv": drecv}, n * tokens * row + uniq * row, 1,
+           {"op": "moe_dispatch_dedup", "ranks": n, "hidden": hidden, "rows_out": uniq},
+           inputs=["x"], outputs=["recv"], kernel="moe_dispatch_dedup"),
+        Op("moe_combine_dedup",
+           lambda b: (lambda: M.coll_moe_combine(b["y"], b["ids"], b["pos"], b["w"], b["out"], experts)),
+           {"y": drecv, "ids": dids, "pos": dpos, "w": [torch.from_numpy(w).cuda() for w in ws],
+            "out": [torch.empty_like(t) for t in x]}, uniq * row + pairs * 4 + n * tokens * row, 1,
+           {"op": "moe_combine_dedup", "ranks": n, "hidden": hidden, "rows_in": uniq},
+           inputs=["y"], outputs=["out"], kernel="moe_combine_dedup"),
+    ]
     return ops, {"workload": "moe_dispatch_combine_8vr", "virtual_ranks": n, "tokens": tokens, "hidden": hidden,
                  "experts": experts, "topk": topk, "routing": "softmax(N(0,1)+log Zipf(1.1)) top-8, renormalised"}
 

@@ -305,11 +305,30 @@ COLL_API int coll_moe_route(const int32_t* const* topk_ids, int nranks, int toke
                    void* workspace, size_t workspace_bytes, coll_stream_t stream);
 COLL_API size_t coll_moe_route_workspace_size(int nranks, int tokens, int topk, int n_experts);
 
+/* Route deduplicated per (token, destination rank) ([TUT] 8.5.1 names
+ * dispatch designs that send a token once per rank it must reach; the
+ * tutorial gives no layout, so this one is the plainest): one row per
+ * (token, destination rank), so d_send_counts[s*N+d] is the number of tokens
+ * of source s with at least one chosen expert on rank d.  Send order on a
+ * source: destination rank, then token index; receive order as above.
+ * d_pos[s][t*topk+k] is the row of (t, rank of expert k): the same row for
+ * every k whose experts share a rank.  Dispatch and combine take these
+ * positions unchanged; dispatch writes a row reached by several choices
+ * once.  A repeated or out-of-range expert id raises COLL_DEV_BAD_ROUTE.
+ * Same arguments and workspace (coll_moe_route_workspace_size()) as
+ * coll_moe_route. */
+COLL_API int coll_moe_route_dedup(const int32_t* const* topk_ids, int nranks, int tokens, int topk,
+                         int n_experts, int64_t* d_send_counts, int64_t* d_send_displs,
+                         int64_t* d_recv_displs, int32_t* const* d_pos, int* d_status,
+                         void* workspace, size_t workspace_bytes, coll_stream_t stream);
+
 /* Dispatch (the permute and the all-to-all-v in one pass): for every source
  * s, token t and choice k, recv[d][d_pos[s][t*topk+k]] = x[s][t], a row of
  * `hidden` elements, d = topk_ids[s][t][k] / (n_experts/N).  Each token row
- * is read once.  Rows at or beyond recv_capacity_rows are not written and
- * raise COLL_DEV_SPLIT_OVERFLOW.  Bit copy. */
+ * is read once, and written once per distinct receive row (choices of a
+ * token that share a row, as a deduplicated route gives them, share the
+ * write).  Rows at or beyond recv_capacity_rows are not written and raise
+ * COLL_DEV_SPLIT_OVERFLOW.  Bit copy. */
 COLL_API int coll_moe_dispatch(const void* const* x, const int32_t* const* topk_ids,
                       const int32_t* const* d_pos, void* const* recv, int nranks, int tokens,
                       int topk, int n_experts, size_t hidden, coll_dtype_t dtype,

@@ -67,6 +67,7 @@ _SIGS = {
     "coll_ll_unpack": (_I, [_VP, _VP, _SZ, _I, _U64, _VP, _VP]),
     "coll_all_reduce_packed": (_I, [_PP, _PP, _I, _SZ, _I, _I, _I, _U64, _VP, _VP]),
     "coll_moe_route": (_I, [_PP, _I, _I, _I, _I, _VP, _VP, _VP, _PP, _VP, _VP, _SZ, _VP]),
+    "coll_moe_route_dedup": (_I, [_PP, _I, _I, _I, _I, _VP, _VP, _VP, _PP, _VP, _VP, _SZ, _VP]),
     "coll_moe_route_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "coll_moe_dispatch": (_I, [_PP, _PP, _PP, _PP, _I, _I, _I, _I, _SZ, _I, _I64, _VP, _VP]),
     "coll_moe_combine": (_I, [_PP, _PP, _PP, _PP, _PP, _I, _I, _I, _I, _SZ, _I, _I64, _VP, _VP]),
@@ -411,9 +412,10 @@ def coll_moe_route_workspace_size(nranks: int, tokens: int, topk: int, n_experts
 
 def coll_moe_route(topk_ids, n_experts: int, send_counts: torch.Tensor, send_displs: torch.Tensor,
                    recv_displs: torch.Tensor, pos, status: torch.Tensor | None = None,
-                   workspace: torch.Tensor | None = None, stream=None):
+                   workspace: torch.Tensor | None = None, stream=None, dedup: bool = False):
     """topk_ids: per rank int32 [tokens, topk]; outputs: int64 [N*N] tensors and
-    per-rank int32 [tokens*topk] positions.  ``workspace`` is allocated here when omitted."""
+    per-rank int32 [tokens*topk] positions.  ``workspace`` is allocated here when omitted.
+    ``dedup`` calls coll_moe_route_dedup (one row per (token, destination rank))."""
     topk_ids = _ranks(topk_ids, "topk_ids", torch.int32)
     pos = _ranks(pos, "pos", torch.int32)
     n = len(topk_ids)
@@ -429,9 +431,18 @@ def coll_moe_route(topk_ids, n_experts: int, send_counts: torch.Tensor, send_dis
     pi, _k1 = _ptrs(topk_ids)
     pp, _k2 = _ptrs(pos)
     with torch.cuda.device(topk_ids[0].device):
-        _check("coll_moe_route", lib().coll_moe_route(
+        fn = "coll_moe_route_dedup" if dedup else "coll_moe_route"
+        _check(fn, getattr(lib(), fn)(
             pi, n, tokens, topk, n_experts, send_counts.data_ptr(), send_displs.data_ptr(), recv_displs.data_ptr(),
             pp, st, workspace.data_ptr(), _nbytes(workspace), _stream(stream)))
+
+
+def coll_moe_route_dedup(topk_ids, n_experts: int, send_counts: torch.Tensor, send_displs: torch.Tensor,
+                         recv_displs: torch.Tensor, pos, status: torch.Tensor | None = None,
+                         workspace: torch.Tensor | None = None, stream=None):
+    """The route with one row per (token, destination rank); see coll_moe_route."""
+    coll_moe_route(topk_ids, n_experts, send_counts, send_displs, recv_displs, pos, status, workspace, stream,
+                   dedup=True)
 
 
 def coll_moe_dispatch(x, topk_ids, pos, recv, n_experts: int, status: torch.Tensor | None = None, stream=None):

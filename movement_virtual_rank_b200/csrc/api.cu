@@ -643,9 +643,10 @@ size_t coll_moe_route_workspace_size(int nranks, int tokens, int topk, int n_exp
   return moe_route_workspace(nranks, tokens, topk, n_experts);
 }
 
-int coll_moe_route(const int32_t* const* topk_ids, int nranks, int tokens, int topk, int n_experts,
-                   int64_t* d_send_counts, int64_t* d_send_displs, int64_t* d_recv_displs, int32_t* const* d_pos,
-                   int* d_status, void* workspace, size_t workspace_bytes, coll_stream_t stream) {
+static int moe_route_impl(const int32_t* const* topk_ids, int nranks, int tokens, int topk, int n_experts,
+                          int64_t* d_send_counts, int64_t* d_send_displs, int64_t* d_recv_displs,
+                          int32_t* const* d_pos, int* d_status, void* workspace, size_t workspace_bytes,
+                          coll_stream_t stream, bool dedup) {
   if (!moe_shape_ok(nranks, tokens, topk, n_experts)) return COLL_ERR_INVALID_ARG;
   if (topk_ids == nullptr || d_pos == nullptr || !d_send_counts || !d_send_displs || !d_recv_displs)
     return COLL_ERR_INVALID_ARG;
@@ -666,11 +667,30 @@ int coll_moe_route(const int32_t* const* topk_ids, int nranks, int tokens, int t
   a.topk = topk;
   a.n_experts = n_experts;
   a.tiles = std::max(1, (tokens + 255) / 256);
+  a.dedup = dedup ? 1 : 0;
+  a.buckets = dedup ? nranks : n_experts;
+  a.bpr = dedup ? 1 : n_experts / nranks;
+  // the layout of the per-expert route; the deduplicated one uses a prefix of each array
   const size_t cells = static_cast<size_t>(nranks) * n_experts * a.tiles;
   a.tile_cnt = static_cast<int32_t*>(workspace);
   a.tile_base = reinterpret_cast<int64_t*>(static_cast<char*>(workspace) + (cells * 4 + 255) / 256 * 256);
   a.status = d_status;
   return launch_moe_route(a, S(stream));
+}
+
+int coll_moe_route(const int32_t* const* topk_ids, int nranks, int tokens, int topk, int n_experts,
+                   int64_t* d_send_counts, int64_t* d_send_displs, int64_t* d_recv_displs, int32_t* const* d_pos,
+                   int* d_status, void* workspace, size_t workspace_bytes, coll_stream_t stream) {
+  return moe_route_impl(topk_ids, nranks, tokens, topk, n_experts, d_send_counts, d_send_displs, d_recv_displs, d_pos,
+                        d_status, workspace, workspace_bytes, stream, false);
+}
+
+int coll_moe_route_dedup(const int32_t* const* topk_ids, int nranks, int tokens, int topk, int n_experts,
+                         int64_t* d_send_counts, int64_t* d_send_displs, int64_t* d_recv_displs,
+                         int32_t* const* d_pos, int* d_status, void* workspace, size_t workspace_bytes,
+                         coll_stream_t stream) {
+  return moe_route_impl(topk_ids, nranks, tokens, topk, n_experts, d_send_counts, d_send_displs, d_recv_displs, d_pos,
+                        d_status, workspace, workspace_bytes, stream, true);
 }
 
 int coll_moe_dispatch(const void* const* x, const int32_t* const* topk_ids, const int32_t* const* d_pos,

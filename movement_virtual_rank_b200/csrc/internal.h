@@ -114,6 +114,9 @@ struct MoeRouteArgs {
   int64_t* tile_base;    // workspace [N][E][tiles]
   int* status;
   int n, tokens, topk, n_experts, tiles;
+  // route buckets: experts (one row per (token, expert)), or destination
+  // ranks when deduplicated (one row per (token, rank)); bpr = buckets per rank
+  int dedup, buckets, bpr;
 };
 size_t moe_route_workspace(int n, int tokens, int topk, int n_experts);
 int launch_moe_route(const MoeRouteArgs& a, cudaStream_t s);

@@ -4,19 +4,24 @@
 // per-pair lengths differ, so the exchange is an all-to-all-v).
 //
 // Route (three launches, deterministic -- no result depends on atomics'
-// order):
-//  1. k_moe_count  per (source, tile of 256 tokens): a token x expert bitmap
+// order).  A bucket is an expert (one row per (token, expert) pair) or, for
+// the route deduplicated per (token, destination rank) that the tutorial
+// names in 8.5.1, a destination rank (one row per (token, rank)):
+//  1. k_moe_count  per (source, tile of 256 tokens): a token x bucket bitmap
 //                  in shared memory gives every pair its rank among the
-//                  tile's tokens routed to the same expert (popcount of the
-//                  lower tokens' bits) and every expert its count in the tile.
-//  2. k_moe_scan   per source: exclusive scan of the counts in (expert, tile)
-//                  order = the send order (destination, expert, token); the
-//                  per-destination send counts and displacements fall out.
+//                  tile's tokens in the same bucket (popcount of the lower
+//                  tokens' bits) and every bucket its count in the tile; a
+//                  token's second expert on one rank sets the same bit again.
+//  2. k_moe_scan   per source: exclusive scan of the counts in (bucket, tile)
+//                  order = the send order (destination, expert, token), or
+//                  (destination, token); the per-destination send counts and
+//                  displacements fall out.
 //  3. k_moe_pos    per (source, tile): receive displacements (sum over lower
 //                  sources, tutorial 8.1's [from 0, from 1, ...]) plus the
 //                  pair's send offset within its destination block.
 // Dispatch: one CTA per token row at a time reads the row once and writes it
-// to its topk receive rows.  Combine: one CTA per output row reads the topk
+// to its topk receive rows, once per distinct row (a deduplicated route gives
+// the choices of a token that share a rank the same row).  Combine: one CTA per output row reads the topk
 // expert rows and forms acc = fl32(w0*y0), acc = fl32(acc + fl32(wk*yk)).
 #include <algorithm>
 
@@ -43,11 +48,13 @@ size_t moe_route_workspace(int n, int tokens, int topk, int n_experts) {
 __global__ void __launch_bounds__(kTile) k_moe_count(const __grid_constant__ MoeRouteArgs a) {
   pdl_wait();
   pdl_trigger();
-  extern __shared__ uint32_t bits[];  // [n_experts][kWords]
+  extern __shared__ uint32_t bits[];  // [buckets][kWords]
   const int s = blockIdx.x / a.tiles;
   const int tile = blockIdx.x % a.tiles;
   const int E = a.n_experts;
-  for (int i = threadIdx.x; i < E * kWords; i += blockDim.x) bits[i] = 0;
+  const int B = a.buckets;
+  const int epr = E / a.n;
+  for (int i = threadIdx.x; i < B * kWords; i += blockDim.x) bits[i] = 0;
   __syncthreads();
   const int t = threadIdx.x;
   const int tok = tile * kTile + t;
@@ -62,8 +69,13 @@ __global__ void __launch_bounds__(kTile) k_moe_count(const __grid_constant__ Moe
         ++bad;
         continue;
       }
-      const uint32_t old = atomicOr(&bits[e * kWords + (t >> 5)], me);
-      if (old & me) ++bad;  // the same expert twice for one token
+      const int b = a.dedup ? e / epr : e;
+      const uint32_t old = atomicOr(&bits[b * kWords + (t >> 5)], me);
+      if (a.dedup) {
+        for (int k2 = 0; k2 < k; ++k2) bad += ids[k2] == e;  // the same expert twice for one token
+      } else if (old & me) {
+        ++bad;
+      }
     }
   }
   __syncthreads();
@@ -72,17 +84,17 @@ __global__ void __launch_bounds__(kTile) k_moe_count(const __grid_constant__ Moe
     for (int k = 0; k < a.topk; ++k) {
       const int e = ids[k];
       if (e < 0 || e >= E) continue;
-      const uint32_t* row = bits + e * kWords;
+      const uint32_t* row = bits + (a.dedup ? e / epr : e) * kWords;
       int rank = __popc(row[t >> 5] & (me - 1u));
       for (int w = 0; w < (t >> 5); ++w) rank += __popc(row[w]);
       pos[k] = rank;  // local rank; k_moe_pos adds the block offsets
     }
   }
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
     int c = 0;
 #pragma unroll
-    for (int w = 0; w < kWords; ++w) c += __popc(bits[e * kWords + w]);
-    a.tile_cnt[(static_cast<int64_t>(s) * E + e) * a.tiles + tile] = c;
+    for (int w = 0; w < kWords; ++w) c += __popc(bits[b * kWords + w]);
+    a.tile_cnt[(static_cast<int64_t>(s) * B + b) * a.tiles + tile] = c;
   }
   report_warp(a.status, COLL_DEV_BAD_ROUTE, bad);
 }
@@ -94,7 +106,7 @@ __global__ void __launch_bounds__(kScanThreads) k_moe_scan(const __grid_constant
   pdl_trigger();
   __shared__ int64_t warp_sums[kScanThreads / 32];
   const int s = blockIdx.x;
-  const int64_t m = static_cast<int64_t>(a.n_experts) * a.tiles;  // cells of this source
+  const int64_t m = static_cast<int64_t>(a.buckets) * a.tiles;  // cells of this source
   const int32_t* cnt = a.tile_cnt + s * m;
   int64_t* base = a.tile_base + s * m;
   const int64_t per = (m + kScanThreads - 1) / kScanThreads;
@@ -129,12 +141,12 @@ __global__ void __launch_bounds__(kScanThreads) k_moe_scan(const __grid_constant
     run += cnt[i];
   }
   __syncthreads();
-  // per destination: experts [d*epr, (d+1)*epr) are cells [d*epr*tiles, (d+1)*epr*tiles)
-  const int epr = a.n_experts / a.n;
+  // per destination: buckets [d*bpr, (d+1)*bpr) are cells [d*bpr*tiles, (d+1)*bpr*tiles)
+  const int bpr = a.bpr;
   if (threadIdx.x < a.n) {
     const int d = threadIdx.x;
-    const int64_t c0 = static_cast<int64_t>(d) * epr * a.tiles;
-    const int64_t c1 = c0 + static_cast<int64_t>(epr) * a.tiles;
+    const int64_t c0 = static_cast<int64_t>(d) * bpr * a.tiles;
+    const int64_t c1 = c0 + static_cast<int64_t>(bpr) * a.tiles;
     // base[c] is visible: written above by this block, ordered by __syncthreads
     const int64_t b0 = c0 < m ? base[c0] : 0;
     int64_t total = 0;
@@ -175,19 +187,20 @@ __global__ void __launch_bounds__(kTile) k_moe_pos(const __grid_constant__ MoeRo
   const int epr = E / n;
   const int32_t* ids = a.ids[s] + static_cast<int64_t>(tok) * a.topk;
   int32_t* pos = a.pos[s] + static_cast<int64_t>(tok) * a.topk;
-  const int64_t* base = a.tile_base + static_cast<int64_t>(s) * E * a.tiles;
+  const int64_t* base = a.tile_base + static_cast<int64_t>(s) * a.buckets * a.tiles;
   for (int k = 0; k < a.topk; ++k) {
     const int e = ids[k];
     if (e < 0 || e >= E) continue;
     const int d = e / epr;
-    const int64_t off = base[static_cast<int64_t>(e) * a.tiles + tile] - sdispl[d];
+    const int b = a.dedup ? d : e;
+    const int64_t off = base[static_cast<int64_t>(b) * a.tiles + tile] - sdispl[d];
     pos[k] = static_cast<int32_t>(rdispl[d] + off + pos[k]);
   }
 }
 
 int launch_moe_route(const MoeRouteArgs& a, cudaStream_t s) {
   const unsigned grid = static_cast<unsigned>(a.n * a.tiles);
-  const size_t smem = static_cast<size_t>(a.n_experts) * kWords * sizeof(uint32_t);
+  const size_t smem = static_cast<size_t>(a.buckets) * kWords * sizeof(uint32_t);
   static int smem_set[COLL_MAX_RANKS] = {0};  // per device ordinal: largest limit set so far
   const int ok = allow_dynamic_smem(reinterpret_cast<const void*>(k_moe_count), smem, smem_set);
   if (ok != COLL_OK) return ok;
@@ -211,7 +224,8 @@ template <int U>
 __global__ void __launch_bounds__(kMoveThreads) k_moe_dispatch(const __grid_constant__ MoeMoveArgs a) {
   pdl_wait();
   pdl_trigger();
-  __shared__ char* dst[kMaxTopk];
+  __shared__ char* cand[kMaxTopk];
+  __shared__ char* dst[kMaxTopk];  // cand with repeats of an earlier choice's row dropped
   __shared__ int nbad;
   const int64_t rows = static_cast<int64_t>(a.n) * a.tokens;
   const uint64_t ru = a.row_bytes / U;
@@ -225,11 +239,18 @@ __global__ void __launch_bounds__(kMoveThreads) k_moe_dispatch(const __grid_cons
       const int64_t p = a.pos[s][j];
       const int d = e / a.epr;
       if (e < 0 || d >= a.n || p < 0 || p >= a.capacity) {
-        dst[threadIdx.x] = nullptr;
+        cand[threadIdx.x] = nullptr;
         ++bad;
       } else {
-        dst[threadIdx.x] = a.y[d] + static_cast<uint64_t>(p) * a.row_bytes;
+        cand[threadIdx.x] = a.y[d] + static_cast<uint64_t>(p) * a.row_bytes;
       }
+    }
+    __syncthreads();
+    if (threadIdx.x < a.topk) {
+      char* c = cand[threadIdx.x];
+      for (int k2 = 0; k2 < threadIdx.x; ++k2)
+        if (cand[k2] == c) c = nullptr;
+      dst[threadIdx.x] = c;
     }
     __syncthreads();
     const char* src = a.x[s] + static_cast<uint64_t>(t) * a.row_bytes;
@@ -302,8 +323,12 @@ __global__ void __launch_bounds__(32) k_moe_dispatch_tma(const __grid_constant__
     if (lane == 0) {
       ok = mbar_wait_bounded(&bar[st], (i / kDispStages) & 1) ? 1 : 0;
       if (ok) {
-        for (int k = 0; k < a.topk; ++k)
-          if (dst[st][k] != nullptr) bulk_store(dst[st][k], stage_buf + st * stage_bytes, rb);
+        for (int k = 0; k < a.topk; ++k) {
+          char* d = dst[st][k];
+          for (int k2 = 0; k2 < k && d != nullptr; ++k2)
+            if (dst[st][k2] == d) d = nullptr;  // the same row as an earlier choice: written once
+          if (d != nullptr) bulk_store(d, stage_buf + st * stage_bytes, rb);
+        }
         bulk_commit();
       }
     }
