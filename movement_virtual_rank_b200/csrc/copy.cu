@@ -19,14 +19,12 @@
 #include "common.cuh"
 #include "internal.h"
 
-// The fan-out uses bulk copies when every CTA gets at least this many tiles
-// to pipeline (below that a CTA waits for one load, then one store round,
-// and the element path is faster); compile-time tunable.
-#ifndef MVR_FANOUT_TMA_MIN_TILES_PER_CTA
-#define MVR_FANOUT_TMA_MIN_TILES_PER_CTA 4
-#endif
-
 namespace mvr {
+
+// The fan-out and the copy lists use bulk copies when every CTA gets at least
+// this many tiles to pipeline (below that a CTA waits for one load, then one
+// store round, and the element path is faster).
+constexpr uint64_t kTmaMinTilesPerCta = 4;
 
 static int pick_unit(uint64_t bits) {
   // largest power of two <= 16 that divides every address / length OR-ed into `bits`
@@ -143,7 +141,7 @@ int launch_fanout(const FanoutArgs& a, cudaStream_t s) {
   for (int q = 0; q < a.nd; ++q) bits |= reinterpret_cast<uintptr_t>(a.dst[q]);
   const uint64_t tiles = (a.bytes + kTmaTile - 1) / kTmaTile * a.ns;
   const uint64_t tma_grid = static_cast<uint64_t>(num_sms()) * 6;  // 6 x 32 KB of stages per SM
-  if ((bits & 15) == 0 && (a.bytes & 15) == 0 && tiles >= MVR_FANOUT_TMA_MIN_TILES_PER_CTA * tma_grid) {
+  if ((bits & 15) == 0 && (a.bytes & 15) == 0 && tiles >= kTmaMinTilesPerCta * tma_grid) {
     const uint64_t grid = tma_grid;
     launch_pdl(k_fanout_tma, dim3(static_cast<unsigned>(grid)), dim3(32), kTmaStages * kTmaTile, s, a);
     return launch_status(cudaGetLastError());
@@ -299,7 +297,7 @@ int launch_copy_jobs(const CopyJob* jobs, int njobs, cudaStream_t s) {
     uint64_t tiles = 0;
     for (const CopyJob& j : v) tiles += (j.bytes + kTmaTile - 1) / kTmaTile;
     const uint64_t tma_grid = static_cast<uint64_t>(num_sms()) * 6;
-    if (tiles >= MVR_FANOUT_TMA_MIN_TILES_PER_CTA * tma_grid) {
+    if (tiles >= kTmaMinTilesPerCta * tma_grid) {
       static thread_local TmaJobsArgs targs;  // ~29 KB: keep it off the stack
       for (size_t first = 0; first < v.size(); first += kMaxTmaJobs) {
         const int nj = static_cast<int>(std::min<size_t>(kMaxTmaJobs, v.size() - first));

@@ -6,7 +6,9 @@
 // of coll_all_reduce(RING) (TP communication essay; NCCL's ring kernel named
 // in "From NCCL Ring LL to PCIe IPC AllReduce"), so the result is
 // bit-identical.  CTA r of a cluster of N plays virtual rank r; the segment
-// is cut into tiles of kRcThreads x VN elements per chunk, and the clusters
+// is cut into tiles of TH x VN elements per chunk (TH = 64 threads per CTA for
+// most messages up to 512 KB per rank, whose hops then carry fewer bytes and
+// land sooner; 128 above), and the clusters
 // walk the tiles with a stride (persistent: about as many clusters as fit on
 // the GPU at once).  Thread t owns VN elements of each chunk of a tile.
 //
@@ -36,7 +38,7 @@
 
 namespace mvr {
 
-constexpr int kRcThreads = 128;
+constexpr size_t kRcSmallBytes = 512 * 1024;  // per rank: 64-thread CTAs up to here, 128 above
 constexpr int kRcMaxRanks = 8;                    // portable cluster size
 constexpr long long kRcBudgetCycles = 1ll << 28;  // about 0.14 s per wait
 constexpr long long kRcDrainCycles = 1ll << 17;   // about 70 us per slot, abort path only
@@ -101,19 +103,19 @@ __device__ __forceinline__ bool try_wait_cluster(uint64_t* bar, uint32_t parity)
   return ok != 0;
 }
 
-template <int DT, int OP>
-__global__ void __launch_bounds__(kRcThreads) k_ring_cluster(const __grid_constant__ RingClusterArgs a) {
+template <int DT, int OP, int TH>
+__global__ void __launch_bounds__(TH) k_ring_cluster(const __grid_constant__ RingClusterArgs a) {
   using A = typename Elem<DT>::A;
   using S = typename Elem<DT>::S;
   constexpr int VN = Vec<DT>::kN;  // elements per thread (16 bytes of input)
   constexpr int NQ = VN / 4;       // 16-byte pieces of fp32 / int32 partials per thread
   constexpr int ES = Elem<DT>::kSize;
-  constexpr uint64_t TE = static_cast<uint64_t>(kRcThreads) * VN;  // elements of a chunk per tile
+  constexpr uint64_t TE = static_cast<uint64_t>(TH) * VN;  // elements of a chunk per tile
   // reduce-scatter hops carry fp32 / int32 partials, all-gather hops the
   // rounded values in the storage type (16 bytes per thread)
-  constexpr uint32_t kWideBytes = kRcThreads * NQ * 16;
-  constexpr uint32_t kNarrowBytes = kRcThreads * 16;
-  constexpr uint32_t kSlotU4 = kRcThreads * NQ;  // slot size in 16-byte units
+  constexpr uint32_t kWideBytes = TH * NQ * 16;
+  constexpr uint32_t kNarrowBytes = TH * 16;
+  constexpr uint32_t kSlotU4 = TH * NQ;  // slot size in 16-byte units
   extern __shared__ __align__(16) uint4 slot_buf[];  // [slot][kSlotU4]
   __shared__ __align__(8) uint64_t bar[kRcMaxRanks];
   __shared__ uint32_t abort_word;
@@ -338,14 +340,14 @@ __global__ void __launch_bounds__(kRcThreads) k_ring_cluster(const __grid_consta
 }
 
 // clusters of n CTAs that fit on the device at once (cached per device and n)
-template <int DT, int OP>
+template <int DT, int OP, int TH>
 static uint64_t resident_clusters(int n, size_t smem, int dev) {
   static int cache[COLL_MAX_RANKS][kRcMaxRanks + 1] = {};
   const bool cached = dev >= 0 && dev < COLL_MAX_RANKS;
   if (cached && cache[dev][n] > 0) return static_cast<uint64_t>(cache[dev][n]);
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(n));
-  cfg.blockDim = dim3(kRcThreads);
+  cfg.blockDim = dim3(TH);
   cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -355,7 +357,7 @@ static uint64_t resident_clusters(int n, size_t smem, int dev) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int v = 0;
-  if (cudaOccupancyMaxActiveClusters(&v, k_ring_cluster<DT, OP>, &cfg) != cudaSuccess || v <= 0) {
+  if (cudaOccupancyMaxActiveClusters(&v, k_ring_cluster<DT, OP, TH>, &cfg) != cudaSuccess || v <= 0) {
     (void)cudaGetLastError();
     v = std::max(1, num_sms() / n);
   }
@@ -363,28 +365,28 @@ static uint64_t resident_clusters(int n, size_t smem, int dev) {
   return static_cast<uint64_t>(v);
 }
 
-template <int DT, int OP>
+template <int DT, int OP, int TH>
 static int launch_ring_cluster_t(RingClusterArgs a, cudaStream_t s) {
   constexpr int VN = Vec<DT>::kN;
-  const uint64_t per_tile = static_cast<uint64_t>(kRcThreads) * VN;
+  const uint64_t per_tile = static_cast<uint64_t>(TH) * VN;
   a.tiles = std::max<uint64_t>(1, (a.seg + per_tile - 1) / per_tile);
-  const size_t smem = static_cast<size_t>(a.n) * kRcThreads * VN * 4;
+  const size_t smem = static_cast<size_t>(a.n) * TH * VN * 4;
   static int smem_set[COLL_MAX_RANKS] = {0};  // per device ordinal: largest limit set so far
-  const int st = allow_dynamic_smem(reinterpret_cast<const void*>(k_ring_cluster<DT, OP>), smem, smem_set);
+  const int st = allow_dynamic_smem(reinterpret_cast<const void*>(k_ring_cluster<DT, OP, TH>), smem, smem_set);
   if (st != COLL_OK) return st;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
   static bool carveout_set[COLL_MAX_RANKS] = {};  // as many CTAs per SM as shared memory allows
   if (dev >= 0 && dev < COLL_MAX_RANKS && !carveout_set[dev]) {
-    if (cudaFuncSetAttribute(k_ring_cluster<DT, OP>, cudaFuncAttributePreferredSharedMemoryCarveout,
+    if (cudaFuncSetAttribute(k_ring_cluster<DT, OP, TH>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       (void)cudaGetLastError();  // a preference only
     carveout_set[dev] = true;
   }
-  const uint64_t clusters = std::min<uint64_t>(a.tiles, resident_clusters<DT, OP>(a.n, smem, dev));
+  const uint64_t clusters = std::min<uint64_t>(a.tiles, resident_clusters<DT, OP, TH>(a.n, smem, dev));
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(clusters * a.n));
-  cfg.blockDim = dim3(kRcThreads);
+  cfg.blockDim = dim3(TH);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
@@ -396,20 +398,30 @@ static int launch_ring_cluster_t(RingClusterArgs a, cudaStream_t s) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_ring_cluster<DT, OP>, a);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_ring_cluster<DT, OP, TH>, a);
   if (e != cudaSuccess) (void)cudaGetLastError();  // reported here; keep it from surfacing in a later call
   return launch_status(e);
 }
 
-template <int DT>
-static int launch_ring_cluster_dt(const RingClusterArgs& a, coll_op_t op, cudaStream_t s) {
+template <int DT, int TH>
+static int launch_ring_cluster_op(const RingClusterArgs& a, coll_op_t op, cudaStream_t s) {
   switch (op) {
-    case COLL_SUM: return launch_ring_cluster_t<DT, COLL_SUM>(a, s);
-    case COLL_MAX: return launch_ring_cluster_t<DT, COLL_MAX>(a, s);
-    case COLL_MIN: return launch_ring_cluster_t<DT, COLL_MIN>(a, s);
-    case COLL_PROD: return launch_ring_cluster_t<DT, COLL_PROD>(a, s);
+    case COLL_SUM: return launch_ring_cluster_t<DT, COLL_SUM, TH>(a, s);
+    case COLL_MAX: return launch_ring_cluster_t<DT, COLL_MAX, TH>(a, s);
+    case COLL_MIN: return launch_ring_cluster_t<DT, COLL_MIN, TH>(a, s);
+    case COLL_PROD: return launch_ring_cluster_t<DT, COLL_PROD, TH>(a, s);
   }
   return COLL_ERR_UNSUPPORTED;
+}
+
+template <int DT>
+static int launch_ring_cluster_dt(const RingClusterArgs& a, coll_op_t op, cudaStream_t s) {
+  // 64-thread CTAs for small messages, except where a chunk fits one 128-thread
+  // tile but not one 64-thread tile: one cluster then measured faster than two
+  constexpr uint64_t VN = Vec<DT>::kN;
+  const bool one_wide_tile = a.seg > 64 * VN && a.seg <= 128 * VN;
+  if (a.count * Elem<DT>::kSize <= kRcSmallBytes && !one_wide_tile) return launch_ring_cluster_op<DT, 64>(a, op, s);
+  return launch_ring_cluster_op<DT, 128>(a, op, s);
 }
 
 bool ring_cluster_supported(int n) { return n >= 2 && n <= kRcMaxRanks; }
