@@ -260,7 +260,10 @@ COLL_API int coll_all_to_all_v(const void* const* send, void* const* recv, int n
 COLL_API size_t coll_packed_bytes(size_t bytes, coll_proto_t proto);
 
 /* Encode `bytes` bytes of `src` into coll_packed_bytes(bytes, proto) bytes
- * at `packed`.  No overlap allowed. */
+ * at `packed`.  No overlap allowed.  Long 16-byte aligned LL messages go
+ * through shared memory with bulk copies, whose waits are bounded (~2 s); a
+ * wait that ran out (never seen) would leave the packet incomplete, and the
+ * unpack of it reports the lines whose flags are wrong. */
 COLL_API int coll_ll_pack(const void* src, void* packed, size_t bytes, coll_proto_t proto,
                  uint64_t step, coll_stream_t stream);
 

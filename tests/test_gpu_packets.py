@@ -176,3 +176,53 @@ def test_ll_sweep_sizes_sampled(log2):
                 seg = np.zeros(per // 2, np.uint16)
                 seg[:hi - lo] = red
                 assert np.array_equal(host[L, :per].view(np.uint16), seg)
+
+
+@pytest.mark.parametrize("proto", [M.LL, M.LL128])
+@pytest.mark.parametrize("nbytes", [16 << 20, (16 << 20) + 4, (16 << 20) + 120 * 7 + 3, 10_000_000, 3 * (1 << 22) + 1000])
+def test_pack_unpack_bulk_path(proto, nbytes):
+    """Long aligned messages take the bulk-copy codec for whole tiles and the
+    element kernels for the tail: the packet bytes are the oracle's, the
+    round trip is exact, and bytes past either buffer stay untouched."""
+    need_gpu()
+    msg = u8(nbytes, nbytes % 1000 + 5)
+    step = 0x0BAD_CAFE if proto == M.LL else (0x5A5A << 36) + 3
+    src = torch.from_numpy(msg).cuda()
+    pb = M.coll_packed_bytes(nbytes, proto)
+    packed = torch.full((pb + 256,), 0xEE, dtype=torch.uint8, device="cuda")
+    M.coll_ll_pack(src, packed[:pb], proto, step)
+    torch.cuda.synchronize()
+    assert np.array_equal(packed[:pb].cpu().numpy(), oracle.pack(msg, proto, step))
+    assert (packed[pb:] == 0xEE).all()
+    out = torch.full((nbytes + 256,), 0x33, dtype=torch.uint8, device="cuda")
+    st = status_tensor()
+    M.coll_ll_unpack(packed[:pb], out[:nbytes], proto, step, status=st)
+    torch.cuda.synchronize()
+    assert torch.equal(out[:nbytes], src)
+    assert (out[nbytes:] == 0x33).all()
+    assert st.tolist() == [0, 0]
+
+
+@pytest.mark.parametrize("proto", [M.LL, M.LL128])
+def test_unpack_counts_bad_flags_bulk_path(proto):
+    """Corrupted flags spread over the bulk-copy tiles and the tail are
+    counted exactly."""
+    need_gpu()
+    nbytes = (16 << 20) + 1000
+    msg = u8(nbytes, 77)
+    step = 9
+    pk = oracle.pack(msg, proto, step)
+    line = 8 if proto == M.LL else 128
+    flag_at = 4 if proto == M.LL else 120
+    nlines = pk.size // line
+    g = W.rng(W.W_MISC, 3, salt=78)
+    bad_lines = np.unique(np.concatenate([g.choice(nlines, 300, replace=False), [0, nlines - 1, nlines - 2]]))
+    for L in bad_lines:
+        pk[L * line + flag_at] ^= 0x40
+    packed = torch.from_numpy(pk).cuda()
+    out = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    st = status_tensor()
+    M.coll_ll_unpack(packed, out, proto, step, status=st)
+    torch.cuda.synchronize()
+    assert st.tolist() == [M.DEV_FLAG_MISMATCH, int(bad_lines.size)]
+    assert torch.equal(out, torch.from_numpy(msg).cuda())  # the data are written all the same
