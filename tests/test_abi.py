@@ -125,6 +125,17 @@ def test_invalid_arguments_rejected_on_host():
     # ring without workspace
     assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, M.RING, None, 0, None) == -5
     assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, M.RING, BASE + 0x50000000, 8, None) == -5
+    assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, M.RING_STEPS, None, 0, None) == -5
+    # fused LL two-shot: workspace missing, too small, or not 256-byte aligned
+    need = L.coll_all_reduce_workspace_size(4, 16, M.BF16, M.TWOSHOT_LL)
+    assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, M.TWOSHOT_LL, None, 0, None) == -5
+    assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, M.TWOSHOT_LL, BASE + 0x50000000, need - 1, None) == -5
+    assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, M.TWOSHOT_LL, BASE + 0x50000010, need, None) == -5
+    # a workspace inside a rank's buffer
+    assert L.coll_all_reduce(p, q, 4, 1 << 16, M.BF16, M.SUM, M.TWOSHOT_LL, BASE + 0x100, 1 << 24, None) == -3
+    # the deduplicated MoE route validates like the plain one
+    assert L.coll_moe_route_dedup(p, 4, 16, 0, 8, BASE, BASE, BASE, q, None, BASE, 1 << 20, None) == -1
+    assert L.coll_moe_route_dedup(p, 4, 16, 2, 8, BASE, BASE, BASE, q, None, BASE + 8, 1 << 20, None) == -5
     # packets: step 0, LL step with zero low word, misaligned packet buffer
     assert L.coll_ll_pack(BASE, BASE + 0x100000, 64, M.LL, 0, None) == -1
     assert L.coll_ll_pack(BASE, BASE + 0x100000, 64, M.LL, 1 << 32, None) == -1
