@@ -586,6 +586,36 @@ def cpu_cores_used() -> int:
     return 1  # numpy element-wise kernels run on the calling thread
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def empty_kernel_graph_us(stream, reps: int = 50) -> float:
+    """Context for the latency floors: device time per launch of an empty
+    (zero-cycle sleep) kernel, ``reps`` of them back to back in one CUDA graph."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(reps):
+            torch.cuda._sleep(0)
+    for _ in range(3):
+        g.replay()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    g.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    us = a.elapsed_time(b) * 1e3 / reps
+    del g
+    return round(us, 3)
+
+
 def time_oracle(ops, min_s: float = 10.0, max_s: float = 30.0):
     """Run the oracle version of the step's ops, whole steps at a time, until
     about ``min_s`` seconds of CPU work (at most ``max_s``); returns
@@ -754,9 +784,12 @@ def main():
         stream.synchronize()
         op.single = [a.elapsed_time(b) * 1e-3 for a, b in pairs[1:]]
     graph_us = {}
+    empty_us = None
     if not args.no_graph:
         with torch.cuda.stream(stream):
             graph_us = graph_latency(ops, stream)
+            if graph_us:
+                empty_us = empty_kernel_graph_us(stream)
 
     step_s = [sum(op.times[k] for op in ops) for k in range(args.steps)]
     total_s = sum(step_s)
@@ -833,7 +866,8 @@ def main():
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
         v, sample, secs = time_oracle(ops)
-        cpu = {"value": round(v, 4) if v else None, "unit": "GB/s", "cores": cpu_cores_used(), "kind": "oracle",
+        cpu = {"value": round(v, 4) if v else None, "unit": "GB/s", "cores": cpu_cores_used(), "cpu_model": cpu_model(),
+               "kind": "oracle",
                "sample": sample, "seconds": round(secs, 2)}
 
     if rank == 0:
@@ -847,7 +881,12 @@ def main():
                            "timing": "CUDA events around a CUDA-graph replay of the R calls, after a "
                                      f"{args.lead_us:.0f} us sleep kernel; op time = replay time / R"},
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-                "clocks": clocks, "wall_s_timed_region": round(wall, 3), "ops": per_op}
+                "clocks": clocks, "wall_s_timed_region": round(wall, 3),
+                "latency_floor_context": {"empty_kernel_graph_us": empty_us,
+                                          "note": "graph_us of an op (<= 256 KB per rank) is its warm back-to-back "
+                                                  "latency in a CUDA graph; an empty kernel launched the same way "
+                                                  "costs empty_kernel_graph_us"},
+                "ops": per_op}
         print(json.dumps(line), flush=True)
     graphs.clear()
     if world > 1:
@@ -879,7 +918,8 @@ def main_reference(args, rank, world):
             "warmup": args.warmup, "ms_per_step": round(total / len(times) * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "reference",
             "config": cfg,
-            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cpu_cores_used(), "kind": "oracle",
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cpu_cores_used(), "cpu_model": cpu_model(),
+                             "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
