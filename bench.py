@@ -799,36 +799,72 @@ def main():
     hbm, hbm_src = peaks()
 
     # end-to-end: host->device of each op's inputs (pinned), the call through
-    # the Python binding, device->host of its outputs; events around the three
+    # the Python binding, device->host of its outputs.  Three streams: copies
+    # in, calls, copies out.  An op's upload waits for the previous call (ops
+    # of one shape share input buffers) and, when its inputs are the previous
+    # op's outputs, for their download; so the upload of one op overlaps the
+    # download of the one before (PCIe is full duplex).  Events bracket whole
+    # steps.
     e2e = None
     if not args.no_e2e and all(op.inputs and op.outputs for op in ops):
         pinned = {id(op): ([(t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True))
                             for nm in op.inputs for t in _as_list(op.bufs[nm])],
                            [(t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True))
                             for nm in op.outputs for t in _as_list(op.bufs[nm])]) for op in ops}
-        e_ev = []
-        with torch.cuda.stream(stream):
-            for k in range(-1, args.steps):
-                for op in ops:
-                    ins, outs = pinned[id(op)]
-                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    a.record(stream)
+
+        def spans(ts):
+            return [(t.data_ptr(), t.data_ptr() + t.numel() * t.element_size()) for t in ts]
+
+        def overlap(a, b):
+            return any(x0 < y1 and y0 < x1 for x0, x1 in a for y0, y1 in b)
+
+        in_spans = {id(op): spans([d for d, _ in pinned[id(op)][0]]) for op in ops}
+        out_spans = {id(op): spans([d for d, _ in pinned[id(op)][1]]) for op in ops}
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        prev = None  # (op, call done, download done)
+        for k in range(-1, args.steps):
+            if k == 0:
+                if prev is not None:
+                    stream.wait_event(prev[2])
+                t0.record(stream)
+                s_in.wait_event(t0)
+            for op in ops:
+                ins, outs = pinned[id(op)]
+                if prev is not None:
+                    s_in.wait_event(prev[1])
+                    if overlap(in_spans[id(op)], out_spans[id(prev[0])]):
+                        s_in.wait_event(prev[2])
+                with torch.cuda.stream(s_in):
                     for d, h in ins:
                         d.copy_(h, non_blocking=True)
+                ev_in = torch.cuda.Event()
+                ev_in.record(s_in)
+                stream.wait_event(ev_in)
+                if prev is not None and overlap(out_spans[id(op)], out_spans[id(prev[0])]):
+                    stream.wait_event(prev[2])  # the previous download still reads these buffers
+                with torch.cuda.stream(stream):
                     op.run()
+                ev_run = torch.cuda.Event()
+                ev_run.record(stream)
+                s_out.wait_event(ev_run)
+                with torch.cuda.stream(s_out):
                     for d, h in outs:
                         h.copy_(d, non_blocking=True)
-                    b.record(stream)
-                    if k >= 0:
-                        e_ev.append((a, b))
-        stream.synchronize()
-        e2e_s = max_over_ranks(sum(a.elapsed_time(b) * 1e-3 for a, b in e_ev), world, "cuda")
+                ev_out = torch.cuda.Event()
+                ev_out.record(s_out)
+                prev = (op, ev_run, ev_out)
+        stream.wait_event(prev[2])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        e2e_s = max_over_ranks(t0.elapsed_time(t1) * 1e-3, world, "cuda")
         h2d = sum(d.numel() * d.element_size() for op in ops for d, _ in pinned[id(op)][0])
         d2h = sum(d.numel() * d.element_size() for op in ops for d, _ in pinned[id(op)][1])
         e2e = {"value": round(world * bytes_step * args.steps / e2e_s / 1e9, 3), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "how": "per op: pinned host->device copy of its inputs, the call through the Python binding of the "
-                      "C ABI, device->host copy of its outputs; CUDA events around the three"}
+                      "C ABI, device->host copy of its outputs, on three streams (an upload overlaps the previous "
+                      "op's download); CUDA events around the timed steps"}
 
     per_op, by_kernel = [], {}
     for op in ops:
