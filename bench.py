@@ -106,7 +106,8 @@ def _dev(a: np.ndarray, dtype):
     return torch.from_numpy(np.ascontiguousarray(a).view(view).copy()).view(dtype).cuda()
 
 
-FORM_NAMES = {1: "oneshot", 2: "twoshot", 4: "ring_ll", 5: "ring_cluster", 6: "ring_steps"}
+FORM_NAMES = {1: "oneshot", 2: "twoshot", 4: "ring_ll", 5: "ring_cluster", 6: "ring_steps", 7: "twoshot_ll",
+              8: "ring_cta"}
 
 
 def build_tp_decode(M, oracle):
@@ -304,7 +305,8 @@ def build_ring_compare(M, oracle):
     ranks, bf16): the ring as one launch per step (RING_STEPS), as one
     cooperative launch with LL packets between ranks (RING_LL) and as one
     launch of 8-CTA clusters with the hops over distributed shared memory
-    (RING_CLUSTER); the two-shot with LL packets fused into one cooperative
+    (RING_CLUSTER) and as one launch whose CTAs hold all 8 ranks as warp
+    groups, the hops in shared memory (RING_CTA); the two-shot with LL packets fused into one cooperative
     launch (TWOSHOT_LL); and the stream-ordered packet path of the LL sweep
     (per-rank LL pack, packetised two-shot, per-rank unpack)."""
     import torch
@@ -316,7 +318,8 @@ def build_ring_compare(M, oracle):
         S = count * 2
         send = [_dev(x, torch.bfloat16) for x in xs]
         for algo, aname, launches in ((M.RING_STEPS, "ring_steps", 2 * (n - 1)), (M.RING_LL, "ring_ll", 1),
-                                      (M.RING_CLUSTER, "ring_cluster", 1), (M.TWOSHOT_LL, "twoshot_ll", 1)):
+                                      (M.RING_CLUSTER, "ring_cluster", 1), (M.RING_CTA, "ring_cta", 1),
+                                      (M.TWOSHOT_LL, "twoshot_ll", 1)):
             need = max(64, M.coll_all_reduce_workspace_size(n, count, torch.bfloat16, algo))
             ops.append(Op(f"all_reduce/{aname}",
                           lambda b, algo=algo: (lambda: M.coll_all_reduce(b["send"], b["recv"], algo=algo,
@@ -347,6 +350,7 @@ def build_ring_compare(M, oracle):
     return ops, {"workload": "ring_compare_8vr", "virtual_ranks": n, "shapes": W.tp_decode_shapes(),
                  "variants": ["ring_steps (launch per step)", "ring_ll (one launch, LL packets)",
                               "ring_cluster (one launch, cluster DSMEM hops)",
+                              "ring_cta (one launch, ranks as warp groups, shared-memory hops)",
                               "twoshot_ll (one launch, LL packets, fused)",
                               "LL pack + packetised two-shot + unpack (stream-ordered)"]}
 

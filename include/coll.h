@@ -82,7 +82,8 @@ typedef enum {
   COLL_ALGO_RING_LL = 4, /* the same ring in one launch, LL packets between ranks */
   COLL_ALGO_RING_CLUSTER = 5, /* the same ring, ranks = CTAs of a cluster, hops over DSMEM */
   COLL_ALGO_RING_STEPS = 6,   /* the same ring, one stream-ordered launch per step */
-  COLL_ALGO_TWOSHOT_LL = 7    /* TWOSHOT in one launch, LL packets between ranks */
+  COLL_ALGO_TWOSHOT_LL = 7,   /* TWOSHOT in one launch, LL packets between ranks */
+  COLL_ALGO_RING_CTA = 8      /* the same ring, ranks = warp groups of one CTA, hops in shared memory */
 } coll_algo_t;
 typedef enum { COLL_PROTO_SIMPLE = 0, COLL_PROTO_LL = 1, COLL_PROTO_LL128 = 2 } coll_proto_t;
 
@@ -190,6 +191,14 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    else it returns COLL_ERR_UNSUPPORTED.  `workspace` is optional:
  *    when at least 24 bytes are given, bytes 16..23 receive the status pair
  *    (COLL_DEV_TIMEOUT if a bounded wait ran out).
+ *  RING_CTA: the RING schedule, chunk order and rounding (bit-identical
+ *    result) in one launch in which every CTA holds all N virtual ranks,
+ *    one group of 32 threads each: each hop is a store into shared memory
+ *    of the same SM plus an mbarrier arrive, so the partials never leave
+ *    the SM.  The CTAs (up to two per SM) walk the message tile by tile.
+ *    Needs 2 <= N <= 8 and 16-byte aligned buffers, with the same fallback
+ *    and the same optional `workspace` (status pair at bytes 16..23) as
+ *    RING_CLUSTER.
  *  TWOSHOT_LL ([RLL] "Traditional LL Protocols" and the "Pro5000 ?" two-shot,
  *    fused): the TWOSHOT segments and arithmetic (bit-identical result) in
  *    ONE cooperative launch.  Every rank writes each 16-byte group of its
@@ -211,8 +220,8 @@ COLL_API int coll_all_reduce(const void* const* send, void* const* recv, int nra
 COLL_API size_t coll_all_reduce_workspace_size(int nranks, size_t count, coll_dtype_t dtype,
                                       coll_algo_t algo);
 /* The form coll_all_reduce() runs for these arguments when nranks >= 2 and
- * count >= 1: ONESHOT, TWOSHOT, TWOSHOT_LL, RING_LL, RING_CLUSTER or
- * RING_STEPS (AUTO and RING resolved; `aligned` != 0 when every buffer is
+ * count >= 1: ONESHOT, TWOSHOT, TWOSHOT_LL, RING_LL, RING_CLUSTER, RING_CTA
+ * or RING_STEPS (AUTO and RING resolved; `aligned` != 0 when every buffer is
  * 16-byte aligned).  RING_STEPS launches 2(N-1) kernels, the others one.
  * Returns a negative COLL_ERR_* for an invalid rank count, dtype or algo.
  * Library introspection; the sources have no counterpart. */

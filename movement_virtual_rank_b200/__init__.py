@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libmvrcoll.so")
 
 BF16, FP16, FP32, INT32 = 0, 1, 2, 3
 SUM, MAX, MIN, PROD = 0, 1, 2, 3
-ALGO_AUTO, ONESHOT, TWOSHOT, RING, RING_LL, RING_CLUSTER, RING_STEPS, TWOSHOT_LL = 0, 1, 2, 3, 4, 5, 6, 7
+ALGO_AUTO, ONESHOT, TWOSHOT, RING, RING_LL, RING_CLUSTER, RING_STEPS, TWOSHOT_LL, RING_CTA = 0, 1, 2, 3, 4, 5, 6, 7, 8
 SIMPLE, LL, LL128 = 0, 1, 2
 DEV_OK, DEV_FLAG_MISMATCH, DEV_TIMEOUT, DEV_SPLIT_OVERFLOW, DEV_BAD_ROUTE = 0, 1, 2, 3, 4
 MAX_RANKS = 64
@@ -31,7 +31,8 @@ _DTYPES = {torch.bfloat16: BF16, torch.float16: FP16, torch.float32: FP32, torch
 _ESIZE = {BF16: 2, FP16: 2, FP32: 4, INT32: 4}
 OPS = {"sum": SUM, "max": MAX, "min": MIN, "prod": PROD}
 ALGOS = {"auto": ALGO_AUTO, "oneshot": ONESHOT, "twoshot": TWOSHOT, "ring": RING, "ring_ll": RING_LL,
-         "ring_cluster": RING_CLUSTER, "ring_steps": RING_STEPS, "twoshot_ll": TWOSHOT_LL}
+         "ring_cluster": RING_CLUSTER, "ring_steps": RING_STEPS, "twoshot_ll": TWOSHOT_LL,
+         "ring_cta": RING_CTA}
 PROTOS = {"simple": SIMPLE, "ll": LL, "ll128": LL128}
 
 
@@ -241,7 +242,7 @@ def coll_all_reduce_workspace_size(nranks: int, count: int, dtype: torch.dtype, 
 
 def coll_all_reduce_form(nranks: int, count: int, dtype: torch.dtype, algo=TWOSHOT, aligned: bool = True) -> int:
     """The form coll_all_reduce() runs: ONESHOT, TWOSHOT, TWOSHOT_LL, RING_LL,
-    RING_CLUSTER (one launch each) or RING_STEPS (2(N-1) launches)."""
+    RING_CLUSTER, RING_CTA (one launch each) or RING_STEPS (2(N-1) launches)."""
     algo = ALGOS[algo] if isinstance(algo, str) else int(algo)
     rc = int(lib().coll_all_reduce_form(nranks, count, _DTYPES[dtype], algo, 1 if aligned else 0))
     if rc < 0:
@@ -255,8 +256,8 @@ def coll_all_reduce(send, recv, op="sum", algo=TWOSHOT, workspace: torch.Tensor 
     coll_all_reduce_workspace_size() bytes (zero-filled before its first
     RING_LL / TWOSHOT_LL use) and get a zeroed one allocated here when it
     is omitted;
-    RING_CLUSTER uses one, when given, for its status pair and its fallback
-    to RING_STEPS."""
+    RING_CLUSTER and RING_CTA use one, when given, for their status pair and
+    their fallback to RING_STEPS."""
     algo = ALGOS[algo] if isinstance(algo, str) else int(algo)
     send = _ranks(send, "send", send[0].dtype)
     recv = _ranks(recv, "recv", send[0].dtype)

@@ -87,7 +87,10 @@ def test_all_reduce_form():
     assert L.coll_all_reduce_form(8, 1000, M.BF16, M.TWOSHOT_LL, 0) == M.TWOSHOT
     assert L.coll_all_reduce_form(0, 1000, M.BF16, M.RING, 1) == -1
     assert L.coll_all_reduce_form(8, 1000, 9, M.RING, 1) == -1
-    assert L.coll_all_reduce_form(8, 1000, M.BF16, 8, 1) == -2
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING_CTA, 1) == M.RING_CTA
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING_CTA, 0) == M.RING_STEPS
+    assert L.coll_all_reduce_form(9, 1000, M.BF16, M.RING_CTA, 1) == M.RING_STEPS
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, 9, 1) == -2
     # RING and RING_STEPS: a 256-byte header, then 4 bytes of partial per element
     for algo in (M.RING, M.RING_STEPS):
         assert L.coll_all_reduce_workspace_size(8, 1000, M.BF16, algo) == 256 + 4096

@@ -128,32 +128,40 @@ def test_bounded_wait_times_out_and_context_survives():
     assert all(np.array_equal(g, w) for g, w in zip(got, want))
 
 
-# --------------------------------------------------------- cluster ring ----
+# ------------------------------------------- cluster ring and CTA ring ----
+# RING_CLUSTER (ranks = CTAs of a cluster, hops over distributed shared
+# memory) and RING_CTA (ranks = warp groups of one CTA, hops in its shared
+# memory) take the same tests.
 
-def run_cluster(xs, dtype, op, in_place=False, ws=None):
+ONE_LAUNCH = pytest.mark.parametrize("algo", [M.RING_CLUSTER, M.RING_CTA], ids=["cluster", "cta"])
+
+
+def run_cluster(xs, dtype, op, in_place=False, ws=None, algo=M.RING_CLUSTER):
     send = [to_dev(x, dtype) for x in xs]
     recv = send if in_place else [torch.empty_like(t) for t in send]
-    M.coll_all_reduce(send, recv, op=op, algo=M.RING_CLUSTER, workspace=ws)
+    M.coll_all_reduce(send, recv, op=op, algo=algo, workspace=ws)
     torch.cuda.synchronize()
     return [from_dev(t, dtype) for t in recv]
 
 
+@ONE_LAUNCH
 @pytest.mark.parametrize("n", [2, 3, 4, 5, 8])
 @pytest.mark.parametrize("count", [1, 9, 8 * 37 + 3, 65536 + 24, 300007])
-def test_ring_cluster_bf16_sum(n, count):
+def test_ring_cluster_bf16_sum(algo, n, count):
     """Virtual ranks as the CTAs of a thread-block cluster, hops over
     distributed shared memory: bit-identical to the ring oracle."""
     need_gpu()
     xs = W.ranks_values(W.W_MISC, n, count, "bf16", "normal", salt=count + 11 * n)
     want = oracle.all_reduce_ring(xs, 0, "bf16")
-    got = run_cluster(xs, "bf16", 0, in_place=(count % 2 == 1))
+    got = run_cluster(xs, "bf16", 0, in_place=(count % 2 == 1), algo=algo)
     for q in range(n):
         assert np.array_equal(got[q], want[q]), q
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp16", "fp32", "int32"])
 @pytest.mark.parametrize("op", [0, 1, 2, 3])
-def test_ring_cluster_dtypes_ops(dtype, op):
+@ONE_LAUNCH
+def test_ring_cluster_dtypes_ops(algo, dtype, op):
     need_gpu()
     n, count = 7, 12301
     if dtype == "int32":
@@ -163,23 +171,25 @@ def test_ring_cluster_dtypes_ops(dtype, op):
         xs = W.ranks_values(W.W_MISC, n, count, dtype, "uniform" if op == 3 else "normal", salt=op + 90)
     want = oracle.all_reduce_ring(xs, op, dtype)
     ws = torch.zeros(64, dtype=torch.uint8, device="cuda")
-    got = run_cluster(xs, dtype, op, ws=ws)
+    got = run_cluster(xs, dtype, op, ws=ws, algo=algo)
     for q in range(n):
         assert np.array_equal(bits(got[q]), bits(want[q])), q
     assert ws[16:24].view(torch.int32).tolist() == [0, 0]
 
 
-def test_ring_cluster_tp_decode_workload():
+@ONE_LAUNCH
+def test_ring_cluster_tp_decode_workload(algo):
     need_gpu()
     for tokens, hidden in W.tp_decode_shapes():
         xs = W.tp_decode(tokens, hidden)
-        got = run_cluster(xs, "bf16", 0)
+        got = run_cluster(xs, "bf16", 0, algo=algo)
         want = oracle.all_reduce_ring(xs, 0, "bf16")
         for q in range(8):
             assert np.array_equal(got[q], want[q]), (tokens, hidden, q)
 
 
-def test_ring_cluster_fallbacks():
+@ONE_LAUNCH
+def test_ring_cluster_fallbacks(algo):
     """Unaligned buffers or more than 8 ranks: with a RING workspace the call
     takes the RING path (same result); without one it is refused."""
     need_gpu()
@@ -191,10 +201,10 @@ def test_ring_cluster_fallbacks():
         send[r].copy_(to_dev(xs[r], "bf16"))
     recv = [torch.empty(count + 8, dtype=torch.bfloat16, device="cuda")[3:count + 3] for _ in range(n)]
     with pytest.raises(M.CollError):
-        M.coll_all_reduce(send, recv, algo=M.RING_CLUSTER)
+        M.coll_all_reduce(send, recv, algo=algo)
     ws = torch.zeros(M.coll_all_reduce_workspace_size(n, count, torch.bfloat16, M.RING), dtype=torch.uint8,
                      device="cuda")
-    M.coll_all_reduce(send, recv, algo=M.RING_CLUSTER, workspace=ws)
+    M.coll_all_reduce(send, recv, algo=algo, workspace=ws)
     torch.cuda.synchronize()
     want = oracle.all_reduce_ring(xs, 0, "bf16")
     for q in range(n):
@@ -202,14 +212,15 @@ def test_ring_cluster_fallbacks():
     xs9 = W.ranks_values(W.W_MISC, 9, 1000, "bf16", "normal", salt=79)
     ws9 = torch.zeros(M.coll_all_reduce_workspace_size(9, 1000, torch.bfloat16, M.RING), dtype=torch.uint8,
                       device="cuda")
-    got = run_cluster(xs9, "bf16", 0, ws=ws9)
+    got = run_cluster(xs9, "bf16", 0, ws=ws9, algo=algo)
     want = oracle.all_reduce_ring(xs9, 0, "bf16")
     assert all(np.array_equal(g, w) for g, w in zip(got, want))
 
 
 @pytest.mark.parametrize("n,count,dtype", [(2, 3_000_017, "bf16"), (5, 2_500_001, "bf16"), (8, 4_194_311, "bf16"),
                                            (3, 2_000_003, "fp32"), (8, 1_048_583, "int32"), (7, 999_999, "fp16")])
-def test_ring_cluster_many_tiles(n, count, dtype):
+@ONE_LAUNCH
+def test_ring_cluster_many_tiles(algo, n, count, dtype):
     """Messages of many tiles per cluster (the clusters walk the tiles, two
     slot sets alternating), with a ragged tail."""
     need_gpu()
@@ -219,14 +230,15 @@ def test_ring_cluster_many_tiles(n, count, dtype):
     else:
         xs = W.ranks_values(W.W_MISC, n, count, dtype, "normal", salt=count % 977)
     ws = torch.zeros(64, dtype=torch.uint8, device="cuda")
-    got = run_cluster(xs, dtype, 0, in_place=(n % 2 == 1), ws=ws)
+    got = run_cluster(xs, dtype, 0, in_place=(n % 2 == 1), ws=ws, algo=algo)
     want = oracle.all_reduce_ring(xs, 0, dtype)
     for q in range(n):
         assert np.array_equal(bits(got[q]), bits(want[q])), q
     assert ws[16:24].view(torch.int32).tolist() == [0, 0]
 
 
-def test_ring_cluster_back_to_back():
+@ONE_LAUNCH
+def test_ring_cluster_back_to_back(algo):
     """Consecutive calls on one stream (the next launch may start early and
     wait for this one): every result matches."""
     need_gpu()
@@ -236,7 +248,7 @@ def test_ring_cluster_back_to_back():
     outs = []
     for _ in range(3):
         recv = [torch.empty_like(t) for t in send]
-        M.coll_all_reduce(send, recv, algo=M.RING_CLUSTER)
+        M.coll_all_reduce(send, recv, algo=algo)
         outs.append(recv)
     torch.cuda.synchronize()
     want = oracle.all_reduce_ring(xs, 0, "bf16")
@@ -256,7 +268,7 @@ def test_ring_forms_agree(tokens, hidden):
     form = M.coll_all_reduce_form(n, count, torch.bfloat16, M.RING)
     assert form == (M.RING_CLUSTER if count * 2 <= 5 << 19 else M.RING_STEPS)
     want = oracle.all_reduce_ring(xs, 0, "bf16")
-    for algo in (M.RING, M.RING_STEPS, M.RING_CLUSTER):
+    for algo in (M.RING, M.RING_STEPS, M.RING_CLUSTER, M.RING_CTA):
         send = [to_dev(x, "bf16") for x in xs]
         recv = [torch.empty_like(t) for t in send]
         ws = torch.zeros(M.coll_all_reduce_workspace_size(n, count, torch.bfloat16, M.RING), dtype=torch.uint8,
