@@ -298,13 +298,11 @@ int coll_reduce_scatter(const void* const* send, void* const* recv, int nranks, 
 }
 
 // ------------------------------------------------------------- AllReduce ----
-// RING runs as one cluster launch up to this many bytes per rank (where it
-// measured faster on B200 than the stream-ordered steps), as steps above it
-constexpr size_t kRingClusterMaxBytes = size_t(5) << 19;  // 2.5 MiB
-
-static coll_algo_t ring_form(int nranks, size_t bytes, bool vec) {
-  return (vec && ring_cluster_supported(nranks) && bytes <= kRingClusterMaxBytes) ? COLL_ALGO_RING_CLUSTER
-                                                                                  : COLL_ALGO_RING_STEPS;
+// RING runs as one launch of CTAs that each hold all ranks (RING_CTA) when
+// the buffers allow it: on B200 that measured faster than the cluster form
+// and the stream-ordered steps at every size tried (8 KB .. 32 MiB per rank)
+static coll_algo_t ring_form(int nranks, bool vec) {
+  return (vec && ring_cta_supported(nranks)) ? COLL_ALGO_RING_CTA : COLL_ALGO_RING_STEPS;
 }
 
 size_t coll_all_reduce_workspace_size(int nranks, size_t count, coll_dtype_t dtype, coll_algo_t algo) {
@@ -323,7 +321,7 @@ int coll_all_reduce_form(int nranks, size_t count, coll_dtype_t dtype, coll_algo
   const bool vec = aligned != 0;
   switch (algo) {
     case COLL_ALGO_AUTO: return COLL_ALGO_TWOSHOT;
-    case COLL_ALGO_RING: return ring_form(nranks, count * es, vec);
+    case COLL_ALGO_RING: return ring_form(nranks, vec);
     case COLL_ALGO_RING_LL: return vec ? COLL_ALGO_RING_LL : COLL_ALGO_RING_STEPS;
     case COLL_ALGO_TWOSHOT_LL: return vec ? COLL_ALGO_TWOSHOT_LL : COLL_ALGO_TWOSHOT;
     case COLL_ALGO_RING_CLUSTER:
@@ -362,7 +360,7 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
   bool vec = true;
   for (int r = 0; r < nranks; ++r) vec = vec && al16(send[r]) && al16(recv[r]);
   const size_t seg = seg_elems(count, nranks, es);
-  if (algo == COLL_ALGO_RING) algo = ring_form(nranks, bytes, vec);  // workspace checked above
+  if (algo == COLL_ALGO_RING) algo = ring_form(nranks, vec);  // workspace checked above
   if (algo == COLL_ALGO_RING_CLUSTER || algo == COLL_ALGO_RING_CTA) {
     const bool has_ws = workspace != nullptr && workspace_bytes >= 24;
     const bool cta = algo == COLL_ALGO_RING_CTA;

@@ -69,14 +69,13 @@ def test_workspace_sizes():
 def test_all_reduce_form():
     """Which form coll_all_reduce runs (host logic only, no device call)."""
     L = M.lib()
-    limit = 5 << 19  # 2.5 MiB per rank
-    assert L.coll_all_reduce_form(8, limit // 2, M.BF16, M.RING, 1) == M.RING_CLUSTER
-    assert L.coll_all_reduce_form(8, limit // 2 + 1, M.BF16, M.RING, 1) == M.RING_STEPS
-    assert L.coll_all_reduce_form(8, limit // 4, M.FP32, M.RING, 1) == M.RING_CLUSTER
-    assert L.coll_all_reduce_form(8, 256 * 7168, M.BF16, M.RING, 1) == M.RING_STEPS
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING, 1) == M.RING_CTA
+    assert L.coll_all_reduce_form(8, 256 * 7168, M.BF16, M.RING, 1) == M.RING_CTA
+    assert L.coll_all_reduce_form(8, 1 << 30, M.FP32, M.RING, 1) == M.RING_CTA  # every size
     assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING, 0) == M.RING_STEPS  # unaligned
-    assert L.coll_all_reduce_form(9, 1000, M.BF16, M.RING, 1) == M.RING_STEPS  # beyond a portable cluster
-    assert L.coll_all_reduce_form(2, 1000, M.BF16, M.RING, 1) == M.RING_CLUSTER
+    assert L.coll_all_reduce_form(9, 1000, M.BF16, M.RING, 1) == M.RING_STEPS  # more ranks than a CTA holds
+    assert L.coll_all_reduce_form(2, 1000, M.BF16, M.RING, 1) == M.RING_CTA
+    assert L.coll_all_reduce_form(8, 5 << 20, M.BF16, M.RING_CLUSTER, 1) == M.RING_CLUSTER
     assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING_CLUSTER, 0) == M.RING_STEPS
     assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING_LL, 1) == M.RING_LL
     assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING_LL, 0) == M.RING_STEPS

@@ -259,14 +259,14 @@ def test_ring_cluster_back_to_back(algo):
 
 @pytest.mark.parametrize("tokens,hidden", [(1, 4096), (32, 7168), (160, 8192), (161, 8192), (256, 7168)])
 def test_ring_forms_agree(tokens, hidden):
-    """RING takes the one-launch cluster form up to 2.5 MiB per rank and the
-    stream-ordered steps above; both forms give the same bits, and the
+    """RING takes the one-launch CTA form for aligned buffers; every form
+    (CTA, cluster, stream-ordered steps) gives the same bits, and the
     workspace header's status pair stays clear."""
     need_gpu()
     xs = W.tp_decode(tokens, hidden)
     n, count = len(xs), tokens * hidden
     form = M.coll_all_reduce_form(n, count, torch.bfloat16, M.RING)
-    assert form == (M.RING_CLUSTER if count * 2 <= 5 << 19 else M.RING_STEPS)
+    assert form == M.RING_CTA
     want = oracle.all_reduce_ring(xs, 0, "bf16")
     for algo in (M.RING, M.RING_STEPS, M.RING_CLUSTER, M.RING_CTA):
         send = [to_dev(x, "bf16") for x in xs]
