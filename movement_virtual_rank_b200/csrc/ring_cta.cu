@@ -20,9 +20,10 @@
 // dependencies keep a sender within N-1 hops of its receiver, so N slots per
 // group need no credits.
 //
-// The kernel is bound by instruction issue, not by HBM, so the tiles in which
-// every chunk is full (all but the last one or two of a chunk) take a path
-// with no bounds checks and with chunk offsets stepped by one addition.
+// The kernel is bound by instruction issue, not by HBM, so the tiles that are
+// full in every chunk (those that end within the last chunk, the shortest)
+// take a path with no bounds checks and with chunk offsets stepped by one
+// addition; the other tiles check each vector against its chunk's end.
 //
 // Every wait is bounded: a thread whose wait runs out raises COLL_DEV_TIMEOUT
 // and sets the CTA's abort word; the others stop at their next wait, and all
