@@ -223,6 +223,15 @@ def m_ring_starts_at_owner(mp):
     _patch(mp, "all_reduce_ring", f)
 
 
+def m_ring_partials_in_storage_type(mp):
+    """the ring rounds its partials to the storage type at every hop (a
+    bf16 wire type) instead of carrying fp32 to the owner"""
+    def f(acc, v, op, dtype):
+        r = _orig_combine(acc, v, op, dtype)
+        return _orig_widen(_orig_narrow(r, dtype), dtype) if dtype in ("bf16", "fp16") else r
+    mp.setattr(C, "combine", f)
+
+
 def m_segment_unaligned(mp):
     _patch(mp, "segment_elems", lambda count, n, dtype: -(-count // n) + 1)
 

@@ -9,6 +9,10 @@ the oracle's own arithmetic:
 * the ring's rotated order can change a floating-point sum only by rounding,
   but integer sums (mod 2^32) and MAX / MIN of distinct finite values are
   order-free, so there the ring equals the rank-order reduction exactly;
+* where every fp32 partial is exact, the bf16 ring sum is the exact sum
+  rounded once (to nearest even, as torch rounds it), whatever the order;
+  elsewhere its error stays within 2^-8 (half a bf16 ulp, relative) of the
+  sum of the magnitudes, plus the fp32 partials' own error;
 * movement composes: gather then scatter returns every rank's block, and an
   all-to-all-v followed by the transposed one returns every rank's rows;
 * unpack(pack(message)) is the message with no flag mismatch, for LL and LL128;
@@ -17,6 +21,7 @@ the oracle's own arithmetic:
 """
 import numpy as np
 import pytest
+import torch
 from hypothesis import given, settings, strategies as st
 
 import oracle
@@ -82,6 +87,45 @@ def test_ring_max_min_of_distinct_values_are_order_free(n, count, op, seed):
     ref = oracle.all_reduce(xs, op, "fp32")
     for q, y in enumerate(oracle.all_reduce_ring(xs, op, "fp32")):
         assert np.array_equal(bits(y), bits(ref[q]))
+
+
+def bf16_bits_of(x64):
+    """torch's round-to-nearest-even of fp64 values that fp32 holds exactly"""
+    t = torch.from_numpy(np.asarray(x64, np.float64).astype(np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def bf16_value(bits):
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+@SET
+@given(n=st.integers(2, 9), count=st.integers(1, 300), seed=st.integers(0, 10**6))
+def test_ring_bf16_sum_of_exact_partials_is_the_rounded_exact_sum(n, count, seed):
+    g = np.random.default_rng(seed)
+    # k * 2^-e with |k| < 256 and 0 <= e <= 8: exact in bf16 (8 significant
+    # bits), while any partial sum of up to 9 of them lies on the 2^-8 grid
+    # below 2^12 and so is exact in fp32 (20 bits) but usually needs more
+    # bits than bf16 has: only the final rounding may act
+    v = g.integers(-255, 256, (n, count)) * 2.0 ** -g.integers(0, 9, (n, count))
+    xs = [bf16_bits_of(x) for x in v]
+    assert all(np.array_equal(bf16_value(x), w) for x, w in zip(xs, v))
+    want = bf16_bits_of(v.sum(axis=0))
+    for y in oracle.all_reduce_ring(xs, 0, "bf16"):
+        assert np.array_equal(y, want)
+
+
+@SET
+@given(n=st.integers(2, 9), count=st.integers(1, 300), seed=st.integers(0, 10**6))
+def test_ring_bf16_sum_error_is_bounded_by_the_magnitudes(n, count, seed):
+    g = np.random.default_rng(seed)
+    xs = [bf16_bits_of(g.standard_normal(count) * 4) for _ in range(n)]
+    vals = np.stack([bf16_value(x) for x in xs])
+    exact = vals.sum(axis=0)  # fp64: exact for these magnitudes
+    # one final rounding (<= 2^-8 relative) and n - 1 fp32 additions (<= 2^-24 each)
+    tol = (2.0 ** -8 + (n - 1) * 2.0 ** -24) * np.abs(vals).sum(axis=0) + 2.0 ** -133
+    for y in oracle.all_reduce_ring(xs, 0, "bf16"):
+        assert np.all(np.abs(bf16_value(y) - exact) <= tol)
 
 
 @SET
