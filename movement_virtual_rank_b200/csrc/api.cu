@@ -315,6 +315,7 @@ size_t coll_all_reduce_workspace_size(int nranks, size_t count, coll_dtype_t dty
 }
 
 int coll_all_reduce_form(int nranks, size_t count, coll_dtype_t dtype, coll_algo_t algo, int aligned) {
+  (void)count;  // no form depends on the size today; the ABI keeps it for choices that will
   const int es = elem_size(dtype);
   if (!es || !valid_n(nranks)) return COLL_ERR_INVALID_ARG;
   if (algo < COLL_ALGO_AUTO || algo > COLL_ALGO_RING_CTA) return COLL_ERR_UNSUPPORTED;
