@@ -110,6 +110,19 @@ FORM_NAMES = {1: "oneshot", 2: "twoshot", 4: "ring_ll", 5: "ring_cluster", 6: "r
               8: "ring_cta"}
 
 
+def tp_decode_cfg(n):
+    """The TP-decode workload's description, the same for both arms."""
+    return {"workload": "tp_decode_allreduce_8vr", "virtual_ranks": n, "dtype": "bf16",
+            "tokens": list(W.TP_DECODE_TOKENS), "hidden": list(W.TP_DECODE_HIDDEN),
+            "algos": ["oneshot", "twoshot", "ring"], "plus": "broadcast int32[256] src=7",
+            "values": "N(0,1) bf16 per rank, seeded"}
+
+
+def twoshot_160k_cfg(n):
+    return {"workload": "allreduce_twoshot_4vr_160KB", "virtual_ranks": n, "dtype": "bf16",
+            "values": "uniform[-1,1] bf16, seeded"}
+
+
 def build_tp_decode(M, oracle):
     import torch
     ops = []
@@ -143,10 +156,7 @@ def build_tp_decode(M, oracle):
                   {"bufs": [_dev(x, torch.int32) for x in ids]}, S * n, 1,
                   {"op": "broadcast", "src": 7, "ranks": n, "dtype": "int32", "count": 256, "bytes_per_rank": S},
                   inputs=["bufs"], outputs=["bufs"], ref=lambda ids=ids: oracle.broadcast(ids, 7), kernel="broadcast"))
-    cfg = {"workload": "tp_decode_allreduce_8vr", "virtual_ranks": n, "dtype": "bf16",
-           "tokens": list(W.TP_DECODE_TOKENS), "hidden": list(W.TP_DECODE_HIDDEN),
-           "algos": ["oneshot", "twoshot", "ring"], "plus": "broadcast int32[256] src=7",
-           "values": "N(0,1) bf16 per rank, seeded"}
+    cfg = tp_decode_cfg(n)
     return ops, cfg
 
 
@@ -161,8 +171,7 @@ def build_twoshot_160k(M, oracle):
               {"op": "all_reduce", "algo": "twoshot", "ranks": n, "bytes_per_rank": S},
               inputs=["send"], outputs=["recv"], ref=lambda: oracle.all_reduce_two_shot(xs, 0, "bf16"),
               kernel="all_reduce/twoshot")]
-    return ops, {"workload": "allreduce_twoshot_4vr_160KB", "virtual_ranks": n, "dtype": "bf16",
-                 "values": "uniform[-1,1] bf16, seeded"}
+    return ops, twoshot_160k_cfg(n)
 
 
 def build_sp_prefill(M, oracle):
@@ -977,14 +986,12 @@ def host_ops(workload: str, oracle):
                 ops.append((2 * n * S, lambda xs=xs, ref=ref: ref(xs, 0, "bf16")))
         ids = W.sampled_token_ids(n)
         ops.append((256 * 4 * n, lambda: oracle.broadcast(ids, 7)))
-        cfg = {"workload": "tp_decode_allreduce_8vr", "virtual_ranks": n, "dtype": "bf16",
-               "tokens": list(W.TP_DECODE_TOKENS), "hidden": list(W.TP_DECODE_HIDDEN),
-               "algos": ["oneshot", "twoshot", "ring"], "plus": "broadcast int32[256] src=7"}
+        cfg = tp_decode_cfg(n)
         return ops, cfg
     if workload == "twoshot_160k":
         xs = W.twoshot_160k(4)
         ops.append((2 * 4 * xs[0].size * 2, lambda: oracle.all_reduce_two_shot(xs, 0, "bf16")))
-        return ops, {"workload": "allreduce_twoshot_4vr_160KB", "virtual_ranks": 4}
+        return ops, twoshot_160k_cfg(4)
     raise SystemExit(f"--impl reference supports tp_decode and twoshot_160k, not {workload}")
 
 

@@ -34,7 +34,7 @@ def test_reference_arm_prints_one_contract_line():
     assert d["metric"] == bench.METRIC and d["unit"] == "GB/s" and d["higher_is_better"] is True
     assert d["steps"] == 2 and d["warmup"] == 1 and d["n_gpus"] == 1
     assert d["value"] > 0 and d["ms_per_step"] > 0
-    assert d["config"]["workload"] == "allreduce_twoshot_4vr_160KB"
+    assert d["config"] == bench.twoshot_160k_cfg(4)  # the GPU arm's workload description
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["unit"] == "GB/s" and cb["cores"] >= 1
     assert "sample" in cb
