@@ -128,6 +128,15 @@ def test_invalid_arguments_rejected_on_host():
     assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, M.RING, None, 0, None) == -5
     assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, M.RING, BASE + 0x50000000, 8, None) == -5
     assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, M.RING_STEPS, None, 0, None) == -5
+    # CTA ring: no one-launch form (9 ranks, or unaligned buffers) and no RING workspace for the
+    # stream-ordered fallback; a status workspace that is misaligned or inside a rank's buffer
+    p9, _k6 = _arr([BASE + i * 0x100000 for i in range(9)])
+    q9, _k7 = _arr([BASE + 0x10000000 + i * 0x100000 for i in range(9)])
+    pu, _k8 = _arr([BASE + 2 + i * 0x100000 for i in range(4)])
+    assert L.coll_all_reduce(p9, q9, 9, 16, M.BF16, M.SUM, M.RING_CTA, None, 0, None) == -2
+    assert L.coll_all_reduce(pu, q, 4, 16, M.BF16, M.SUM, M.RING_CTA, None, 0, None) == -2
+    assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, M.RING_CTA, BASE + 0x50000008, 64, None) == -5
+    assert L.coll_all_reduce(p, q, 4, 1 << 16, M.BF16, M.SUM, M.RING_CTA, BASE + 0x100, 64, None) == -3
     # fused LL two-shot: workspace missing, too small, or not 256-byte aligned
     need = L.coll_all_reduce_workspace_size(4, 16, M.BF16, M.TWOSHOT_LL)
     assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, M.TWOSHOT_LL, None, 0, None) == -5
