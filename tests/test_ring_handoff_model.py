@@ -1,0 +1,195 @@
+"""A model of the one-launch rings' hop hand-off, run under random schedules
+(CPU only).
+
+Both one-launch ring forms (RING_CTA: ranks are warps of one CTA; RING_CLUSTER:
+ranks are CTAs of a cluster) pass hop h from rank r to rank r+1 through slot
+h mod N of rank r+1, with one mbarrier per slot and no credit flowing back.
+They rely on three claims:
+
+* a sender never overwrites a slot before the receiving thread has read the
+  hop it held (the ring's own dependencies keep a sender within N-1 hops);
+* every wait sees the barrier at most one phase ahead of the phase it waits
+  for, so the parity test is exact (no stale read, no missed phase);
+* an arrival (or transaction count) always lands in the phase of its own hop.
+
+The model runs every thread (lane) of every rank as its own process, with the
+per-tile program both kernels share (send, then receive/send alternating,
+ending on a receive: 2N-2 of each per tile), and the two barrier mechanisms:
+
+* "arrive" (RING_CTA): barrier count = lanes; each sender lane arrives once
+  per hop;
+* "tx" (RING_CLUSTER): barrier count 1; the receiver's lane 0 arms the slot
+  (its arrival plus the expected bytes) for hops 0..N-1 at the start and for
+  hop h+N right after reading hop h; each sender lane's store completes its
+  bytes, possibly before the slot is armed.
+
+A random scheduler picks any enabled step; a receive is enabled when the
+hardware's parity test passes.  The checks are the three claims above, and
+that every schedule finishes (no deadlock).
+"""
+import random
+
+import pytest
+
+
+class Barrier:
+    def __init__(self, count, armed_tx=0):
+        self.count = count
+        self.pending = count
+        self.tx = 0
+        self.done = 0  # completed phases
+        if armed_tx:  # armed before anyone can store (initial expect_tx)
+            self.pending -= 1
+            self.tx += armed_tx
+
+    def _maybe_complete(self):
+        if self.pending == 0 and self.tx == 0:
+            self.done += 1
+            self.pending = self.count
+            self.tx = 0
+
+    def arrive(self, expect_tx=0):
+        assert self.pending > 0
+        self.pending -= 1
+        self.tx += expect_tx
+        self._maybe_complete()
+
+    def complete_tx(self, nbytes):
+        self.tx -= nbytes
+        self._maybe_complete()
+
+    def parity_passes(self, phase):
+        """try_wait.parity: true when the current phase's parity differs
+        from the awaited phase's parity"""
+        return (self.done & 1) != (phase & 1)
+
+
+def simulate(n, lanes, tiles, mode, seed):
+    rng = random.Random(seed)
+    H = tiles * (2 * n - 2)  # hops sent (and received) by every rank
+    program = []
+    for _ in range(tiles):
+        program += ["S"] + ["R", "S"] * (2 * n - 3) + ["R"]
+    assert program.count("S") == program.count("R") == H
+
+    if mode == "arrive":
+        bars = [[Barrier(lanes) for _ in range(n)] for _ in range(n)]  # [receiver][slot]
+    else:  # slots of hops that never come stay unarmed
+        bars = [[Barrier(1, armed_tx=lanes if j < H else 0) for j in range(n)] for _ in range(n)]
+    slot = [[[None] * lanes for _ in range(n)] for _ in range(n)]  # hop id held, [receiver][slot][lane]
+    read = [[[True] * lanes for _ in range(n)] for _ in range(n)]  # has the receiver lane read it
+    pc = {(r, t): 0 for r in range(n) for t in range(lanes)}
+    sent = {(r, t): 0 for r in range(n) for t in range(lanes)}
+    recv = {(r, t): 0 for r in range(n) for t in range(lanes)}
+
+    def enabled(p):
+        r, t = p
+        if pc[p] == len(program):
+            return False
+        if program[pc[p]] == "S":
+            return True
+        h = recv[p]
+        b = bars[r][h % n]
+        if not b.parity_passes(h // n):
+            return False
+        # the claim behind the parity test: the barrier is exactly one phase past the awaited one
+        assert b.done == h // n + 1, (mode, n, lanes, seed, "stale or missed phase", r, t, h, b.done)
+        return True
+
+    steps = 0
+    while True:
+        ready = [p for p in pc if enabled(p)]
+        if not ready:
+            assert all(pc[p] == len(program) for p in pc), (mode, n, lanes, tiles, seed, "deadlock")
+            break
+        p = rng.choice(ready)
+        r, t = p
+        steps += 1
+        if program[pc[p]] == "S":
+            h = sent[p]
+            q = (r + 1) % n
+            j = h % n
+            # the slot piece must be free: empty, or holding hop h - n already read by lane t of q
+            assert slot[q][j][t] is None or (slot[q][j][t] == h - n and read[q][j][t]), \
+                (mode, n, lanes, seed, "overwrite before read", r, t, h)
+            slot[q][j][t] = h
+            read[q][j][t] = False
+            b = bars[q][j]
+            # the arrival / bytes belong to the phase of this hop
+            assert b.done == h // n, (mode, n, lanes, seed, "landed in another phase", r, t, h, b.done)
+            if mode == "arrive":
+                b.arrive()
+            else:
+                b.complete_tx(1)
+            sent[p] += 1
+        else:
+            h = recv[p]
+            j = h % n
+            assert slot[r][j][t] == h and not read[r][j][t], (mode, n, lanes, seed, "stale data", r, t, h)
+            read[r][j][t] = True
+            if mode == "tx" and t == 0 and h + n < H:
+                b = bars[r][j]
+                assert b.done == (h + n) // n, (mode, n, lanes, seed, "armed in another phase", r, h, b.done)
+                b.arrive(expect_tx=lanes)
+            recv[p] += 1
+        pc[p] += 1
+    assert all(sent[p] == H and recv[p] == H for p in pc)
+    return steps
+
+
+@pytest.mark.parametrize("mode", ["arrive", "tx"])
+@pytest.mark.parametrize("n", [2, 3, 4, 5, 8])
+@pytest.mark.parametrize("lanes", [1, 2, 3])
+def test_handoff_protocol_under_random_schedules(mode, n, lanes):
+    for seed in range(40):
+        simulate(n, lanes, tiles=1 + seed % 3, mode=mode, seed=seed * 7919 + n * 31 + lanes)
+
+
+def test_model_catches_too_few_slots():
+    """The model is not vacuous: with N-1 slots per receiver (a sender may
+    then reach a slot whose previous hop is still unread) some schedule
+    breaks one of the claims."""
+    def simulate_fewer_slots(n, seed):
+        rng = random.Random(seed)
+        s = n - 1
+        H = 2 * (2 * n - 2)
+        program = (["S"] + ["R", "S"] * (2 * n - 3) + ["R"]) * 2
+        bars = [[Barrier(1) for _ in range(s)] for _ in range(n)]
+        slot = [[None] * s for _ in range(n)]
+        read = [[True] * s for _ in range(n)]
+        pc = [0] * n
+        sent = [0] * n
+        recv = [0] * n
+        while True:
+            ready = []
+            for r in range(n):
+                if pc[r] == len(program):
+                    continue
+                if program[pc[r]] == "S":
+                    ready.append(r)
+                else:
+                    h = recv[r]
+                    if bars[r][h % s].parity_passes(h // s):
+                        ready.append(r)
+            if not ready:
+                return all(pc[r] == len(program) for r in range(n))
+            r = rng.choice(ready)
+            if program[pc[r]] == "S":
+                h, q = sent[r], (r + 1) % n
+                if not (slot[q][h % s] is None or (slot[q][h % s] == h - s and read[q][h % s])):
+                    return False
+                if bars[q][h % s].done != h // s:
+                    return False
+                slot[q][h % s] = h
+                read[q][h % s] = False
+                bars[q][h % s].arrive()
+                sent[r] += 1
+            else:
+                h = recv[r]
+                if slot[r][h % s] != h:
+                    return False
+                read[r][h % s] = True
+                recv[r] += 1
+            pc[r] += 1
+
+    assert not all(simulate_fewer_slots(4, seed) for seed in range(200))
