@@ -179,6 +179,9 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    caller).  The workspace (coll_all_reduce_workspace_size() bytes,
  *    256-byte aligned) must be zero-filled once before its first use and
  *    serves one call at a time; the library keeps a call counter in it.
+ *    The counter occupies the flag's upper 25 bits: zero-fill the workspace
+ *    again before its 2^25-th call (the flags of a line left unwritten that
+ *    long would otherwise repeat).
  *    Buffers that are not 16-byte aligned take the RING_STEPS path.
  *  RING_CLUSTER: the RING schedule, chunk order and rounding (bit-identical
  *    result) in one launch of thread-block clusters of N CTAs, CTA r playing
@@ -209,7 +212,9 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    coll_all_reduce_workspace_size() bytes (256 + 4 N^2 seg size-of-dtype),
  *    256-byte aligned, zero-filled once before its first use, one call at a
  *    time; header as RING_LL (call counter, status pair at byte offset 16,
- *    COLL_DEV_TIMEOUT if a bounded poll ran out).  Buffers that are not
+ *    COLL_DEV_TIMEOUT if a bounded poll ran out).  The counter occupies the
+ *    flag's upper 30 bits: zero-fill the workspace again before its 2^30-th
+ *    call.  Buffers that are not
  *    16-byte aligned take the TWOSHOT kernel.  Needs N x (CTAs per SM) to
  *    fit on the GPU at once (COLL_ERR_UNSUPPORTED otherwise).
  *  AUTO picks TWOSHOT.  ONESHOT and TWOSHOT ignore `workspace`.
