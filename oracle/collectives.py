@@ -16,7 +16,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .numerics import ESIZE, SUM, combine, narrow, reduce_ranks, widen
+from .numerics import ESIZE, combine, narrow, reduce_ranks, widen
 
 
 def _copy(xs):

@@ -13,7 +13,7 @@ import torch
 import movement_virtual_rank_b200 as M
 import oracle
 import workloads as W
-from gpu_util import ESIZE, Guarded, from_dev, need_gpu, to_dev
+from gpu_util import Guarded, from_dev, need_gpu, to_dev
 
 pytestmark = pytest.mark.gpu
 

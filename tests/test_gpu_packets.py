@@ -13,7 +13,7 @@ import torch
 import movement_virtual_rank_b200 as M
 import oracle
 import workloads as W
-from gpu_util import from_dev, need_gpu, status_tensor, to_dev
+from gpu_util import need_gpu, status_tensor, to_dev
 
 pytestmark = pytest.mark.gpu
 SIZES = [1, 2, 3, 4, 5, 15, 16, 17, 31, 32, 33, 119, 120, 121, 239, 240, 241, 1000, 4097, 65536 + 12, 1 << 20]

@@ -10,7 +10,6 @@ import datetime
 import os
 import socket
 
-import pytest
 import torch.distributed as dist
 import torch.multiprocessing as mp
 

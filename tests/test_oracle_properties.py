@@ -20,7 +20,6 @@ the oracle's own arithmetic:
   bits as the per-(token, expert) route.
 """
 import numpy as np
-import pytest
 import torch
 from hypothesis import given, settings, strategies as st
 
