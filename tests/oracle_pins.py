@@ -49,6 +49,43 @@ def pin_bf16_rne_vs_torch():
     assert np.all(got[nan] == 0x7FC0)
 
 
+def pin_bf16_ulp_diff_brute_force():
+    """bf16_ulp_diff against a count of representable values: every finite
+    bf16 value, widened by torch to float64, sorted into one ladder (+0 and -0
+    are one rung); the distance of two values is how many rungs apart they
+    sit.  Random pairs, neighbours, sign flips, and the edges: the zeros, the
+    subnormals either side of zero, the largest finite values."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    vals = bf16_to_float(bits)
+    finite = np.isfinite(vals)
+    ladder = np.unique(vals[finite])
+    assert ladder.size == 2 * (0x7F80 - 1) + 1  # 0x0001..0x7F7F each side, and one zero
+
+    def rungs(a, b):
+        ia = np.searchsorted(ladder, bf16_to_float(a))
+        ib = np.searchsorted(ladder, bf16_to_float(b))
+        return np.abs(ia - ib)
+
+    fin = bits[finite]
+    g = np.random.default_rng(5)
+    a = g.choice(fin, 40000)
+    b = np.concatenate([g.choice(fin, 20000), a[20000:]])
+    near = a[20000:30000].astype(np.int32) + g.integers(-3, 4, 10000)
+    near = np.clip(near, 0, 0xFFFF).astype(np.uint16)
+    near = np.where(np.isfinite(bf16_to_float(near)), near, a[20000:30000])
+    b[20000:30000] = near
+    b[30000:] = a[30000:] ^ np.uint16(0x8000)  # the same magnitude, the other sign
+    edges = [(0x0000, 0x8000, 0), (0x0000, 0x0001, 1), (0x8000, 0x0001, 1), (0x8001, 0x0001, 2),
+             (0x8002, 0x0003, 5), (0x007F, 0x0080, 1), (0x3F7F, 0x3F80, 1), (0x7F7E, 0x7F7F, 1),
+             (0xFF7F, 0x7F7F, 2 * 0x7F7F), (0xBF80, 0x3F80, 2 * 0x3F80)]
+    ea = np.array([e[0] for e in edges], np.uint16)
+    eb = np.array([e[1] for e in edges], np.uint16)
+    assert np.array_equal(rungs(ea, eb), [e[2] for e in edges])  # the ladder itself, by hand
+    a, b = np.concatenate([a, ea]), np.concatenate([b, eb])
+    assert np.array_equal(oracle.bf16_ulp_diff(a, b), rungs(a, b))
+    assert np.array_equal(oracle.bf16_ulp_diff(b, a), rungs(a, b))
+
+
 def pin_bf16_hand_cases():
     one = 1.0
     cases = {

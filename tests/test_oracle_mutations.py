@@ -236,6 +236,18 @@ def m_segment_unaligned(mp):
     _patch(mp, "segment_elems", lambda count, n, dtype: -(-count // n) + 1)
 
 
+def m_ulp_diff_no_sign_fold(mp):
+    """the ulp distance compares magnitudes only (the sign bit dropped)"""
+    _patch(mp, "bf16_ulp_diff", lambda a, b: np.abs((np.asarray(a, np.uint16).astype(np.int32) & 0x7FFF)
+                                                    - (np.asarray(b, np.uint16).astype(np.int32) & 0x7FFF)))
+
+
+def m_ulp_diff_raw_bits(mp):
+    """the ulp distance subtracts the raw 16-bit patterns"""
+    _patch(mp, "bf16_ulp_diff", lambda a, b: np.abs(np.asarray(a, np.uint16).astype(np.int32)
+                                                    - np.asarray(b, np.uint16).astype(np.int32)))
+
+
 MUTANTS = [v for k, v in sorted(globals().items()) if k.startswith("m_")]
 
 
