@@ -23,18 +23,22 @@
  *   DEVICE pointers, one per virtual rank, read during the call only.  All
  *   device buffers belong to the caller and must stay alive until the work
  *   enqueued on `stream` has finished.  The library never allocates device
- *   memory; kernels that need scratch take a caller-provided `workspace`
- *   whose size the matching *_workspace_size() function returns.
+ *   memory at run time; kernels that need scratch take a caller-provided
+ *   `workspace` whose size the matching *_workspace_size() function returns.
+ *   The one exception is coll_all_reduce_ring_noalloc (near the end of this
+ *   file), whose scratch is a fixed array compiled into the library.
  * - Every call only ENQUEUES work on `stream` (NULL = legacy default
  *   stream) and never synchronises.  Calls are thread-safe; the library keeps
- *   no state besides a per-device cache of the SM count.
+ *   no state besides per-device caches (the SM count, kernel attributes set
+ *   once, and the address of the no-allocation entry point's array).
  * - Counts are in ELEMENTS of `dtype` unless stated otherwise; buffers are
  *   dense (contiguous).  N = nranks, 1 <= N <= COLL_MAX_RANKS.
  * - Return value: COLL_OK or a negative COLL_ERR_* code, decided on the host
  *   before anything is enqueued (argument errors) or right after the launch
  *   (COLL_ERR_CUDA).  coll_strerror() gives a message.
  * - Errors only the device can see (a packet flag that does not match, a
- *   row index beyond a receive buffer, a malformed route) are reported in an
+ *   row index beyond a receive buffer, a malformed route, a used-up LL call
+ *   counter) are reported in an
  *   optional device word pair `int d_status[2]`: d_status[0] receives the
  *   first COLL_DEV_* code raised (atomic compare-and-swap from 0) and
  *   d_status[1] is incremented by the number of offending items.  The caller
@@ -104,6 +108,13 @@ typedef enum { COLL_PROTO_SIMPLE = 0, COLL_PROTO_LL = 1, COLL_PROTO_LL128 = 2 } 
 #define COLL_DEV_TIMEOUT 2        /* reserved for bounded in-kernel waits              */
 #define COLL_DEV_SPLIT_OVERFLOW 3 /* a row index fell outside the receive buffer       */
 #define COLL_DEV_BAD_ROUTE 4      /* expert id out of range, or repeated within a token */
+#define COLL_DEV_EPOCH_WRAP 5     /* an LL workspace's call counter is used up: the call did
+                                     nothing; zero-fill the workspace before the next call */
+
+/* Calls one zero-filled workspace serves in RING_LL and TWOSHOT_LL (the call
+ * counter is the little-endian u32 at byte 0 of the workspace). */
+#define COLL_RING_LL_CALLS_PER_FILL (1u << 25)
+#define COLL_TWOSHOT_LL_CALLS_PER_FILL (1u << 30)
 
 /* ------------------------------------------------------------------------ */
 
@@ -179,9 +190,12 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    caller).  The workspace (coll_all_reduce_workspace_size() bytes,
  *    256-byte aligned) must be zero-filled once before its first use and
  *    serves one call at a time; the library keeps a call counter in it.
- *    The counter occupies the flag's upper 25 bits: zero-fill the workspace
- *    again before its 2^25-th call (the flags of a line left unwritten that
- *    long would otherwise repeat).
+ *    The counter occupies the flag's upper 25 bits, so one fill serves
+ *    COLL_RING_LL_CALLS_PER_FILL calls: a call made after those (its flags
+ *    would repeat those of the first call, and a line left unwritten that
+ *    long would pass for current) enqueues a kernel that does nothing but
+ *    raise COLL_DEV_EPOCH_WRAP in the status pair; zero-fill the workspace
+ *    again to go on.
  *    Buffers that are not 16-byte aligned take the RING_STEPS path.
  *  RING_CLUSTER: the RING schedule, chunk order and rounding (bit-identical
  *    result) in one launch of thread-block clusters of N CTAs, CTA r playing
@@ -196,12 +210,12 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    (COLL_DEV_TIMEOUT if a bounded wait ran out).
  *  RING_CTA: the RING schedule, chunk order and rounding (bit-identical
  *    result) in one launch in which every CTA holds all N virtual ranks,
- *    one group of 32 threads each: each hop is a store into shared memory
- *    of the same SM plus an mbarrier arrive, so the partials never leave
- *    the SM.  The CTAs (up to two per SM) walk the message tile by tile.
- *    Needs 2 <= N <= 8 and 16-byte aligned buffers, with the same fallback
- *    and the same optional `workspace` (status pair at bytes 16..23) as
- *    RING_CLUSTER.
+ *    one warp each: each hop is a store into a shared-memory slot of the
+ *    same SM and one CTA-wide barrier, so the partials never leave the SM
+ *    and nothing waits on another CTA.  The CTAs (up to three per SM) walk
+ *    the message tile by tile.  Needs 2 <= N <= 8 and 16-byte aligned
+ *    buffers, with the same fallback as RING_CLUSTER; `workspace` is
+ *    optional and unused (this form raises no device status).
  *  TWOSHOT_LL ([RLL] "Traditional LL Protocols" and the "Pro5000 ?" two-shot,
  *    fused): the TWOSHOT segments and arithmetic (bit-identical result) in
  *    ONE cooperative launch.  Every rank writes each 16-byte group of its
@@ -213,8 +227,9 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    256-byte aligned, zero-filled once before its first use, one call at a
  *    time; header as RING_LL (call counter, status pair at byte offset 16,
  *    COLL_DEV_TIMEOUT if a bounded poll ran out).  The counter occupies the
- *    flag's upper 30 bits: zero-fill the workspace again before its 2^30-th
- *    call.  Buffers that are not
+ *    flag's upper 30 bits: one fill serves COLL_TWOSHOT_LL_CALLS_PER_FILL
+ *    calls, and a later call only raises COLL_DEV_EPOCH_WRAP, as in RING_LL.
+ *    Buffers that are not
  *    16-byte aligned take the TWOSHOT kernel.  Needs N x (CTAs per SM) to
  *    fit on the GPU at once (COLL_ERR_UNSUPPORTED otherwise).
  *  AUTO picks TWOSHOT.  ONESHOT and TWOSHOT ignore `workspace`.
@@ -381,6 +396,13 @@ COLL_API int coll_moe_combine(const void* const* y, const int32_t* const* topk_i
  *    calls return COLL_ERR_WORKSPACE and enqueue nothing.
  *  - The first call on a device (with that device current) looks up the
  *    array's device address; make that first call before any stream capture.
+ *    Under lazy module loading (CUDA_MODULE_LOADING=LAZY, the default since
+ *    CUDA 12.2) that lookup is also when the driver places the array on the
+ *    device, so a process that reserves all of its device memory up front
+ *    should make one call first -- a call with count == 0 is enough, since
+ *    the lookup comes before every shortcut -- or run with
+ *    CUDA_MODULE_LOADING=EAGER, which places the array when the library's
+ *    kernels are loaded.
  *  - All calls share the one array, so calls whose work overlaps on the GPU
  *    (other streams, other threads) race: serialise them.  The array keeps
  *    the last call's partials; nothing in it needs to start at zero, because

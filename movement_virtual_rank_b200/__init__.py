@@ -24,7 +24,8 @@ BF16, FP16, FP32, INT32 = 0, 1, 2, 3
 SUM, MAX, MIN, PROD = 0, 1, 2, 3
 ALGO_AUTO, ONESHOT, TWOSHOT, RING, RING_LL, RING_CLUSTER, RING_STEPS, TWOSHOT_LL, RING_CTA = 0, 1, 2, 3, 4, 5, 6, 7, 8
 SIMPLE, LL, LL128 = 0, 1, 2
-DEV_OK, DEV_FLAG_MISMATCH, DEV_TIMEOUT, DEV_SPLIT_OVERFLOW, DEV_BAD_ROUTE = 0, 1, 2, 3, 4
+DEV_OK, DEV_FLAG_MISMATCH, DEV_TIMEOUT, DEV_SPLIT_OVERFLOW, DEV_BAD_ROUTE, DEV_EPOCH_WRAP = 0, 1, 2, 3, 4, 5
+RING_LL_CALLS_PER_FILL, TWOSHOT_LL_CALLS_PER_FILL = 1 << 25, 1 << 30  # calls one zero-filled workspace serves
 MAX_RANKS = 64
 
 _DTYPES = {torch.bfloat16: BF16, torch.float16: FP16, torch.float32: FP32, torch.int32: INT32}
@@ -256,8 +257,8 @@ def coll_all_reduce(send, recv, op="sum", algo=TWOSHOT, workspace: torch.Tensor 
     coll_all_reduce_workspace_size() bytes (zero-filled before its first
     RING_LL / TWOSHOT_LL use) and get a zeroed one allocated here when it
     is omitted;
-    RING_CLUSTER and RING_CTA use one, when given, for their status pair and
-    their fallback to RING_STEPS."""
+    RING_CLUSTER uses one, when given, for its status pair and its fallback
+    to RING_STEPS; RING_CTA only for that fallback."""
     algo = ALGOS[algo] if isinstance(algo, str) else int(algo)
     send = _ranks(send, "send", send[0].dtype)
     recv = _ranks(recv, "recv", send[0].dtype)
@@ -287,7 +288,9 @@ def coll_all_reduce_ring_noalloc(send, recv, op="sum", stream=None):
     callers that may not allocate device memory: its partial sums live in a
     fixed 8 MiB array inside the library (at most RING_NOALLOC_MAX_COUNT
     elements per rank).  Same result as coll_all_reduce(..., algo=RING).
-    Calls that overlap on the GPU share that array and race."""
+    Calls that overlap on the GPU share that array and race.  The first call
+    on a device looks up the array (and, under lazy module loading, is when
+    the driver places it): a call with empty tensors is a warm-up."""
     send = _ranks(send, "send", send[0].dtype)
     recv = _ranks(recv, "recv", send[0].dtype)
     if len(send) != len(recv):

@@ -18,7 +18,8 @@
 // may still be read, and no back-pressure is needed.  A line's flag is
 // (epoch << 7) | (slot + 1), where the epoch is a per-workspace call counter
 // kept in the workspace header (advanced by the last CTA to finish), so lines
-// left by an earlier call never match.
+// left by an earlier call never match.  The epoch has 25 bits: a call that
+// finds the counter at 2^25 does nothing and raises COLL_DEV_EPOCH_WRAP.
 //
 // All CTAs are co-resident (cooperative launch).  Every poll is bounded: after
 // the budget a CTA raises COLL_DEV_TIMEOUT, sets the header's abort word (so
@@ -84,6 +85,14 @@ __global__ void __launch_bounds__(kRingLLThreads) k_ring_ll(const __grid_constan
   const int g = blockIdx.x / n;
   const int slots = 2 * n - 2;
   const uint32_t epoch = ld_volatile32(a.hdr);
+  // every CTA reads the same counter (only the last CTA of a call advances
+  // it, after all have read it), so all take this exit together: past the
+  // last epoch the flags would repeat those of epoch 0, and a line no call
+  // has rewritten since could pass for a current one
+  if (epoch >= COLL_RING_LL_CALLS_PER_FILL) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) report(a.status, COLL_DEV_EPOCH_WRAP, 1);
+    return;
+  }
   const int rs = (r + 1) % n;  // receiver of my sends
   bool alive = true;
 

@@ -18,7 +18,8 @@
 //
 // A line's flag is (epoch << 2) | phase, where the epoch is a call counter
 // in the workspace header advanced by the last CTA to finish, so lines left
-// by an earlier call never match.  Every poll is bounded: after the budget a
+// by an earlier call never match.  The epoch has 30 bits: a call that finds
+// the counter at 2^30 does nothing and raises COLL_DEV_EPOCH_WRAP.  Every poll is bounded: after the budget a
 // thread raises COLL_DEV_TIMEOUT and sets the header's abort word, which
 // stops the other polls.
 #include <algorithm>
@@ -71,6 +72,13 @@ __global__ void __launch_bounds__(kTsllThreads) k_twoshot_ll(const __grid_consta
   const int r = blockIdx.x % n;
   const int g = blockIdx.x / n;
   const uint32_t epoch = tsll_ld32(a.hdr);
+  // all CTAs read the same counter (the last CTA of a call advances it after
+  // every CTA has read it) and leave together: past the last epoch the flags
+  // would repeat those of epoch 0
+  if (epoch >= COLL_TWOSHOT_LL_CALLS_PER_FILL) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) report(a.status, COLL_DEV_EPOCH_WRAP, 1);
+    return;
+  }
   const uint32_t flag_rs = (epoch << 2) | 1u, flag_ag = (epoch << 2) | 2u;
   const uint64_t units_per_seg = a.seg * ES / 8;  // 16-byte units (8 payload bytes each) per segment
   const uint64_t first = static_cast<uint64_t>(g) * blockDim.x + threadIdx.x;

@@ -42,6 +42,29 @@ def test_exports_match_nm():
     assert {e for e in exported if e.startswith("coll_")} == set(declared())
 
 
+def _header_value(name: str) -> int:
+    """The value of a #define in coll.h (integer expressions of literals, shifts
+    and other defines)."""
+    txt = open(HEADER).read()
+    m = re.search(rf"^#define\s+{name}\s+(.+?)(?:/\*.*)?$", txt, flags=re.M)
+    assert m, name
+    expr = re.sub(r"\b(COLL_\w+)\b", lambda k: str(_header_value(k.group(1))), m.group(1))
+    expr = re.sub(r"(\d+)u\b", r"\1", expr)
+    return int(eval(expr, {"__builtins__": {}}))  # digits, parentheses, shifts and divisions only
+
+
+def test_binding_constants_match_header():
+    """The Python binding's copies of the header's numbers are the header's."""
+    assert M.RING_NOALLOC_MAX_COUNT == _header_value("COLL_RING_NOALLOC_MAX_COUNT")
+    assert M.RING_LL_CALLS_PER_FILL == _header_value("COLL_RING_LL_CALLS_PER_FILL")
+    assert M.TWOSHOT_LL_CALLS_PER_FILL == _header_value("COLL_TWOSHOT_LL_CALLS_PER_FILL")
+    assert M.MAX_RANKS == _header_value("COLL_MAX_RANKS")
+    for py, c in (("DEV_OK", "COLL_DEV_OK"), ("DEV_FLAG_MISMATCH", "COLL_DEV_FLAG_MISMATCH"),
+                  ("DEV_TIMEOUT", "COLL_DEV_TIMEOUT"), ("DEV_SPLIT_OVERFLOW", "COLL_DEV_SPLIT_OVERFLOW"),
+                  ("DEV_BAD_ROUTE", "COLL_DEV_BAD_ROUTE"), ("DEV_EPOCH_WRAP", "COLL_DEV_EPOCH_WRAP")):
+        assert getattr(M, py) == _header_value(c), py
+
+
 def test_version_and_strerror():
     assert M.coll_version() == 10000
     for code in (0, -1, -2, -3, -4, -5):

@@ -1,10 +1,9 @@
-"""A model of the one-launch rings' hop hand-off, run under random schedules
+"""Models of the one-launch rings' hop hand-offs, run under random schedules
 (CPU only).
 
-Both one-launch ring forms (RING_CTA: ranks are warps of one CTA; RING_CLUSTER:
-ranks are CTAs of a cluster) pass hop h from rank r to rank r+1 through slot
-h mod N of rank r+1, with one mbarrier per slot and no credit flowing back.
-They rely on three claims:
+RING_CLUSTER (ranks are CTAs of a cluster) passes hop h from rank r to rank
+r+1 through slot h mod N of rank r+1, with one mbarrier per slot and no credit
+flowing back.  It relies on three claims:
 
 * a sender never overwrites a slot before the receiving thread has read the
   hop it held (the ring's own dependencies keep a sender within N-1 hops);
@@ -12,20 +11,28 @@ They rely on three claims:
   for, so the parity test is exact (no stale read, no missed phase);
 * an arrival (or transaction count) always lands in the phase of its own hop.
 
-The model runs every thread (lane) of every rank as its own process, with the
-per-tile program both kernels share (send, then receive/send alternating,
-ending on a receive: 2N-2 of each per tile), and the two barrier mechanisms:
+That model runs every thread (lane) of every rank as its own process, with
+the per-tile program of the kernel (send, then receive/send alternating,
+ending on a receive: 2N-2 of each per tile), and two barrier mechanisms:
 
-* "arrive" (RING_CTA): barrier count = lanes; each sender lane arrives once
-  per hop;
 * "tx" (RING_CLUSTER): barrier count 1; the receiver's lane 0 arms the slot
   (its arrival plus the expected bytes) for hops 0..N-1 at the start and for
   hop h+N right after reading hop h; each sender lane's store completes its
-  bytes, possibly before the slot is armed.
+  bytes, possibly before the slot is armed;
+* "arrive": barrier count = lanes; each sender lane arrives once per hop
+  (the hand-off an earlier form of the CTA ring used; kept as a second
+  mechanism the protocol argument covers).
+
+RING_CTA (ranks are warps of one CTA) uses no mbarrier: at hop h every warp
+stores into the next warp's slot of buffer h mod 2, the CTA passes one
+barrier, and every warp reads its own slot.  Its model lets the warps run
+freely between barriers and checks that every read sees its own hop and that
+no store lands on a hop not yet read; with one buffer instead of two, some
+schedule breaks that.
 
 A random scheduler picks any enabled step; a receive is enabled when the
-hardware's parity test passes.  The checks are the three claims above, and
-that every schedule finishes (no deadlock).
+hardware's test passes.  The checks are the claims above, and that every
+schedule finishes (no deadlock).
 """
 import random
 
@@ -193,3 +200,55 @@ def test_model_catches_too_few_slots():
             pc[r] += 1
 
     assert not all(simulate_fewer_slots(4, seed) for seed in range(200))
+
+
+def simulate_lockstep(n, tiles, buffers, seed):
+    """RING_CTA's hand-off: per hop, store into the next warp's slot of buffer
+    h mod ``buffers``, one CTA-wide barrier, read the own slot.  Returns
+    False at the first violation (overwrite of an unread hop, or a read of
+    the wrong hop); True when every schedule step was clean."""
+    rng = random.Random(seed)
+    H = tiles * (2 * n - 2)
+    program = ["S", "B", "R"] * H
+    slot = [[None] * n for _ in range(buffers)]  # hop held, [buffer][receiving warp]
+    read = [[True] * n for _ in range(buffers)]
+    pc = [0] * n
+    while True:
+        ready = []
+        for w in range(n):
+            if pc[w] == len(program):
+                continue
+            if program[pc[w]] == "B":
+                # every warp must have arrived at this barrier (the same index in every program)
+                if all(pc[v] >= pc[w] for v in range(n)):
+                    ready.append(w)
+            else:
+                ready.append(w)
+        if not ready:
+            assert all(pc[w] == len(program) for w in range(n)), ("deadlock", n, seed)
+            return True
+        w = rng.choice(ready)
+        h = pc[w] // 3
+        op = program[pc[w]]
+        b = h % buffers
+        if op == "S":
+            q = (w + 1) % n
+            if not (slot[b][q] is None or (slot[b][q] == h - buffers and read[b][q])):
+                return False
+            slot[b][q] = h
+            read[b][q] = False
+        elif op == "R":
+            if slot[b][w] != h or read[b][w]:
+                return False
+            read[b][w] = True
+        pc[w] += 1
+
+
+@pytest.mark.parametrize("n", [2, 3, 4, 5, 8])
+def test_cta_ring_double_buffer_under_random_schedules(n):
+    for seed in range(200):
+        assert simulate_lockstep(n, tiles=1 + seed % 3, buffers=2, seed=seed * 131 + n)
+
+
+def test_cta_ring_model_catches_a_single_buffer():
+    assert not all(simulate_lockstep(4, tiles=2, buffers=1, seed=seed) for seed in range(200))
