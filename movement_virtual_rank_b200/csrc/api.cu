@@ -86,6 +86,37 @@ int launch_ring_rs_step(const RingStepArgs& a, coll_dtype_t dt, coll_op_t op, bo
   return COLL_ERR_UNSUPPORTED;
 }
 
+int launch_ring_steps(const char* const* in, char* const* out, int n, size_t count, coll_dtype_t dt, coll_op_t op,
+                      char* partial, bool vec, cudaStream_t s) {
+  const int es = elem_size(dt);
+  const size_t g = 16 / es;
+  const size_t seg = ((count + n - 1) / n + g - 1) / g * g;
+  RingStepArgs a{};
+  for (int r = 0; r < n; ++r) {
+    a.in[r] = in[r];
+    a.out[r] = out[r];
+  }
+  a.partial = partial;
+  a.count = count;
+  a.seg = seg;
+  a.n = n;
+  for (int k = 1; k < n; ++k) {  // reduce-scatter phase
+    a.k = k;
+    const int st = launch_ring_rs_step(a, dt, op, vec, s);
+    if (st != COLL_OK) return st;
+  }
+  std::vector<CopyJob> jobs(n);
+  for (int j = 1; j < n; ++j) {  // all-gather phase: rank c+j copies chunk c from rank c+j-1
+    for (int c = 0; c < n; ++c) {
+      const size_t lo = std::min(count, c * seg), hi = std::min(count, lo + seg);
+      jobs[c] = {out[(c + j - 1) % n] + lo * es, out[(c + j) % n] + lo * es, (hi - lo) * es};
+    }
+    const int st = launch_copy_jobs(jobs.data(), n, s);
+    if (st != COLL_OK) return st;
+  }
+  return COLL_OK;
+}
+
 }  // namespace mvr
 
 using namespace mvr;
@@ -413,32 +444,14 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
     algo = COLL_ALGO_TWOSHOT;  // unaligned buffers: the plain two-shot kernel, the same result
   }
   if (algo == COLL_ALGO_RING_STEPS) {
-    RingStepArgs a{};
+    const char* in[COLL_MAX_RANKS];
+    char* out[COLL_MAX_RANKS];
     for (int r = 0; r < nranks; ++r) {
-      a.in[r] = static_cast<const char*>(send[r]);
-      a.out[r] = static_cast<char*>(recv[r]);
+      in[r] = static_cast<const char*>(send[r]);
+      out[r] = static_cast<char*>(recv[r]);
     }
-    a.partial = static_cast<char*>(workspace) + 256;  // after the header
-    a.count = count;
-    a.seg = seg;
-    a.n = nranks;
-    for (int k = 1; k < nranks; ++k) {  // reduce-scatter phase
-      a.k = k;
-      const int st = launch_ring_rs_step(a, dtype, op, vec, S(stream));
-      if (st != COLL_OK) return st;
-    }
-    std::vector<CopyJob> jobs(nranks);
-    for (int j = 1; j < nranks; ++j) {  // all-gather phase: rank c+j copies chunk c from rank c+j-1
-      int nj = 0;
-      for (int c = 0; c < nranks; ++c) {
-        const size_t lo = std::min(count, c * seg), hi = std::min(count, lo + seg);
-        jobs[nj++] = {static_cast<const char*>(recv[(c + j - 1) % nranks]) + lo * es,
-                      static_cast<char*>(recv[(c + j) % nranks]) + lo * es, (hi - lo) * es};
-      }
-      const int st = launch_copy_jobs(jobs.data(), nj, S(stream));
-      if (st != COLL_OK) return st;
-    }
-    return COLL_OK;
+    // partials after the 256-byte header
+    return launch_ring_steps(in, out, nranks, count, dtype, op, static_cast<char*>(workspace) + 256, vec, S(stream));
   }
   ReduceArgs a{};
   for (int r = 0; r < nranks; ++r) {

@@ -45,6 +45,12 @@ struct RingStepArgs {
 };
 int launch_ring_rs_step(const RingStepArgs& a, coll_dtype_t dt, coll_op_t op, bool vec,
                         cudaStream_t s);
+// The whole stream-ordered ring (RING_STEPS): N-1 reduce-scatter step
+// launches whose partials live at `partial` (count elements of the
+// arithmetic type), then N-1 all-gather copy launches.  Shared by
+// coll_all_reduce and coll_all_reduce_ring_noalloc, so both give the same bits.
+int launch_ring_steps(const char* const* in, char* const* out, int n, size_t count, coll_dtype_t dt, coll_op_t op,
+                      char* partial, bool vec, cudaStream_t s);
 
 size_t twoshot_ll_workspace(int n, size_t count, int es);
 int launch_twoshot_ll(const char* const* in, char* const* out, int n, size_t count, coll_dtype_t dt, coll_op_t op,

@@ -14,10 +14,12 @@
 // Host code cannot use g_ring_scratch's name as an address (on the host it
 // names a stand-in object, not device memory), so the first call on each
 // device, with that device current, looks up the array's device address with
-// cudaGetSymbolAddress and caches it.
+// cudaGetSymbolAddress and caches it.  Under lazy module loading (the CUDA
+// default) that lookup is also when the driver places the array on the
+// device, so it is done before any shortcut: a call with count == 0 is the
+// warm-up a caller makes before reserving the rest of the device's memory.
 #include <atomic>
 #include <mutex>
-#include <vector>
 
 #include "coll.h"
 #include "common.cuh"
@@ -70,6 +72,14 @@ extern "C" int coll_all_reduce_ring_noalloc(const void* const* send, void* const
   if (nranks < 1 || nranks > COLL_MAX_RANKS || send == nullptr || recv == nullptr) return COLL_ERR_INVALID_ARG;
   for (int r = 0; r < nranks; ++r)
     if (send[r] == nullptr || recv[r] == nullptr) return COLL_ERR_INVALID_ARG;
+  // The address comes first, before the count == 0 and N == 1 shortcuts: the
+  // first call on a device is where the driver places the array (under lazy
+  // module loading, the default, that is when this file's module is loaded),
+  // so a call with count == 0 serves as a warm-up that a caller can make
+  // before it reserves the rest of the device's memory.
+  void* scratch = nullptr;
+  const int st0 = scratch_for_current_device(&scratch);
+  if (st0 != COLL_OK) return st0;
   const size_t bytes = count * es;
   if (bytes == 0) return COLL_OK;
   if (count > COLL_RING_NOALLOC_MAX_COUNT) return COLL_ERR_WORKSPACE;  // beyond the fixed scratch
@@ -84,38 +94,15 @@ extern "C" int coll_all_reduce_ring_noalloc(const void* const* send, void* const
     CopyJob j{static_cast<const char*>(send[0]), static_cast<char*>(recv[0]), bytes};
     return launch_copy_jobs(&j, 1, s);
   }
-  void* scratch = nullptr;
-  const int st0 = scratch_for_current_device(&scratch);
-  if (st0 != COLL_OK) return st0;
-
   bool vec = true;
-  for (int r = 0; r < nranks; ++r)
-    vec = vec && (reinterpret_cast<uintptr_t>(send[r]) & 15) == 0 && (reinterpret_cast<uintptr_t>(recv[r]) & 15) == 0;
-  const size_t g = 16 / es;
-  const size_t seg = ((count + nranks - 1) / nranks + g - 1) / g * g;
-  RingStepArgs a{};
+  const char* in[COLL_MAX_RANKS];
+  char* out[COLL_MAX_RANKS];
   for (int r = 0; r < nranks; ++r) {
-    a.in[r] = static_cast<const char*>(send[r]);
-    a.out[r] = static_cast<char*>(recv[r]);
+    in[r] = static_cast<const char*>(send[r]);
+    out[r] = static_cast<char*>(recv[r]);
+    vec = vec && (reinterpret_cast<uintptr_t>(send[r]) & 15) == 0 && (reinterpret_cast<uintptr_t>(recv[r]) & 15) == 0;
   }
-  a.partial = static_cast<char*>(scratch);  // every partial is written before it is read: no clearing needed
-  a.count = count;
-  a.seg = seg;
-  a.n = nranks;
-  for (int k = 1; k < nranks; ++k) {
-    a.k = k;
-    const int st = launch_ring_rs_step(a, dtype, op, vec, s);
-    if (st != COLL_OK) return st;
-  }
-  std::vector<CopyJob> jobs(nranks);
-  for (int j = 1; j < nranks; ++j) {
-    for (int c = 0; c < nranks; ++c) {
-      const size_t lo = std::min(count, c * seg), hi = std::min(count, lo + seg);
-      jobs[c] = {static_cast<const char*>(recv[(c + j - 1) % nranks]) + lo * es,
-                 static_cast<char*>(recv[(c + j) % nranks]) + lo * es, (hi - lo) * es};
-    }
-    const int st = launch_copy_jobs(jobs.data(), nranks, s);
-    if (st != COLL_OK) return st;
-  }
-  return COLL_OK;
+  // the same launches as coll_all_reduce(RING_STEPS); every partial is
+  // written before it is read, so the array needs no clearing
+  return launch_ring_steps(in, out, nranks, count, dtype, op, static_cast<char*>(scratch), vec, s);
 }
