@@ -1,13 +1,27 @@
 """Benchmark of the virtual-rank collectives on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload tp_decode|twoshot_160k|sp_prefill|moe|ll_sweep|
-                               single_image|ring_compare|movement]
+                    [--workload full_step|tp_decode|twoshot_160k|sp_prefill|moe|
+                               ll_sweep|single_image|ring_compare|movement]
 
 One "step" is one call of every op of the chosen workload on seeded synthetic
 inputs resident in HBM.  ``value`` is the ops' algorithmic bytes (what each
 collective must read plus write, once) over the step's device time, summed
 over all GPUs, in GB/s.
+
+Default workload (``full_step``): every op of the hot path, 8 virtual ranks,
+at the largest sizes the workloads give:
+  * sequence-parallel prefill: all_gather bf16 [1024,8192] -> [8192,8192],
+    reduce_scatter [8192,8192] -> [1024,8192], gather of fp32 [256,16032]
+    logits shards to rank 0;
+  * MoE: route, dispatch and combine of 4096 tokens per rank, hidden 7168
+    bf16, 256 experts, top-8 Zipf-skewed routing;
+  * all_reduce of bf16 uniform[-1,1] messages of 16 MiB and 256 MiB per rank:
+    the Simple two-shot, and the LL and LL128 paths (encode every rank,
+    packetised all-reduce, decode every rank);
+  * the TP-decode all_reduce of bf16 [256,7168] by one-shot, two-shot and
+    ring, and the broadcast of int32 sampled_token_ids[256] from rank 7;
+  * reduce to rank 0 and scatter from rank 0, 16 MiB per rank.
 
 How an op's device time is measured.  The op is replicated on R distinct
 copies of its buffers (R = 1 for ops larger than L2, up to 256 for the
@@ -22,17 +36,15 @@ timed alone between two events (``us_single``, which includes the ~2.5 us cost
 of an event pair) and, for messages up to 256 KB per rank, the warm-L2
 latency floor of back-to-back calls (``graph_us``).
 
-Default workload (``tp_decode``): 8 virtual ranks, the TP-decode all-reduce
-after RowParallelLinear (bf16 [tokens, hidden], tokens 1..256, hidden
-4096/7168, N(0,1)) by one-shot, two-shot and ring, plus the broadcast of
-int32 sampled_token_ids[256] from rank 7.
-
 With --gpus N > 1 (torchrun, one process per GPU) every GPU runs its own
 independent replica: the virtual ranks live inside one GPU, so there is no
 exchange between GPUs (weak scaling; timing is the max over ranks).
 
 ``--impl reference`` times the CPU oracle (the plain definition of each op)
-on this host's cores on the same workload.
+on this host's cores on a bounded sample of the same workload: every op at
+1/16 of its size (the first part of each rank's own seeded input, MoE the
+first 1/16 of each rank's tokens), each op split into independent parts that
+worker processes (one per core) run in parallel.
 """
 from __future__ import annotations
 
@@ -44,6 +56,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -65,7 +78,8 @@ class Op:
     bind(bufs) -> callable that launches the op on those device buffers
     bufs:       dict of name -> tensor or list of tensors (device)
     inputs / outputs: names in ``bufs`` copied host->device / device->host by
-                the end-to-end leg
+                the end-to-end leg (empty for the inner ops of a chain, whose
+                inputs are the previous op's device outputs)
     ref():      the oracle's version of the op on the host inputs
     """
 
@@ -121,6 +135,27 @@ def tp_decode_cfg(n):
 def twoshot_160k_cfg(n):
     return {"workload": "allreduce_twoshot_4vr_160KB", "virtual_ranks": n, "dtype": "bf16",
             "values": "uniform[-1,1] bf16, seeded"}
+
+
+FULL_STEP_AR_BYTES = (16 << 20, 256 << 20)  # all-reduce bytes per rank: the >= 16 MiB end of the LL sweep
+FULL_STEP_MOVE_BYTES = 16 << 20             # reduce / scatter bytes per rank
+
+
+def full_step_cfg(n=8):
+    """The default workload's description, the same for both arms."""
+    return {"workload": "all_hot_path_ops_largest_configs_8vr", "virtual_ranks": n,
+            "sp_prefill": {"all_gather": "bf16 [1024,8192] -> [8192,8192]",
+                           "reduce_scatter": "bf16 [8192,8192] -> [1024,8192]",
+                           "gather": "fp32 [256,16032] -> dst 0 [256,128256]"},
+            "moe": {"tokens": 4096, "hidden": 7168, "experts": 256, "topk": 8,
+                    "routing": "softmax(N(0,1)+log Zipf(1.1)) top-8, renormalised",
+                    "ops": ["route", "dispatch", "combine"]},
+            "all_reduce": {"bytes_per_rank": list(FULL_STEP_AR_BYTES), "values": "uniform[-1,1] bf16",
+                           "paths": ["simple two-shot", "LL: pack, packetised all-reduce, unpack",
+                                     "LL128: pack, packetised all-reduce, unpack"]},
+            "tp_decode": {"shape": [256, 7168], "algos": ["oneshot", "twoshot", "ring"],
+                          "plus": "broadcast int32[256] src=7"},
+            "movement": {"bytes_per_rank": FULL_STEP_MOVE_BYTES, "ops": ["reduce to rank 0", "scatter from rank 0"]}}
 
 
 def build_tp_decode(M, oracle):
@@ -208,13 +243,20 @@ def build_sp_prefill(M, oracle):
 MOE_TOKENS = 4096  # tokens per rank of the MoE workload (and of the all-to-all-v split matrix); --moe-tokens
 
 
-def build_moe(M, oracle):
+def moe_ops(M, oracle, dedup: bool = True, chain: bool = False):
+    """The MoE workload's ops (8 virtual ranks x MOE_TOKENS tokens, hidden
+    7168 bf16, 256 experts, top-8): route, dispatch and combine, plus, with
+    ``dedup``, the same three on the route deduplicated per (token,
+    destination rank).  ``chain``: the end-to-end leg uploads only what a
+    caller holds on the host (expert ids, token rows, weights) and downloads
+    only the combined tokens."""
     import torch
     n, tokens, topk, experts, hidden = 8, MOE_TOKENS, 8, 256, 7168
     ids, ws = W.moe_routing(tokens, experts, topk, n)
     xs = W.moe_tokens(tokens, hidden, n)
     dids = [torch.from_numpy(i).cuda() for i in ids]
     x = [_dev(v, torch.bfloat16) for v in xs]
+    del xs
     split = {"sc": torch.empty(n * n, dtype=torch.int64, device="cuda")}
     split["sd"], split["rd"] = torch.empty_like(split["sc"]), torch.empty_like(split["sc"])
     pos = [torch.empty(tokens * topk, dtype=torch.int32, device="cuda") for _ in range(n)]
@@ -223,26 +265,38 @@ def build_moe(M, oracle):
     torch.cuda.synchronize()
     cap = int(split["sc"].view(n, n).sum(0).max().item())
     recv = [torch.empty(cap * hidden, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+    dw = [torch.from_numpy(w).cuda() for w in ws]
     row = hidden * 2
     pairs = n * tokens * topk
-    ops = [
-        Op("moe_route",
-           lambda b: (lambda: M.coll_moe_route(b["ids"], experts, b["sc"], b["sd"], b["rd"], b["pos"],
-                                               workspace=b["ws"])),
-           {"ids": dids, "pos": pos, "ws": wsp, **split}, pairs * 4 * 2, 3,
-           {"op": "moe_route", "ranks": n, "tokens": tokens, "topk": topk, "experts": experts},
-           inputs=["ids"], outputs=["pos"], ref=lambda: oracle.moe_route(ids, experts), kernel="moe_route"),
-        Op("moe_dispatch", lambda b: (lambda: M.coll_moe_dispatch(b["x"], b["ids"], b["pos"], b["recv"], experts)),
-           {"x": x, "ids": dids, "pos": pos, "recv": recv}, n * tokens * row + pairs * row, 1,
-           {"op": "moe_dispatch", "ranks": n, "hidden": hidden, "rows_out": pairs},
-           inputs=["x"], outputs=["recv"], kernel="moe_dispatch"),
-        Op("moe_combine",
-           lambda b: (lambda: M.coll_moe_combine(b["y"], b["ids"], b["pos"], b["w"], b["out"], experts)),
-           {"y": recv, "ids": dids, "pos": pos, "w": [torch.from_numpy(w).cuda() for w in ws],
-            "out": [torch.empty_like(t) for t in x]}, pairs * row + pairs * 4 + n * tokens * row, 1,
-           {"op": "moe_combine", "ranks": n, "hidden": hidden},
-           inputs=["y"], outputs=["out"], kernel="moe_combine"),
-    ]
+
+    def io_of(inp, out):
+        if not chain:
+            return [inp], [out]
+        return ([inp] if inp else []), ([out] if out else [])
+
+    ops = []
+    i, o = io_of("ids", None if chain else "pos")
+    ops.append(Op("moe_route",
+                  lambda b: (lambda: M.coll_moe_route(b["ids"], experts, b["sc"], b["sd"], b["rd"], b["pos"],
+                                                      workspace=b["ws"])),
+                  {"ids": dids, "pos": pos, "ws": wsp, **split}, pairs * 4 * 2, 3,
+                  {"op": "moe_route", "ranks": n, "tokens": tokens, "topk": topk, "experts": experts},
+                  inputs=i, outputs=o, ref=lambda: oracle.moe_route(ids, experts), kernel="moe_route"))
+    i, o = io_of("x", None if chain else "recv")
+    ops.append(Op("moe_dispatch", lambda b: (lambda: M.coll_moe_dispatch(b["x"], b["ids"], b["pos"], b["recv"],
+                                                                         experts)),
+                  {"x": x, "ids": dids, "pos": pos, "recv": recv}, n * tokens * row + pairs * row, 1,
+                  {"op": "moe_dispatch", "ranks": n, "hidden": hidden, "rows_out": pairs},
+                  inputs=i, outputs=o, kernel="moe_dispatch"))
+    i, o = io_of("w" if chain else "y", "out")
+    ops.append(Op("moe_combine",
+                  lambda b: (lambda: M.coll_moe_combine(b["y"], b["ids"], b["pos"], b["w"], b["out"], experts)),
+                  {"y": recv, "ids": dids, "pos": pos, "w": dw,
+                   "out": [torch.empty_like(t) for t in x]}, pairs * row + pairs * 4 + n * tokens * row, 1,
+                  {"op": "moe_combine", "ranks": n, "hidden": hidden},
+                  inputs=i, outputs=o, kernel="moe_combine"))
+    if not dedup:
+        return ops
     # the route deduplicated per (token, destination rank): one row per pair reached
     dsplit = {k: torch.empty_like(v) for k, v in split.items()}
     dpos = [torch.empty_like(p) for p in pos]
@@ -265,13 +319,18 @@ def build_moe(M, oracle):
            inputs=["x"], outputs=["recv"], kernel="moe_dispatch_dedup"),
         Op("moe_combine_dedup",
            lambda b: (lambda: M.coll_moe_combine(b["y"], b["ids"], b["pos"], b["w"], b["out"], experts)),
-           {"y": drecv, "ids": dids, "pos": dpos, "w": [torch.from_numpy(w).cuda() for w in ws],
+           {"y": drecv, "ids": dids, "pos": dpos, "w": dw,
             "out": [torch.empty_like(t) for t in x]}, uniq * row + pairs * 4 + n * tokens * row, 1,
            {"op": "moe_combine_dedup", "ranks": n, "hidden": hidden, "rows_in": uniq},
            inputs=["y"], outputs=["out"], kernel="moe_combine_dedup"),
     ]
-    return ops, {"workload": "moe_dispatch_combine_8vr", "virtual_ranks": n, "tokens": tokens, "hidden": hidden,
-                 "experts": experts, "topk": topk, "routing": "softmax(N(0,1)+log Zipf(1.1)) top-8, renormalised"}
+    return ops
+
+
+def build_moe(M, oracle):
+    return moe_ops(M, oracle, dedup=True), {
+        "workload": "moe_dispatch_combine_8vr", "virtual_ranks": 8, "tokens": MOE_TOKENS, "hidden": 7168,
+        "experts": 256, "topk": 8, "routing": "softmax(N(0,1)+log Zipf(1.1)) top-8, renormalised"}
 
 
 LL_SIZES = None  # bytes per rank of the LL sweep (default 1 KB .. 256 MB, powers of 4); --ll-sizes
@@ -456,7 +515,110 @@ def build_single_image(M, oracle):
                  "n_tok": [256, 1024, 4096], "paths": ["padded all_gather (old)", "broadcast (new)"]}
 
 
+def _protocol_ops(M, nbytes, n=8):
+    """All-reduce of a bf16 uniform[-1,1] message of ``nbytes`` per rank by
+    the Simple two-shot and by the LL and LL128 paths (every rank encodes its
+    message, the packetised all-reduce sums the packets and re-encodes the
+    result, every rank decodes it).  The three share the input buffers; the
+    end-to-end leg uploads the message and downloads the decoded sum."""
+    import torch
+    count = nbytes // 2
+    xs = W.ll_message(nbytes, n)
+    send = [_dev(x, torch.bfloat16) for x in xs]
+    del xs
+    tag = f"{nbytes >> 20}MiB"
+    ops = [Op(f"all_reduce/twoshot/{tag}",
+              lambda b: (lambda: M.coll_all_reduce(b["send"], b["recv"], algo=M.TWOSHOT)),
+              {"send": send, "recv": [torch.empty_like(t) for t in send]}, 2 * n * nbytes, 1,
+              {"op": "all_reduce", "algo": "twoshot", "proto": "simple", "ranks": n, "bytes_per_rank": nbytes},
+              inputs=["send"], outputs=["recv"], kernel="all_reduce/twoshot")]
+    for proto, pname in ((M.LL, "ll"), (M.LL128, "ll128")):
+        pb = M.coll_packed_bytes(nbytes, proto)
+        pin = [torch.empty(pb, dtype=torch.uint8, device="cuda") for _ in range(n)]
+        pout = [torch.empty(pb, dtype=torch.uint8, device="cuda") for _ in range(n)]
+        recv = [torch.empty_like(t) for t in send]
+
+        def pack(b, proto=proto):
+            return lambda: [M.coll_ll_pack(b["send"][r], b["pin"][r], proto, 1) for r in range(n)]
+
+        def reduce_packed(b, proto=proto):
+            return lambda: M.coll_all_reduce_packed(b["pin"], b["pout"], count, torch.bfloat16, proto, 1)
+
+        def unpack(b, proto=proto):
+            return lambda: [M.coll_ll_unpack(b["pout"][r], b["recv"][r], proto, 1) for r in range(n)]
+
+        ops += [
+            Op(f"{pname}_pack/{tag}", pack, {"send": send, "pin": pin}, n * (nbytes + pb), n,
+               {"op": f"{pname}_pack", "ranks": n, "bytes_per_rank": nbytes, "packed_bytes_per_rank": pb},
+               inputs=["send"], kernel=f"{pname}_pack"),
+            Op(f"all_reduce/{pname}/{tag}", reduce_packed, {"pin": pin, "pout": pout}, 2 * n * nbytes, 1,
+               {"op": "all_reduce_packed", "proto": pname, "ranks": n, "bytes_per_rank": nbytes,
+                "line_bytes": 2 * n * pb, "note": "gbs counts payload bytes; the roofline counts line bytes"},
+               kernel=f"all_reduce/{pname}", per_launch_bytes=2 * n * pb),
+            Op(f"{pname}_unpack/{tag}", unpack, {"pout": pout, "recv": recv}, n * (pb + nbytes), n,
+               {"op": f"{pname}_unpack", "ranks": n, "bytes_per_rank": nbytes, "packed_bytes_per_rank": pb},
+               outputs=["recv"], kernel=f"{pname}_unpack"),
+        ]
+    return ops
+
+
+def build_full_step(M, oracle):
+    """Every op of the hot path at the largest sizes (see the module docstring)."""
+    import torch
+    n = 8
+    sp, _ = build_sp_prefill(M, oracle)
+    for op in sp:
+        op.ref = None
+    ops = list(sp)
+    ops += moe_ops(M, oracle, dedup=False, chain=True)
+    for op in ops:
+        op.ref = None
+    for nbytes in FULL_STEP_AR_BYTES:
+        ops += _protocol_ops(M, nbytes, n)
+    # the TP-decode all-reduce at its largest shape, by the three algorithms
+    tokens, hidden = 256, 7168
+    S = tokens * hidden * 2
+    send = [_dev(x, torch.bfloat16) for x in W.tp_decode(tokens, hidden, n)]
+    for algo, aname in ((M.ONESHOT, "oneshot"), (M.TWOSHOT, "twoshot"), (M.RING, "ring")):
+        form = M.coll_all_reduce_form(n, tokens * hidden, torch.bfloat16, algo)
+        bufs = {"send": send, "recv": [torch.empty_like(t) for t in send]}
+        if algo == M.RING:
+            need = M.coll_all_reduce_workspace_size(n, tokens * hidden, torch.bfloat16, algo)
+            bufs["ws"] = torch.zeros(need, dtype=torch.uint8, device="cuda")
+
+        def bind(b, algo=algo):
+            ws = b.get("ws")
+            return lambda: M.coll_all_reduce(b["send"], b["recv"], algo=algo, workspace=ws)
+
+        ops.append(Op(f"all_reduce/{aname}/{tokens}x{hidden}", bind, bufs, 2 * n * S,
+                      2 * (n - 1) if form == M.RING_STEPS else 1,
+                      {"op": "all_reduce", "algo": aname, "ranks": n, "shape": [tokens, hidden], "bytes_per_rank": S,
+                       "form": FORM_NAMES[form]},
+                      inputs=["send"], outputs=["recv"],
+                      kernel="all_reduce/twoshot" if algo == M.TWOSHOT else f"all_reduce/{aname}"))
+    ids = W.sampled_token_ids(n)
+    ops.append(Op("broadcast", lambda b: (lambda: M.coll_broadcast(b["bufs"], 7)),
+                  {"bufs": [_dev(x, torch.int32) for x in ids]}, 256 * 4 * n, 1,
+                  {"op": "broadcast", "src": 7, "ranks": n, "dtype": "int32", "count": 256, "bytes_per_rank": 1024},
+                  inputs=["bufs"], outputs=["bufs"], kernel="broadcast"))
+    # reduce and scatter (no workload fixes their size): 16 MiB per rank
+    S = FULL_STEP_MOVE_BYTES
+    c = S // 2
+    xs = [_dev(x, torch.bfloat16) for x in W.ranks_values(W.W_MISC, n, c, "bf16", "normal", salt=16)]
+    ops.append(Op("reduce", lambda b: (lambda: M.coll_reduce(b["send"], b["out"], 0)),
+                  {"send": xs, "out": torch.empty(c, dtype=torch.bfloat16, device="cuda")}, n * S + S, 1,
+                  {"op": "reduce", "dst": 0, "ranks": n, "bytes_per_rank": S}, inputs=["send"], outputs=["out"],
+                  kernel="reduce"))
+    ops.append(Op("scatter", lambda b: (lambda: M.coll_scatter(b["src"], b["recv"], 0)),
+                  {"src": torch.cat(xs), "recv": [torch.empty(c, dtype=torch.bfloat16, device="cuda")
+                                                  for _ in range(n)]},
+                  2 * n * S, 1, {"op": "scatter", "src": 0, "ranks": n, "bytes_per_rank": S},
+                  inputs=["src"], outputs=["recv"], kernel="scatter"))
+    return ops, full_step_cfg(n)
+
+
 WORKLOADS = {
+    "full_step": build_full_step,
     "single_image": build_single_image,
     "ring_compare": build_ring_compare,
     "movement": build_movement,
@@ -466,6 +628,348 @@ WORKLOADS = {
     "moe": build_moe,
     "ll_sweep": build_ll_sweep,
 }
+
+
+# ---------------------------------------------------- the oracle on the host ----
+#
+# The CPU baseline and the reference arm run the oracle, as it stands, on a
+# sample of a workload: each op is split into independent parts (element
+# ranges, rows, or groups of tokens, each a smaller instance of the same op on
+# the same kind of inputs) that worker processes, one per core, run at once.
+# The parts' inputs are written once into a file that every worker maps, so a
+# step moves no input between processes; what a step times is the oracle's
+# own work on every part of every op.
+
+ORACLE_SAMPLE = 16  # the oracle's sample is 1/ORACLE_SAMPLE of every op of a workload
+
+
+class HostOp:
+    """One op of a workload for the CPU oracle.  ``kind`` names a task in
+    HOST_TASKS; ``pieces`` are its independent parts, each a dict of arrays
+    (with the part's own parameters in ``params``); ``alg_bytes`` is what the
+    whole (sampled) op must read plus write."""
+
+    def __init__(self, name, kind, pieces, alg_bytes, **params):
+        self.name, self.kind, self.alg_bytes, self.params = name, kind, alg_bytes, params
+        self.pieces = [p for p in pieces if p is not None]
+
+
+HOST_TASKS = {}  # kind -> fn(oracle module, the piece's arrays, params) -> the oracle's result
+
+
+def _host_task(kind):
+    def deco(fn):
+        HOST_TASKS[kind] = fn
+        return fn
+    return deco
+
+
+@_host_task("broadcast")
+def _t_broadcast(o, a, prm):
+    return o.broadcast(list(a["x"]), prm["src"])
+
+
+@_host_task("gather")
+def _t_gather(o, a, prm):
+    return o.gather(list(a["x"]), a["dst"], rows=int(a["x"].shape[1] // prm["cols"]))
+
+
+@_host_task("reduce")
+def _t_reduce(o, a, prm):
+    return o.reduce(list(a["x"]), 0, prm["dtype"])
+
+
+@_host_task("scatter")
+def _t_scatter(o, a, prm):
+    return o.scatter(a["src"], prm["n"])
+
+
+@_host_task("reduce_scatter")
+def _t_reduce_scatter(o, a, prm):
+    return o.reduce_scatter(list(a["x"]), 0, prm["dtype"])
+
+
+@_host_task("all_gather")
+def _t_all_gather(o, a, prm):
+    return o.all_gather(list(a["x"]))
+
+
+@_host_task("all_reduce")
+def _t_all_reduce(o, a, prm):
+    fn = {"oneshot": o.all_reduce_one_shot, "twoshot": o.all_reduce_two_shot, "ring": o.all_reduce_ring}[prm["algo"]]
+    return fn(list(a["x"]), 0, prm["dtype"])
+
+
+@_host_task("pack")
+def _t_pack(o, a, prm):
+    return [o.pack(x, prm["proto"], 1) for x in a["x"]]
+
+
+@_host_task("all_reduce_packed")
+def _t_all_reduce_packed(o, a, prm):
+    p = a["p"]
+    return o.all_reduce_packed(list(p), int(a["count"][0]), "bf16", 0, prm["proto"], 1)
+
+
+@_host_task("unpack")
+def _t_unpack(o, a, prm):
+    nbytes = int(a["count"][0]) * 2
+    return [o.unpack(p, nbytes, prm["proto"], 1) for p in a["p"]]
+
+
+@_host_task("moe_route")
+def _t_moe_route(o, a, prm):
+    return o.moe_route(list(a["ids"]), prm["experts"])
+
+
+@_host_task("moe_dispatch")
+def _t_moe_dispatch(o, a, prm):
+    n = a["ids"].shape[0]
+    return o.moe_dispatch(list(a["x"]), list(a["ids"]), list(a["pos"]), [a[f"recv{d}"] for d in range(n)],
+                          prm["experts"], prm["hidden"])
+
+
+@_host_task("moe_combine")
+def _t_moe_combine(o, a, prm):
+    n = a["ids"].shape[0]
+    return o.moe_combine([a[f"y{d}"] for d in range(n)], list(a["ids"]), list(a["pos"]), list(a["w"]),
+                         prm["experts"], prm["hidden"], "bf16")
+
+
+def _split(total: int, parts: int, align: int = 1):
+    """[lo, hi) ranges cutting [0, total) into at most ``parts`` pieces whose
+    starts are multiples of ``align``."""
+    step = max(align, -(-total // max(1, parts) // align) * align) if total else align
+    return [(lo, min(total, lo + step)) for lo in range(0, total, step)]
+
+
+def _stack(xs):
+    return np.ascontiguousarray(np.stack([np.asarray(x) for x in xs]))
+
+
+def host_ar_pieces(oracle, xs, parts, name, algo, alg_per_elem, align=8, whole=False):
+    n, e = len(xs), xs[0].size
+    x = _stack(xs)
+    rng_ = [(0, e)] if whole else _split(e, parts, align)
+    return HostOp(name, "all_reduce", [{"x": np.ascontiguousarray(x[:, lo:hi])} for lo, hi in rng_],
+                  alg_per_elem * e, algo=algo, dtype="bf16")
+
+
+def host_full_step(oracle, parts: int, frac: int = ORACLE_SAMPLE):
+    """The default workload for the oracle: every op at 1/frac of its size,
+    on the first part of each rank's own input stream (MoE: the first
+    tokens of each rank), each op cut into about ``parts`` pieces."""
+    n = 8
+    ops = []
+    # sequence-parallel prefill
+    rows = 1024 // frac
+    x = _stack(W.sp_allgather(n, rows=rows))
+    e = x.shape[1]
+    ops.append(HostOp("all_gather", "all_gather", [{"x": np.ascontiguousarray(x[:, lo:hi])}
+                                                   for lo, hi in _split(e, parts, 8)], (n + n * n) * e * 2))
+    rows = 8192 // frac
+    x = _stack(W.sp_reduce_scatter(n, rows=rows)).reshape(n, n, -1)  # [rank, output block, element]
+    e = x.shape[2]
+    ops.append(HostOp("reduce_scatter", "reduce_scatter",
+                      [{"x": np.ascontiguousarray(x[:, :, lo:hi]).reshape(n, -1)} for lo, hi in _split(e, parts, 8)],
+                      (n * n * e + n * e) * 2, dtype="bf16"))
+    rows, cols = 256 // frac, 16032
+    x = _stack(W.logits_shards(n, rows=rows)).reshape(n, rows, cols)
+    ops.append(HostOp("gather", "gather",
+                      [{"x": np.ascontiguousarray(x[:, lo:hi]).reshape(n, -1),
+                        "dst": np.zeros((hi - lo) * n * cols, np.float32)} for lo, hi in _split(rows, parts)],
+                      2 * n * rows * cols * 4, cols=cols))
+    # MoE: each piece is the route, dispatch and combine of a group of tokens
+    tokens, topk, experts, hidden = 4096 // frac, 8, 256, 7168
+    ids, ws = W.moe_routing(tokens, experts, topk, n)
+    xt = _stack(W.moe_tokens(tokens, hidden, n)).reshape(n, tokens, hidden)
+    route, disp, comb = [], [], []
+    for lo, hi in _split(tokens, parts):
+        pid = np.ascontiguousarray(np.stack([i[lo:hi] for i in ids]))
+        pw = np.ascontiguousarray(np.stack([w[lo:hi] for w in ws]))
+        px = np.ascontiguousarray(xt[:, lo:hi]).reshape(n, -1)
+        sc, _sd, _rd, pos = oracle.moe_route(list(pid), experts)
+        recv0 = [np.zeros(int(sc[:, d].sum()) * hidden, np.uint16) for d in range(n)]
+        y = oracle.moe_dispatch(list(px), list(pid), pos, recv0, experts, hidden)
+        ppos = np.ascontiguousarray(np.stack(pos))
+        route.append({"ids": pid})
+        disp.append({"ids": pid, "x": px, "pos": ppos, **{f"recv{d}": recv0[d] for d in range(n)}})
+        comb.append({"ids": pid, "w": pw, "pos": ppos, **{f"y{d}": y[d] for d in range(n)}})
+    pairs, row = n * tokens * topk, hidden * 2
+    ops.append(HostOp("moe_route", "moe_route", route, pairs * 4 * 2, experts=experts))
+    ops.append(HostOp("moe_dispatch", "moe_dispatch", disp, n * tokens * row + pairs * row, experts=experts,
+                      hidden=hidden))
+    ops.append(HostOp("moe_combine", "moe_combine", comb, pairs * row + pairs * 4 + n * tokens * row,
+                      experts=experts, hidden=hidden))
+    # all-reduce of the 16 MiB and 256 MiB messages: Simple, LL, LL128
+    for nbytes in FULL_STEP_AR_BYTES:
+        count = nbytes // 2 // frac
+        xs = W.ll_message(nbytes, n, elems=count)
+        tag = f"{nbytes >> 20}MiB"
+        ops.append(host_ar_pieces(oracle, xs, parts, f"all_reduce/twoshot/{tag}", "twoshot", 2 * n * 2, align=960))
+        x = _stack(xs)
+        for proto, pname in ((oracle.LL, "ll"), (oracle.LL128, "ll128")):
+            pk, ar, up = [], [], []
+            for lo, hi in _split(count, parts, 960):  # 1920 bytes: whole 16-byte groups and whole LL128 lines
+                part = np.ascontiguousarray(x[:, lo:hi])
+                packed = np.ascontiguousarray(np.stack([oracle.pack(v, proto, 1) for v in part]))
+                cnt = np.array([hi - lo], np.int64)
+                pk.append({"x": part})
+                ar.append({"p": packed, "count": cnt})
+                up.append({"p": packed, "count": cnt})
+            pb = oracle.packed_bytes(count * 2, proto)
+            ops.append(HostOp(f"{pname}_pack/{tag}", "pack", pk, n * (count * 2 + pb), proto=proto))
+            ops.append(HostOp(f"all_reduce/{pname}/{tag}", "all_reduce_packed", ar, 2 * n * count * 2, proto=proto))
+            ops.append(HostOp(f"{pname}_unpack/{tag}", "unpack", up, n * (count * 2 + pb), proto=proto))
+    # TP decode at [256, 7168]: one-shot, two-shot, ring; the broadcast
+    e = 256 * 7168 // frac
+    xs = W.tp_decode(256, 7168, n, elems=e)
+    ops.append(host_ar_pieces(oracle, xs, parts, "all_reduce/oneshot/256x7168", "oneshot", 2 * n * 2))
+    ops.append(host_ar_pieces(oracle, xs, parts, "all_reduce/twoshot/256x7168", "twoshot", 2 * n * 2))
+    # the ring's chunks (hence its order of addition) follow from the whole
+    # message, so it runs as one piece
+    ops.append(host_ar_pieces(oracle, xs, parts, "all_reduce/ring/256x7168", "ring", 2 * n * 2, whole=True))
+    ops.append(HostOp("broadcast", "broadcast", [{"x": _stack(W.sampled_token_ids(n))}], 256 * 4 * n, src=7))
+    # reduce and scatter
+    c = FULL_STEP_MOVE_BYTES // 2 // frac
+    x = _stack(W.ranks_values(W.W_MISC, n, c, "bf16", "normal", salt=16))
+    ops.append(HostOp("reduce", "reduce", [{"x": np.ascontiguousarray(x[:, lo:hi])} for lo, hi in _split(c, parts, 8)],
+                      (n * c + c) * 2, dtype="bf16"))
+    ops.append(HostOp("scatter", "scatter",
+                      [{"src": np.ascontiguousarray(x[:, lo:hi]).reshape(-1)} for lo, hi in _split(c, parts, 8)],
+                      2 * n * c * 2, n=n))
+    desc = (f"every op of the workload at 1/{frac} of its size (the first 1/{frac} of each rank's own seeded input; "
+            f"MoE: the first {tokens} tokens of each rank), each op cut into up to {parts} independent pieces")
+    return ops, full_step_cfg(n), desc
+
+
+def host_tp_decode(oracle, parts: int):
+    n = 8
+    ops = []
+    for tokens, hidden in W.tp_decode_shapes():
+        xs = W.tp_decode(tokens, hidden, n)
+        for algo in ("oneshot", "twoshot"):
+            ops.append(host_ar_pieces(oracle, xs, parts, f"all_reduce/{algo}/{tokens}x{hidden}", algo, 2 * n * 2))
+        ops.append(host_ar_pieces(oracle, xs, parts, f"all_reduce/ring/{tokens}x{hidden}", "ring", 2 * n * 2,
+                                  whole=True))
+    ops.append(HostOp("broadcast", "broadcast", [{"x": _stack(W.sampled_token_ids(n))}], 256 * 4 * n, src=7))
+    return ops, tp_decode_cfg(n), "every op of the workload at full size, one-shot and two-shot cut into pieces"
+
+
+def host_twoshot_160k(oracle, parts: int):
+    xs = W.twoshot_160k(4)
+    ops = [host_ar_pieces(oracle, xs, parts, "all_reduce/twoshot", "twoshot", 2 * 4 * 2)]
+    return ops, twoshot_160k_cfg(4), "the workload at full size, cut into pieces"
+
+
+HOST_WORKLOADS = {"full_step": host_full_step, "tp_decode": host_tp_decode, "twoshot_160k": host_twoshot_160k}
+
+_WORKER = {}
+
+
+def _worker_init(path, manifest):
+    import oracle
+    mm = np.memmap(path, dtype=np.uint8, mode="c")
+    views = {}
+    for key, arrays in manifest.items():
+        views[key] = {nm: np.ndarray(shape, dtype=np.dtype(dt), buffer=mm, offset=off)
+                      for nm, (off, dt, shape) in arrays.items()}
+    _WORKER.update(oracle=oracle, mm=mm, views=views)
+
+
+def _worker_run(task):
+    i, p, kind, params = task
+    HOST_TASKS[kind](_WORKER["oracle"], _WORKER["views"][(i, p)], params)  # the result stays in the worker
+    return i
+
+
+class OracleRunner:
+    """The host ops of a workload on ``workers`` processes (spawned, so that
+    it is safe after CUDA has been used in the parent)."""
+
+    def __init__(self, ops, workers: int):
+        import multiprocessing as mp
+        import oracle
+        self.ops, self.oracle = ops, oracle
+        self.bytes_per_step = sum(op.alg_bytes for op in ops)
+        self.tasks = [(i, p, op.kind, op.params) for i, op in enumerate(ops) for p in range(len(op.pieces))]
+        # biggest pieces first, so that the last ones to start are short
+        size = {(i, p): sum(a.nbytes for a in ops[i].pieces[p].values()) for i, p, _, _ in self.tasks}
+        self.tasks.sort(key=lambda t: -size[(t[0], t[1])])
+        fd, self.path = tempfile.mkstemp(prefix="mvr_oracle_", suffix=".bin")
+        manifest, off = {}, 0
+        with os.fdopen(fd, "wb") as f:
+            for i, op in enumerate(ops):
+                for p, arrays in enumerate(op.pieces):
+                    entry = {}
+                    for nm, a in arrays.items():
+                        a = np.ascontiguousarray(a)
+                        pad = (-off) % 64
+                        f.write(b"\0" * pad)
+                        off += pad
+                        entry[nm] = (off, a.dtype.str, a.shape)
+                        f.write(a.tobytes())
+                        off += a.nbytes
+                    manifest[(i, p)] = entry
+            f.write(b"\0" * 64)
+        self.workers = workers
+        self.pool = mp.get_context("spawn").Pool(workers, initializer=_worker_init, initargs=(self.path, manifest))
+
+    def step(self) -> float:
+        t0 = time.perf_counter()
+        for _ in self.pool.imap_unordered(_worker_run, self.tasks, chunksize=1):
+            pass
+        return time.perf_counter() - t0
+
+    def single_thread_step(self) -> float:
+        """The same tasks one after another in this process, on one core."""
+        t0 = time.perf_counter()
+        for i, p, kind, params in self.tasks:
+            HOST_TASKS[kind](self.oracle, self.ops[i].pieces[p], params)
+        return time.perf_counter() - t0
+
+    def close(self):
+        self.pool.terminate()
+        self.pool.join()
+        with contextlib.suppress(OSError):
+            os.remove(self.path)
+
+
+def oracle_workers() -> int:
+    """One worker per core this process may run on (at most 64)."""
+    return max(1, min(64, len(os.sched_getaffinity(0))))
+
+
+def host_workload(workload: str, oracle, parts: int):
+    if workload not in HOST_WORKLOADS:
+        raise SystemExit(f"--impl reference supports {', '.join(sorted(HOST_WORKLOADS))}, not {workload}")
+    return HOST_WORKLOADS[workload](oracle, parts)
+
+
+def time_oracle(workload: str, min_s: float = 10.0, max_s: float = 30.0):
+    """The CPU baseline of the GPU arm: whole sampled steps of the workload
+    on all cores until about ``min_s`` seconds (at most ``max_s``), then one
+    step on one core.  Returns the cpu_baseline object, or None when the
+    workload has no oracle step."""
+    import oracle
+    if workload not in HOST_WORKLOADS:
+        return None
+    workers = oracle_workers()
+    ops, _cfg, desc = host_workload(workload, oracle, workers)
+    run = OracleRunner(ops, workers)
+    try:
+        run.step()  # warm-up: workers map their inputs
+        secs, steps = 0.0, 0
+        while secs < min_s and secs < max_s:
+            secs += run.step()
+            steps += 1
+        single = run.single_thread_step()
+    finally:
+        run.close()
+    return {"value": round(run.bytes_per_step * steps / secs / 1e9, 4), "unit": "GB/s", "cores": workers,
+            "cpu_model": cpu_model(), "kind": "oracle", "sample": f"{steps} steps of {desc}",
+            "seconds": round(secs, 2), "single_thread_value": round(run.bytes_per_step / single / 1e9, 4),
+            "single_thread_seconds_per_step": round(single, 3)}
 
 
 # ---------------------------------------------------------------- clocks ----
@@ -595,10 +1099,6 @@ def barrier(world: int):
         dist.barrier()
 
 
-def cpu_cores_used() -> int:
-    return 1  # numpy element-wise kernels run on the calling thread
-
-
 def cpu_model() -> str:
     try:
         for line in open("/proc/cpuinfo"):
@@ -627,31 +1127,6 @@ def empty_kernel_graph_us(stream, reps: int = 50) -> float:
     us = a.elapsed_time(b) * 1e3 / reps
     del g
     return round(us, 3)
-
-
-def time_oracle(ops, min_s: float = 10.0, max_s: float = 30.0):
-    """Run the oracle version of the step's ops, whole steps at a time, until
-    about ``min_s`` seconds of CPU work (at most ``max_s``); returns
-    (GB/s, sample description, seconds)."""
-    refs = [op for op in ops if op.ref is not None]
-    if not refs:
-        return None, "no op of this workload has a CPU definition", 0.0
-    secs, nbytes, ops_done = 0.0, 0, 0
-    while secs < min_s:
-        for op in refs:
-            t0 = time.perf_counter()
-            op.ref()
-            secs += time.perf_counter() - t0
-            nbytes += op.alg_bytes
-            ops_done += 1
-            if secs > max_s:
-                break
-        if secs > max_s:
-            break
-    kinds = sorted(set(op.name.split("/")[0] for op in refs))
-    sample = (f"{ops_done} oracle op calls = {ops_done / max(1, len(refs)):.2f} full steps of the same workload "
-              f"({', '.join(kinds)}), full-size inputs")
-    return (nbytes / secs / 1e9 if secs > 0 else None), sample, secs
 
 
 def graph_latency(ops, stream, reps: int = 50, max_bytes_per_rank: int = 256 * 1024):
@@ -686,7 +1161,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="tp_decode", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="full_step", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
@@ -819,9 +1294,17 @@ def main():
     # download of the one before (PCIe is full duplex).  Events bracket whole
     # steps.
     e2e = None
-    if not args.no_e2e and all(op.inputs and op.outputs for op in ops):
-        pinned = {id(op): ([(t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True))
-                            for nm in op.inputs for t in _as_list(op.bufs[nm])],
+    if not args.no_e2e and any(op.inputs for op in ops) and any(op.outputs for op in ops):
+        host_in = {}  # one pinned source per device input buffer, shared by the ops that upload it
+
+        def pinned_in(t):
+            if t.data_ptr() not in host_in:
+                h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                h.copy_(t)
+                host_in[t.data_ptr()] = h
+            return host_in[t.data_ptr()]
+
+        pinned = {id(op): ([(t, pinned_in(t)) for nm in op.inputs for t in _as_list(op.bufs[nm])],
                            [(t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True))
                             for nm in op.outputs for t in _as_list(op.bufs[nm])]) for op in ops}
 
@@ -877,7 +1360,9 @@ def main():
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "how": "per op: pinned host->device copy of its inputs, the call through the Python binding of the "
                       "C ABI, device->host copy of its outputs, on three streams (an upload overlaps the previous "
-                      "op's download); CUDA events around the timed steps"}
+                      "op's download); in a chain of ops (encode, packetised sum, decode; MoE route, dispatch, "
+                      "combine) only what a caller holds on the host goes up and only the chain's result comes "
+                      "down; CUDA events around the timed steps"}
 
     per_op, by_kernel = [], {}
     for op in ops:
@@ -913,11 +1398,8 @@ def main():
     launches = sum(op.launches * graphs[id(op)][1] for op in ops) * args.steps
 
     cpu = None
-    if rank == 0 and not args.no_cpu_baseline:
-        v, sample, secs = time_oracle(ops)
-        cpu = {"value": round(v, 4) if v else None, "unit": "GB/s", "cores": cpu_cores_used(), "cpu_model": cpu_model(),
-               "kind": "oracle",
-               "sample": sample, "seconds": round(secs, 2)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = time_oracle(args.workload)
 
     if rank == 0:
         line = {"metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -945,54 +1427,34 @@ def main():
 
 
 def main_reference(args, rank, world):
-    """The oracle as it stands, on the host's cores (rank 0 only)."""
+    """The oracle as it stands, on the host's cores (rank 0 only), on a
+    bounded sample of the same workload."""
     if rank != 0:
         return
     import oracle
 
-    ops, cfg = host_ops(args.workload, oracle)
-    times = []
-    nbytes = sum(alg for alg, _ in ops)
-    for k in range(max(args.warmup, 0) + args.steps):
-        t0 = time.perf_counter()
-        for _, ref in ops:
-            ref()
-        dt = time.perf_counter() - t0
-        if k >= args.warmup:
-            times.append(dt)
+    workers = oracle_workers()
+    ops, cfg, desc = host_workload(args.workload, oracle, workers)
+    run = OracleRunner(ops, workers)
+    try:
+        for _ in range(max(args.warmup, 0)):
+            run.step()
+        times = [run.step() for _ in range(args.steps)]
+        single = run.single_thread_step()
+    finally:
+        run.close()
     total = sum(times)
-    value = nbytes * len(times) / total / 1e9
-    sample = f"every op of the workload, full size, {len(times)} timed passes on one core"
+    value = run.bytes_per_step * len(times) / total / 1e9
     line = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(total / len(times) * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "reference",
             "config": cfg,
-            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cpu_cores_used(), "cpu_model": cpu_model(),
-                             "kind": "oracle",
-                             "sample": sample},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": workers, "cpu_model": cpu_model(),
+                             "kind": "oracle", "sample": f"each step: {desc}",
+                             "single_thread_value": round(run.bytes_per_step / single / 1e9, 4),
+                             "single_thread_seconds_per_step": round(single, 3)},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
-
-
-def host_ops(workload: str, oracle):
-    """The workload's ops as (algorithmic bytes, oracle call) on host inputs (no GPU)."""
-    ops = []
-    if workload == "tp_decode":
-        n = 8
-        for tokens, hidden in W.tp_decode_shapes():
-            xs = W.tp_decode(tokens, hidden, n)
-            S = tokens * hidden * 2
-            for ref in (oracle.all_reduce_one_shot, oracle.all_reduce_two_shot, oracle.all_reduce_ring):
-                ops.append((2 * n * S, lambda xs=xs, ref=ref: ref(xs, 0, "bf16")))
-        ids = W.sampled_token_ids(n)
-        ops.append((256 * 4 * n, lambda: oracle.broadcast(ids, 7)))
-        cfg = tp_decode_cfg(n)
-        return ops, cfg
-    if workload == "twoshot_160k":
-        xs = W.twoshot_160k(4)
-        ops.append((2 * 4 * xs[0].size * 2, lambda: oracle.all_reduce_two_shot(xs, 0, "bf16")))
-        return ops, twoshot_160k_cfg(4)
-    raise SystemExit(f"--impl reference supports tp_decode and twoshot_160k, not {workload}")
 
 
 if __name__ == "__main__":

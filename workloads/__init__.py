@@ -124,10 +124,14 @@ def tp_decode_shapes() -> list[tuple[int, int]]:
     return [(t, h) for h in TP_DECODE_HIDDEN for t in TP_DECODE_TOKENS]
 
 
-def tp_decode(tokens: int, hidden: int, nranks: int = 8) -> list[np.ndarray]:
-    """Per-rank RowParallelLinear partial outputs, bf16 [tokens, hidden], N(0,1)."""
+def tp_decode(tokens: int, hidden: int, nranks: int = 8, elems: int | None = None) -> list[np.ndarray]:
+    """Per-rank RowParallelLinear partial outputs, bf16 [tokens, hidden], N(0,1).
+
+    ``elems`` (optional) returns only the first ``elems`` values of each
+    rank's input: a prefix sample of the same workload."""
     salt = tokens * 100003 + hidden
-    return ranks_values(W_TP_DECODE, nranks, tokens * hidden, "bf16", "normal", salt=salt)
+    return ranks_values(W_TP_DECODE, nranks, tokens * hidden if elems is None else elems, "bf16", "normal",
+                        salt=salt)
 
 
 def sampled_token_ids(nranks: int = 8, count: int = 256) -> list[np.ndarray]:
@@ -148,9 +152,11 @@ def logits_shards(nranks: int = 8, rows: int = 256, cols: int = 16032) -> list[n
     return ranks_values(W_SP_PREFILL, nranks, rows * cols, "fp32", "normal", std=2.0, salt=3)
 
 
-def ll_message(nbytes: int, nranks: int = 8) -> list[np.ndarray]:
-    """bf16 uniform[-1, 1] payloads of ``nbytes`` bytes (uint16 bits)."""
-    return ranks_values(W_LL_SWEEP, nranks, nbytes // 2, "bf16", "uniform", salt=nbytes.bit_length())
+def ll_message(nbytes: int, nranks: int = 8, elems: int | None = None) -> list[np.ndarray]:
+    """bf16 uniform[-1, 1] payloads of ``nbytes`` bytes (uint16 bits); with
+    ``elems``, only the first ``elems`` values of each (a prefix sample)."""
+    return ranks_values(W_LL_SWEEP, nranks, nbytes // 2 if elems is None else elems, "bf16", "uniform",
+                        salt=nbytes.bit_length())
 
 
 # --------------------------------------------------------------------------
