@@ -157,9 +157,8 @@ def test_all_gather_in_place_and_unaligned():
 
 
 def test_sp_all_gather_workload():
-    """8 ranks x bf16 [1024, 8192] -> every rank [8192, 8192]: every block of
-    every output compared on the device with the source slice, plus 4096
-    sampled elements per output against the oracle on the host."""
+    """8 ranks x bf16 [1024, 8192] -> every rank [8192, 8192]: every element of
+    every output against the oracle's all-gather."""
     need_gpu()
     n, rows, cols = 8, 1024, 8192
     xs = W.sp_allgather(n, rows, cols)
@@ -168,15 +167,9 @@ def test_sp_all_gather_workload():
     recv = [torch.empty(n * c, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
     M.coll_all_gather(send, recv)
     torch.cuda.synchronize()
+    want = oracle.all_gather(xs)
     for q in range(n):
-        for r in range(n):
-            assert torch.equal(recv[q][r * c:(r + 1) * c].view(torch.int16), send[r].view(torch.int16))
-    g = W.rng(W.W_MISC, 0, salt=5)
-    full = np.concatenate(xs)
-    for q in range(n):
-        idx = g.choice(n * c, 4096, replace=False)
-        got = from_dev(recv[q][torch.from_numpy(idx).cuda()], "bf16")
-        assert np.array_equal(got, full[idx])
+        assert np.array_equal(from_dev(recv[q], "bf16"), want[q]), q
 
 
 @pytest.mark.parametrize("n", [1, 2, 3, 8])

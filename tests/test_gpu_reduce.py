@@ -195,11 +195,12 @@ def test_reduce(dtype, op):
     assert np.array_equal(bits(from_dev(send[2], dtype)), bits(oracle.reduce(xs, op, dtype)))
 
 
-def test_sp_prefill_reduce_scatter_full_size_sampled():
+def test_sp_prefill_reduce_scatter_full_size():
     """8 ranks x bf16 [8192, 8192] -> [1024, 8192] blocks (the sequence-parallel
-    prefill reduce-scatter), checked on 4096 sampled elements per output block
-    against the oracle, plus the identity AllReduce == AllGather(ReduceScatter)
-    on device for one block."""
+    prefill reduce-scatter), every element of every output block against the
+    oracle.  The oracle runs on chunks of the block's element range (each
+    element of a reduce-scatter depends only on the same element of every
+    rank's input), so host memory stays bounded."""
     need_gpu()
     n, rows, cols = 8, 8192, 8192
     xs = W.sp_reduce_scatter(n, rows, cols)
@@ -208,10 +209,37 @@ def test_sp_prefill_reduce_scatter_full_size_sampled():
     recv = [torch.empty(per, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
     M.coll_reduce_scatter(send, recv)
     torch.cuda.synchronize()
-    g = W.rng(W.W_MISC, 0, salt=99)
-    for r in range(n):
-        idx = np.sort(g.choice(per, 4096, replace=False))
-        want = oracle.reduce([x[r * per + idx] for x in xs], 0, "bf16")
-        got = from_dev(recv[r], "bf16")[idx]
-        assert np.array_equal(got, want), r
     del send
+    chunk = 1 << 20
+    for lo in range(0, per, chunk):
+        hi = min(per, lo + chunk)
+        part = [np.concatenate([x[b * per + lo:b * per + hi] for b in range(n)]) for x in xs]
+        want = oracle.reduce_scatter(part, 0, "bf16")
+        for r in range(n):
+            assert np.array_equal(from_dev(recv[r][lo:hi], "bf16"), want[r]), (r, lo)
+
+
+@pytest.mark.parametrize("n,last", [(3, 256 << 10), (4, 64 << 10), (2, None), (8, None)])
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_auto_both_sides_of_each_crossover(n, last, dtype):
+    """AUTO at the measured crossovers: the form it reports on each side, and
+    the result of the call against the oracle (both forms give the
+    rank-order reduction), out of place and in place (always the two-shot)."""
+    need_gpu()
+    es = 2 if dtype == "bf16" else 4
+    edge = last if last is not None else 64 << 10
+    for nbytes in (edge, edge + 16):
+        count = nbytes // es
+        want_form = M.ONESHOT if last is not None and nbytes <= last else M.TWOSHOT
+        tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+        assert M.coll_all_reduce_form(n, count, tdt, M.ALGO_AUTO) == want_form
+        xs = inputs(n, count, dtype, salt=nbytes + n)
+        want = oracle.all_reduce(xs, 0, dtype)
+        send = [to_dev(x, dtype) for x in xs]
+        recv = [torch.empty_like(t) for t in send]
+        M.coll_all_reduce(send, recv, algo=M.ALGO_AUTO)
+        M.coll_all_reduce(send, send, algo=M.ALGO_AUTO)  # in place
+        torch.cuda.synchronize()
+        for q in range(n):
+            assert np.array_equal(bits(from_dev(recv[q], dtype)), bits(want[q])), (nbytes, q)
+            assert np.array_equal(bits(from_dev(send[q], dtype)), bits(want[q])), (nbytes, q)
