@@ -617,8 +617,53 @@ def build_full_step(M, oracle):
     return ops, full_step_cfg(n)
 
 
+FORMS_RANKS = (2, 3, 4, 8)
+FORMS_BYTES = tuple(1 << k for k in range(10, 29, 2))  # 1 KiB .. 256 MiB per rank
+
+
+def build_allreduce_forms(M, oracle):
+    """Every one-launch all-reduce form (one-shot, two-shot, the CTA and
+    cluster rings, the fused LL two-shot and ring) on bf16 messages of 1 KiB
+    .. 256 MiB per rank at 2, 3, 4 and 8 virtual ranks: the measurements the
+    AUTO choice rests on.  The LL forms move 4x the payload through L2 and
+    stop at 16 MiB (two-shot) and 4 MiB (ring) per rank.  Inputs are seeded
+    normal values drawn on the device (timing only)."""
+    import torch
+    g = torch.Generator(device="cuda")
+    g.manual_seed(W.SEED_BASE + 77)
+    ops = []
+    forms = ((M.ONESHOT, "oneshot", None), (M.TWOSHOT, "twoshot", None), (M.RING_CTA, "ring_cta", None),
+             (M.RING_CLUSTER, "ring_cluster", None), (M.TWOSHOT_LL, "twoshot_ll", 16 << 20),
+             (M.RING_LL, "ring_ll", 4 << 20))
+    for n in FORMS_RANKS:
+        for nbytes in FORMS_BYTES:
+            count = nbytes // 2
+            send = [torch.randn(count, generator=g, device="cuda").to(torch.bfloat16) for _ in range(n)]
+            recv = [torch.empty_like(t) for t in send]
+            for algo, aname, cap in forms:
+                if cap is not None and nbytes > cap:
+                    continue
+                bufs = {"send": send, "recv": recv}
+                need = M.coll_all_reduce_workspace_size(n, count, torch.bfloat16, algo)
+                if need:
+                    bufs["ws"] = torch.zeros(need, dtype=torch.uint8, device="cuda")
+
+                def bind(b, algo=algo):
+                    ws = b.get("ws")
+                    return lambda: M.coll_all_reduce(b["send"], b["recv"], algo=algo, workspace=ws)
+
+                ops.append(Op(f"all_reduce/{aname}/{n}x{nbytes}", bind, bufs, 2 * n * nbytes, 1,
+                              {"op": "all_reduce", "algo": aname, "ranks": n, "bytes_per_rank": nbytes},
+                              kernel=f"all_reduce/{aname}"))
+    return ops, {"workload": "allreduce_forms_sweep", "virtual_ranks": list(FORMS_RANKS),
+                 "bytes_per_rank": list(FORMS_BYTES), "dtype": "bf16",
+                 "forms": ["oneshot", "twoshot", "ring_cta", "ring_cluster", "twoshot_ll <= 16 MiB",
+                           "ring_ll <= 4 MiB"]}
+
+
 WORKLOADS = {
     "full_step": build_full_step,
+    "allreduce_forms": build_allreduce_forms,
     "single_image": build_single_image,
     "ring_compare": build_ring_compare,
     "movement": build_movement,

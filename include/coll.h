@@ -79,7 +79,7 @@ typedef struct CUstream_st* coll_stream_t; /* identical to cudaStream_t */
 typedef enum { COLL_BF16 = 0, COLL_FP16 = 1, COLL_FP32 = 2, COLL_INT32 = 3 } coll_dtype_t;
 typedef enum { COLL_SUM = 0, COLL_MAX = 1, COLL_MIN = 2, COLL_PROD = 3 } coll_op_t;
 typedef enum {
-  COLL_ALGO_AUTO = 0,    /* currently TWOSHOT */
+  COLL_ALGO_AUTO = 0,    /* the measured fastest: ONESHOT or TWOSHOT by ranks and size */
   COLL_ALGO_ONESHOT = 1, /* every rank reads all N inputs itself            */
   COLL_ALGO_TWOSHOT = 2, /* owner s reduces segment s, sends it to everyone */
   COLL_ALGO_RING = 3,    /* 2(N-1) neighbour steps: RING_CTA, else RING_STEPS */
@@ -232,7 +232,12 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    Buffers that are not
  *    16-byte aligned take the TWOSHOT kernel.  Needs N x (CTAs per SM) to
  *    fit on the GPU at once (COLL_ERR_UNSUPPORTED otherwise).
- *  AUTO picks TWOSHOT.  ONESHOT and TWOSHOT ignore `workspace`.
+ *  AUTO picks the form measured fastest on B200 for N and the bytes per rank
+ *    (1 KiB .. 256 MiB per rank at 2, 3, 4 and 8 ranks, every one-launch
+ *    form): ONESHOT for N == 3 up to 256 KiB and for N == 4 up to 64 KiB
+ *    per rank, TWOSHOT otherwise, and TWOSHOT for any in-place call (ONESHOT
+ *    cannot run in place).  Both give the rank-order result, so AUTO's bits
+ *    do not depend on the choice.  ONESHOT and TWOSHOT ignore `workspace`.
  * In place (recv[r] == send[r]) is allowed for every algorithm but ONESHOT. */
 COLL_API int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size_t count,
                     coll_dtype_t dtype, coll_op_t op, coll_algo_t algo, void* workspace,
@@ -241,8 +246,8 @@ COLL_API size_t coll_all_reduce_workspace_size(int nranks, size_t count, coll_dt
                                       coll_algo_t algo);
 /* The form coll_all_reduce() runs for these arguments when nranks >= 2 and
  * count >= 1: ONESHOT, TWOSHOT, TWOSHOT_LL, RING_LL, RING_CLUSTER, RING_CTA
- * or RING_STEPS (AUTO and RING resolved; `aligned` != 0 when every buffer is
- * 16-byte aligned).  RING_STEPS launches 2(N-1) kernels, the others one.
+ * or RING_STEPS (AUTO and RING resolved, AUTO for a call that is not in
+ * place; `aligned` != 0 when every buffer is 16-byte aligned).  RING_STEPS launches 2(N-1) kernels, the others one.
  * Returns a negative COLL_ERR_* for an invalid rank count, dtype or algo.
  * Library introspection; the sources have no counterpart. */
 COLL_API int coll_all_reduce_form(int nranks, size_t count, coll_dtype_t dtype, coll_algo_t algo,

@@ -336,6 +336,21 @@ static coll_algo_t ring_form(int nranks, bool vec) {
   return (vec && ring_cta_supported(nranks)) ? COLL_ALGO_RING_CTA : COLL_ALGO_RING_STEPS;
 }
 
+// AUTO: the form measured fastest on B200 for the rank count and the bytes
+// per rank (cold inputs, 1 KiB .. 256 MiB per rank, 2, 3, 4 and 8 virtual
+// ranks, every one-launch form).  At 3 and 4 ranks the one-shot, every output
+// rank reading all inputs itself, beats the owner segments on small messages
+// (by up to 0.3 us); everywhere else the two-shot is fastest or tied (at 8
+// ranks and 256 MiB the CTA ring is within 1.5% of it).  Rank counts that were
+// not measured take the nearest measured rule: 5 and more the 8-rank one.
+// The one-shot cannot run in place, so an in-place call takes the two-shot.
+static coll_algo_t auto_form(int nranks, size_t bytes, bool in_place) {
+  if (in_place) return COLL_ALGO_TWOSHOT;
+  if (nranks == 3 && bytes <= (256u << 10)) return COLL_ALGO_ONESHOT;
+  if (nranks == 4 && bytes <= (64u << 10)) return COLL_ALGO_ONESHOT;
+  return COLL_ALGO_TWOSHOT;
+}
+
 size_t coll_all_reduce_workspace_size(int nranks, size_t count, coll_dtype_t dtype, coll_algo_t algo) {
   if (!valid_n(nranks) || !elem_size(dtype)) return 0;
   // 256-byte header (status pair at bytes 16..23), then the fp32 / int32 partials
@@ -346,13 +361,12 @@ size_t coll_all_reduce_workspace_size(int nranks, size_t count, coll_dtype_t dty
 }
 
 int coll_all_reduce_form(int nranks, size_t count, coll_dtype_t dtype, coll_algo_t algo, int aligned) {
-  (void)count;  // no form depends on the size today; the ABI keeps it for choices that will
   const int es = elem_size(dtype);
   if (!es || !valid_n(nranks)) return COLL_ERR_INVALID_ARG;
   if (algo < COLL_ALGO_AUTO || algo > COLL_ALGO_RING_CTA) return COLL_ERR_UNSUPPORTED;
   const bool vec = aligned != 0;
   switch (algo) {
-    case COLL_ALGO_AUTO: return COLL_ALGO_TWOSHOT;
+    case COLL_ALGO_AUTO: return auto_form(nranks, count * es, false);
     case COLL_ALGO_RING: return ring_form(nranks, vec);
     case COLL_ALGO_RING_LL: return vec ? COLL_ALGO_RING_LL : COLL_ALGO_RING_STEPS;
     case COLL_ALGO_TWOSHOT_LL: return vec ? COLL_ALGO_TWOSHOT_LL : COLL_ALGO_TWOSHOT;
@@ -371,7 +385,11 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
   if (!valid_n(nranks) || !all_nonnull(send, nranks) || !all_nonnull(recv, nranks)) return COLL_ERR_INVALID_ARG;
   const size_t bytes = count * es;
   if (bytes == 0) return COLL_OK;
-  if (algo == COLL_ALGO_AUTO) algo = COLL_ALGO_TWOSHOT;
+  if (algo == COLL_ALGO_AUTO) {
+    bool in_place = false;
+    for (int r = 0; r < nranks; ++r) in_place = in_place || recv[r] == send[r];
+    algo = auto_form(nranks, bytes, in_place);
+  }
   if (!outputs_disjoint(recv, nranks, bytes)) return COLL_ERR_ALIAS;
   for (int q = 0; q < nranks; ++q)
     for (int r = 0; r < nranks; ++r)

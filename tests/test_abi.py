@@ -65,6 +65,21 @@ def test_binding_constants_match_header():
         assert getattr(M, py) == _header_value(c), py
 
 
+# AUTO's measured crossovers (bytes per rank): (ranks, last bytes of the one-shot or None)
+AUTO_ONESHOT_UP_TO = {2: None, 3: 256 << 10, 4: 64 << 10, 5: None, 8: None, 16: None}
+
+
+def test_auto_form_follows_the_measured_crossovers():
+    L = M.lib()
+    for n, last in AUTO_ONESHOT_UP_TO.items():
+        for dt, es in ((M.BF16, 2), (M.FP32, 4), (M.INT32, 4)):
+            for nbytes in (16, 1 << 10, 64 << 10, 256 << 10, 1 << 20, 256 << 20):
+                for b in (nbytes - es, nbytes, nbytes + es):
+                    want = M.ONESHOT if last is not None and b <= last else M.TWOSHOT
+                    for aligned in (0, 1):
+                        assert L.coll_all_reduce_form(n, b // es, dt, M.ALGO_AUTO, aligned) == want, (n, b, dt)
+
+
 def test_version_and_strerror():
     assert M.coll_version() == 10000
     for code in (0, -1, -2, -3, -4, -5):
