@@ -7,10 +7,12 @@
 //
 // LL:    one thread per 16-byte group = two lines; a thread of pack reads 16
 //        message bytes and writes 32 packet bytes.
-// LL128: eight threads per 128-byte line, thread j owning packet bytes
-//        [16j, 16j+16); thread 7's chunk carries 8 data bytes and the flag.
-//        Message offsets 120L + 16j are only 8-byte aligned, so message-side
-//        accesses are 8 bytes wide, packet-side ones 16.
+// LL128: a warp per group of 4 lines (480 message bytes, 512 packet bytes)
+//        when the message is 16-byte aligned, rearranged in shared memory so
+//        that both sides move 16-byte units; otherwise eight threads per
+//        128-byte line, thread j owning packet bytes [16j, 16j+16) (thread
+//        7's chunk carries 8 data bytes and the flag), message-side accesses
+//        8 bytes wide since offsets 120L + 16j are only 8-byte aligned.
 #include "bulk.cuh"
 #include "common.cuh"
 #include "internal.h"
@@ -111,15 +113,54 @@ __global__ void __launch_bounds__(kThreads) k_ll_unpack(const uint8_t* __restric
 
 // --------------------------------------------------------------- LL128 ----
 
+// A group of 4 lines carries 480 message bytes, a whole number of 16-byte
+// units: when the message is 16-byte aligned, a warp moves a group at a
+// time with 16-byte accesses on both sides (30 lanes on the message side, 32
+// on the packet side), rearranging the bytes in its own 480-byte
+// shared-memory buffer; two groups per warp per pass keep two loads in
+// flight.  Lines after the last whole group take the 8-threads-per-line code.
+constexpr int kGroupBytes = 480;  // 4 lines of payload
+constexpr int kWarps = kThreads / 32;
+
 __global__ void __launch_bounds__(kThreads) k_ll128_pack(const uint8_t* __restrict__ src, uint8_t* __restrict__ packed,
-                                                         uint64_t bytes, uint64_t step, int src_al8) {
+                                                         uint64_t bytes, uint64_t step, int src_al8, int src_al16) {
+  __shared__ __align__(16) uint8_t stage[kWarps][2][kGroupBytes];
   pdl_wait();
   pdl_trigger();
   const uint64_t nlines = (bytes + 119) / 120;
-  const uint64_t nthreads = nlines * 8;
+  uint64_t first = 0;  // first line of the 8-threads-per-line part
+  if (src_al16) {
+    const uint64_t groups = bytes / kGroupBytes;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int l = lane >> 3, j = lane & 7;  // line of the group, 16-byte chunk of the line
+    const uint64_t ws = static_cast<uint64_t>(gridDim.x) * kWarps;
+    const uint2 flag = make_uint2(static_cast<uint32_t>(step), static_cast<uint32_t>(step >> 32));
+    for (uint64_t g = static_cast<uint64_t>(blockIdx.x) * kWarps + warp; g < groups; g += 2 * ws) {
+      const bool two = g + ws < groups;
+      uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
+      if (lane < 30) {
+        x0 = ld16(src + kGroupBytes * g + 16 * lane);
+        if (two) x1 = ld16(src + kGroupBytes * (g + ws) + 16 * lane);
+        *reinterpret_cast<uint4*>(stage[warp][0] + 16 * lane) = x0;
+        *reinterpret_cast<uint4*>(stage[warp][1] + 16 * lane) = x1;
+      }
+      __syncwarp();
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (h == 1 && !two) break;
+        const uint8_t* b = stage[warp][h] + 120 * l + 16 * j;
+        const uint2 lo = *reinterpret_cast<const uint2*>(b);
+        const uint2 hi = j < 7 ? *reinterpret_cast<const uint2*>(b + 8) : flag;
+        st16(packed + 512 * (g + h * ws) + 16 * lane, make_uint4(lo.x, lo.y, hi.x, hi.y));
+      }
+      __syncwarp();
+    }
+    first = 4 * groups;
+  }
+  const uint64_t nthreads = (nlines - first) * 8;
   const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
   for (uint64_t t = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < nthreads; t += stride) {
-    const uint64_t L = t >> 3;
+    const uint64_t L = first + (t >> 3);
     const int j = static_cast<int>(t & 7);
     const uint64_t off = 120 * L + 16 * j;
     const uint2 lo = load8_any(src, off, bytes, src_al8);
@@ -131,15 +172,45 @@ __global__ void __launch_bounds__(kThreads) k_ll128_pack(const uint8_t* __restri
 }
 
 __global__ void __launch_bounds__(kThreads) k_ll128_unpack(const uint8_t* __restrict__ packed, uint8_t* __restrict__ dst,
-                                                           uint64_t bytes, uint64_t step, int dst_al8, int* status) {
+                                                           uint64_t bytes, uint64_t step, int dst_al8, int dst_al16,
+                                                           int* status) {
+  __shared__ __align__(16) uint8_t stage[kWarps][2][kGroupBytes];
   pdl_wait();
   pdl_trigger();
   const uint64_t nlines = (bytes + 119) / 120;
-  const uint64_t nthreads = nlines * 8;
-  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
   int bad = 0;
+  uint64_t first = 0;
+  if (dst_al16) {
+    const uint64_t groups = bytes / kGroupBytes;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int l = lane >> 3, j = lane & 7;
+    const uint64_t ws = static_cast<uint64_t>(gridDim.x) * kWarps;
+    for (uint64_t g = static_cast<uint64_t>(blockIdx.x) * kWarps + warp; g < groups; g += 2 * ws) {
+      const bool two = g + ws < groups;
+      const uint4 x0 = ld16(packed + 512 * g + 16 * lane);
+      const uint4 x1 = two ? ld16(packed + 512 * (g + ws) + 16 * lane) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (h == 1 && !two) break;
+        const uint4 x = h == 0 ? x0 : x1;
+        uint8_t* b = stage[warp][h] + 120 * l + 16 * j;
+        *reinterpret_cast<uint2*>(b) = make_uint2(x.x, x.y);
+        if (j < 7) *reinterpret_cast<uint2*>(b + 8) = make_uint2(x.z, x.w);
+        else bad += (static_cast<uint64_t>(x.z) | (static_cast<uint64_t>(x.w) << 32)) != step;
+      }
+      __syncwarp();
+      if (lane < 30) {
+        st16(dst + kGroupBytes * g + 16 * lane, *reinterpret_cast<const uint4*>(stage[warp][0] + 16 * lane));
+        if (two) st16(dst + kGroupBytes * (g + ws) + 16 * lane, *reinterpret_cast<const uint4*>(stage[warp][1] + 16 * lane));
+      }
+      __syncwarp();
+    }
+    first = 4 * groups;
+  }
+  const uint64_t nthreads = (nlines - first) * 8;
+  const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
   for (uint64_t t = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < nthreads; t += stride) {
-    const uint64_t L = t >> 3;
+    const uint64_t L = first + (t >> 3);
     const int j = static_cast<int>(t & 7);
     const uint4 x = ld16(packed + 128 * L + 16 * j);
     const uint64_t off = 120 * L + 16 * j;
@@ -259,8 +330,9 @@ int launch_ll_pack(const void* src, void* packed, size_t bytes, int proto, uint6
                                                                (reinterpret_cast<uintptr_t>(src) & 15) == 0);
   } else {
     const uint64_t nlines = (bytes + 119) / 120;
+    const int al16 = ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(packed)) & 15) == 0;
     launch_pdl(k_ll128_pack, dim3(grid_units(nlines * 8)), dim3(kThreads), 0, s, sp, pp, bytes, step,
-                                                              (reinterpret_cast<uintptr_t>(src) & 7) == 0);
+               static_cast<int>((reinterpret_cast<uintptr_t>(src) & 7) == 0), al16);
   }
   return launch_status(cudaGetLastError());
 }
@@ -276,8 +348,9 @@ int launch_ll_unpack(const void* packed, void* dst, size_t bytes, int proto, uin
                                                                  (reinterpret_cast<uintptr_t>(dst) & 15) == 0, status);
   } else {
     const uint64_t nlines = (bytes + 119) / 120;
+    const int al16 = ((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(packed)) & 15) == 0;
     launch_pdl(k_ll128_unpack, dim3(grid_units(nlines * 8)), dim3(kThreads), 0, s, pp, dp, bytes, step,
-                                                                (reinterpret_cast<uintptr_t>(dst) & 7) == 0, status);
+               static_cast<int>((reinterpret_cast<uintptr_t>(dst) & 7) == 0), al16, status);
   }
   return launch_status(cudaGetLastError());
 }
@@ -316,7 +389,7 @@ struct WordOps {
 };
 
 // LL: thread = one 8-byte line per rank when `single`, else two lines (16 B)
-template <int DT, int OP>
+template <int DT, int OP, int NR>  // NR: ranks known at compile time (0 = runtime): all NR loads issued at once
 __global__ void __launch_bounds__(kThreads) k_ar_ll(const __grid_constant__ PackedReduceArgs a) {
   pdl_wait();
   pdl_trigger();
@@ -331,15 +404,31 @@ __global__ void __launch_bounds__(kThreads) k_ar_ll(const __grid_constant__ Pack
   int bad = 0;
   for (uint64_t g = t0; g < ngroups; g += stride) {
     A acc0[kE], acc1[kE];
-    uint4 x = ld16(a.in[0] + 16 * g);
-    bad += (x.y != flag) + (x.w != flag);
-    W::widen(x.x, acc0);
-    W::widen(x.z, acc1);
-    for (int r = 1; r < a.n; ++r) {
-      x = ld16(a.in[r] + 16 * g);
+    if constexpr (NR > 0) {
+      uint4 xs[NR];
+#pragma unroll
+      for (int r = 0; r < NR; ++r) xs[r] = ld16(a.in[r] + 16 * g);
+      W::widen(xs[0].x, acc0);
+      W::widen(xs[0].z, acc1);
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        bad += (xs[r].y != flag) + (xs[r].w != flag);
+        if (r > 0) {
+          W::step(acc0, xs[r].x);
+          W::step(acc1, xs[r].z);
+        }
+      }
+    } else {
+      uint4 x = ld16(a.in[0] + 16 * g);
       bad += (x.y != flag) + (x.w != flag);
-      W::step(acc0, x.x);
-      W::step(acc1, x.z);
+      W::widen(x.x, acc0);
+      W::widen(x.z, acc1);
+      for (int r = 1; r < a.n; ++r) {
+        x = ld16(a.in[r] + 16 * g);
+        bad += (x.y != flag) + (x.w != flag);
+        W::step(acc0, x.x);
+        W::step(acc1, x.z);
+      }
     }
     const uint64_t e0 = 2 * g * kE;  // first element of line 2g
     const uint4 o = make_uint4(W::narrow(acc0, e0, count), flag, W::narrow(acc1, e0 + kE, count), flag);
@@ -363,7 +452,7 @@ __global__ void __launch_bounds__(kThreads) k_ar_ll(const __grid_constant__ Pack
 }
 
 // LL128: eight threads per line, thread j owns packet bytes [16j, 16j+16)
-template <int DT, int OP>
+template <int DT, int OP, int NR>
 __global__ void __launch_bounds__(kThreads) k_ar_ll128(const __grid_constant__ PackedReduceArgs a) {
   pdl_wait();
   pdl_trigger();
@@ -381,19 +470,30 @@ __global__ void __launch_bounds__(kThreads) k_ar_ll128(const __grid_constant__ P
     const uint64_t poff = 128 * L + 16 * j;
     const uint64_t e0 = (120 * L + 16 * j) / ES;  // first element of this chunk
     A acc[4][kE];
-    uint4 x = ld16(a.in[0] + poff);
-    if (j == 7) bad += ((static_cast<uint64_t>(x.z) | (static_cast<uint64_t>(x.w) << 32)) != a.step);
-    W::widen(x.x, acc[0]);
-    W::widen(x.y, acc[1]);
-    W::widen(x.z, acc[2]);
-    W::widen(x.w, acc[3]);
-    for (int r = 1; r < a.n; ++r) {
-      x = ld16(a.in[r] + poff);
+    auto first = [&](const uint4& x) {
+      if (j == 7) bad += ((static_cast<uint64_t>(x.z) | (static_cast<uint64_t>(x.w) << 32)) != a.step);
+      W::widen(x.x, acc[0]);
+      W::widen(x.y, acc[1]);
+      W::widen(x.z, acc[2]);
+      W::widen(x.w, acc[3]);
+    };
+    auto next = [&](const uint4& x) {
       if (j == 7) bad += ((static_cast<uint64_t>(x.z) | (static_cast<uint64_t>(x.w) << 32)) != a.step);
       W::step(acc[0], x.x);
       W::step(acc[1], x.y);
       W::step(acc[2], x.z);
       W::step(acc[3], x.w);
+    };
+    if constexpr (NR > 0) {
+      uint4 xs[NR];
+#pragma unroll
+      for (int r = 0; r < NR; ++r) xs[r] = ld16(a.in[r] + poff);
+      first(xs[0]);
+#pragma unroll
+      for (int r = 1; r < NR; ++r) next(xs[r]);
+    } else {
+      first(ld16(a.in[0] + poff));
+      for (int r = 1; r < a.n; ++r) next(ld16(a.in[r] + poff));
     }
     uint4 o;
     o.x = W::narrow(acc[0], e0, count);
@@ -412,8 +512,17 @@ __global__ void __launch_bounds__(kThreads) k_ar_ll128(const __grid_constant__ P
 
 template <int DT, int OP>
 static int launch_ar_packed_t(const PackedReduceArgs& a, int proto, cudaStream_t s) {
-  if (proto == COLL_PROTO_LL) launch_pdl(k_ar_ll<DT, OP>, dim3(grid_units(a.nlines / 2 + 1)), dim3(kThreads), 0, s, a);
-  else launch_pdl(k_ar_ll128<DT, OP>, dim3(grid_units(a.nlines * 8)), dim3(kThreads), 0, s, a);
+  // the 8-rank sum (the workloads' rank count) issues its eight loads at once
+  const bool eight = a.n == 8 && OP == COLL_SUM;
+  if (proto == COLL_PROTO_LL) {
+    const dim3 grid(grid_units(a.nlines / 2 + 1));
+    if (eight) launch_pdl(k_ar_ll<DT, OP, 8>, grid, dim3(kThreads), 0, s, a);
+    else launch_pdl(k_ar_ll<DT, OP, 0>, grid, dim3(kThreads), 0, s, a);
+  } else {
+    const dim3 grid(grid_units(a.nlines * 8));
+    if (eight) launch_pdl(k_ar_ll128<DT, OP, 8>, grid, dim3(kThreads), 0, s, a);
+    else launch_pdl(k_ar_ll128<DT, OP, 0>, grid, dim3(kThreads), 0, s, a);
+  }
   return launch_status(cudaGetLastError());
 }
 
