@@ -6,8 +6,8 @@
 // of coll_all_reduce(RING) (TP communication essay; NCCL's ring kernel named
 // in "From NCCL Ring LL to PCIe IPC AllReduce"), so the result is
 // bit-identical.  A CTA holds all N ranks, one warp each (lane t of warp r
-// plays rank r for U 16-byte vectors of every chunk of a tile of 32 x VN x U
-// elements); the CTAs of the grid walk the tiles with a stride.
+// plays rank r for one 16-byte vector of every chunk of a tile of 32 vectors
+// per chunk); the CTAs of the grid walk the tiles with a stride.
 //
 // Hops.  The ring of one tile is 2N-2 hops: N-1 reduce-scatter hops that
 // carry the fp32 / int32 partials (laid out piece-major, so that each
@@ -23,12 +23,17 @@
 //
 // Inputs are prefetched one tile ahead in registers: the vector of step k of
 // the next tile is loaded as soon as step k of this tile has used its own.
-// Tiles that are full in every chunk (those that end within the last chunk,
-// the shortest) take a path with no bounds checks; the others check each
-// vector against its chunk's end and handle a ragged vector element by
-// element.  Nothing leaves the SM but the loads of inputs and the stores of
-// outputs.
+// Chunk boundaries are whole vectors, so every vector the hops carry lies
+// wholly inside its chunk or wholly outside it -- except the one that holds
+// the message's last count mod VN elements.  Those few elements (at most 7)
+// are left out of the hops and reduced at the end by one warp in that
+// chunk's ring order with the same fp32 partials, which gives the same bits.
+// So the hot code moves only 16-byte vectors: tiles full in every chunk take
+// it with no checks, the others with one predicate per vector.  Keeping
+// element-wise code out of the per-step path matters: the steps are unrolled,
+// and inlined element loops made the loop miss in the instruction cache.
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -45,17 +50,69 @@ struct RingCtaArgs {
   int n;
 };
 
-template <int DT, int OP, int U, int MINB>
+template <int DT>
+__device__ __forceinline__ uint32_t a_to_bits(typename Elem<DT>::A x) {
+  if constexpr (std::is_same<typename Elem<DT>::A, float>::value) return __float_as_uint(x);
+  else return static_cast<uint32_t>(x);
+}
+template <int DT>
+__device__ __forceinline__ typename Elem<DT>::A a_from_bits(uint32_t w) {
+  if constexpr (std::is_same<typename Elem<DT>::A, float>::value) return __uint_as_float(w);
+  else return static_cast<typename Elem<DT>::A>(static_cast<int32_t>(w));
+}
+
+// The elements after the message's last whole vector (fewer than VN, all in
+// chunk ct): one thread each adds them in that chunk's ring order (ranks
+// ct+1, ..., n-1, 0, ..., ct) with the same partial type and the one rounding
+// at the end, and stores the result to every rank.  Each element is touched
+// by its own thread only, so in place is safe.
+template <int DT, int OP>
+__device__ void ring_tail(const RingCtaArgs& a, int lane) {
+  using S = typename Elem<DT>::S;
+  constexpr int VN = Vec<DT>::kN;
+  constexpr int ES = Elem<DT>::kSize;
+  const uint64_t vcount = a.count / VN * VN;
+  const uint64_t e = vcount + static_cast<uint64_t>(lane);
+  if (e >= a.count) return;
+  const int n = a.n;
+  const int ct = static_cast<int>(vcount / a.seg);
+  int q = ct + 1 == n ? 0 : ct + 1;
+  auto acc = widen1<DT>(*reinterpret_cast<const S*>(a.in[q] + e * ES));
+  for (int j = 1; j < n; ++j) {
+    q = q + 1 == n ? 0 : q + 1;
+    acc = op_step<OP>(acc, widen1<DT>(*reinterpret_cast<const S*>(a.in[q] + e * ES)));
+  }
+  const S o = narrow1<DT>(acc);
+  for (int r = 0; r < n; ++r) *reinterpret_cast<S*>(a.out[r] + e * ES) = o;
+}
+
+// cp.async of one 16-byte vector into shared memory: `bytes` (16 or 0) read
+// from src, the rest zero-filled; src must be a valid address either way
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int PENDING>
+__device__ __forceinline__ void cp_async_wait_n() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(PENDING) : "memory");
+}
+
+// NR: the rank count at compile time (its loops unrolled and its waits
+// immediate), or 0 for any count in 2..8.
+template <int DT, int OP, int MINB, typename OFF, int NR>
 __global__ void __launch_bounds__(kRtMaxRanks * 32, MINB) k_ring_cta(const __grid_constant__ RingCtaArgs a) {
   using A = typename Elem<DT>::A;
-  using S = typename Elem<DT>::S;
   constexpr int VN = Vec<DT>::kN;  // elements per 16-byte vector
   constexpr int NQ = VN / 4;       // 16-byte pieces of a vector's fp32 / int32 partials
   constexpr int ES = Elem<DT>::kSize;
-  constexpr uint64_t TE = 32ull * VN * U;     // elements of one chunk per tile
-  constexpr uint32_t kSlotU4 = 32 * U * NQ;   // one warp's slot, in 16-byte units
-  extern __shared__ __align__(16) uint4 hop_buf[];  // [2 buffers][N receiving warps][kSlotU4]
-  const int n = a.n;
+  constexpr uint64_t TE = 32ull * VN;    // elements of one chunk per tile
+  constexpr uint32_t kSlotU4 = 32 * NQ;  // one warp's hop slot, in 16-byte units
+  constexpr int KMAX = NR > 0 ? NR : kRtMaxRanks;
+  // [2 buffers][N receiving warps][kSlotU4] hop slots, then [N steps][32 N threads] own inputs
+  extern __shared__ __align__(16) uint4 hop_buf[];
+  const int n = NR > 0 ? NR : a.n;
   const int r = static_cast<int>(threadIdx.x >> 5);
   const int t = static_cast<int>(threadIdx.x & 31);
   pdl_wait();
@@ -66,198 +123,195 @@ __global__ void __launch_bounds__(kRtMaxRanks * 32, MINB) k_ring_cta(const __gri
   uint4* const tx = hop_buf + nxt * kSlotU4 + t;               // the next warp's slot
   const uint4* const rx = hop_buf + r * kSlotU4 + t;           // this warp's slot
   uint32_t bo = 0;                                             // buffer of the current hop
-
-  // chunk c of a rank starts c * seg elements in; reduce-scatter step k
-  // handles chunk (r - 1 - k) mod n, all-gather hop j chunk (r - j) mod n:
-  // both walk the chunks downwards, wrapping from 0 to n - 1
-  const int64_t seg_b = static_cast<int64_t>(a.seg) * ES;
-  const int64_t top_b = static_cast<int64_t>(n - 1) * seg_b;
-  const int c0 = r == 0 ? n - 1 : r - 1;
-  const int64_t off0 = static_cast<int64_t>(c0) * seg_b;
-  const int64_t off_r = static_cast<int64_t>(r) * seg_b;
-  auto down = [&](int64_t off) { return off == 0 ? top_b : off - seg_b; };
-  auto dec = [&](int c) { return c == 0 ? n - 1 : c - 1; };
-  const char* const in_r = a.in[r];
-  char* const out_r = a.out[r];
-  auto chunk_end = [&](int c) { return min(static_cast<uint64_t>(c) * a.seg + a.seg, a.count); };
-  auto vec_elem = [&](uint64_t tile, int u) { return tile * TE + static_cast<uint64_t>(u * 32 + t) * VN; };
-
-  auto to_bits = [](A x) -> uint32_t {
-    if constexpr (std::is_same<A, float>::value) return __float_as_uint(x);
-    else return static_cast<uint32_t>(x);
-  };
-  auto from_bits = [](uint32_t w) -> A {
-    if constexpr (std::is_same<A, float>::value) return __uint_as_float(w);
-    else return static_cast<A>(static_cast<int32_t>(w));
-  };
-
-  // this lane's vectors of chunk c (byte offset off) in `tile`; zero where a
-  // vector is not wholly inside the chunk or the tile is past the end
-  auto load = [&](uint64_t tile, int c, int64_t off, uint4 (&dst)[U]) {
-    const bool full = tile < a.full_tiles;
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const uint64_t e = vec_elem(tile, u);
-      dst[u] = make_uint4(0, 0, 0, 0);
-      if (tile < a.tiles && (full || static_cast<uint64_t>(c) * a.seg + e + VN <= chunk_end(c)))
-        dst[u] = ld16(in_r + off + static_cast<int64_t>(e * ES));
+  // this thread's own inputs of the current tile, one 16-byte cell per
+  // reduce-scatter step (cell k at mine[k * 32 n]); each thread writes and
+  // reads only its own cells
+  uint4* const mine = hop_buf + 2 * other + threadIdx.x;
+  const uint32_t cells = 32u * static_cast<uint32_t>(n);
+  auto wait_cells = [&]() {  // at most n - 1 of this thread's groups in flight
+    if constexpr (NR > 0) {
+      cp_async_wait_n<NR - 1>();
+    } else {
+      switch (n - 1) {
+        case 1: cp_async_wait_n<1>(); break;
+        case 2: cp_async_wait_n<2>(); break;
+        case 3: cp_async_wait_n<3>(); break;
+        case 4: cp_async_wait_n<4>(); break;
+        case 5: cp_async_wait_n<5>(); break;
+        case 6: cp_async_wait_n<6>(); break;
+        default: cp_async_wait_n<7>(); break;
+      }
     }
   };
 
-  const uint64_t G = gridDim.x;
-  uint4 pre[kRtMaxRanks][U];
+  // Reduce-scatter step k handles chunk (r - 1 - k) mod n, whose byte offset
+  // in a rank's buffer is offs[k]; the last step's chunk is r itself, and
+  // all-gather hop j's chunk r - j is offs[j - 1].
+  const OFF seg_b = static_cast<OFF>(a.seg * ES);
+  OFF offs[KMAX];
+  int chunk[KMAX];
   {
-    int c = c0;
-    int64_t off = off0;
+    int c = r == 0 ? n - 1 : r - 1;
 #pragma unroll
-    for (int k = 0; k < kRtMaxRanks; ++k) {
-      if (k < n) {
-        load(blockIdx.x, c, off, pre[k]);
-        off = down(off);
-        c = dec(c);
-      }
+    for (int k = 0; k < KMAX; ++k) {
+      chunk[k] = c;
+      offs[k] = static_cast<OFF>(c) * seg_b;
+      c = c == 0 ? n - 1 : c - 1;
     }
   }
+  // the last step's chunk (rank r's own), kept apart so that a runtime n
+  // never indexes the arrays
+  const int chunk_last = r;
+  const OFF off_last = static_cast<OFF>(r) * seg_b;
+  // the vector at element ee of chunk c lies wholly inside the chunk
+  auto inside = [&](int c, uint64_t ee) {
+    return ee + VN <= a.seg && static_cast<uint64_t>(c) * a.seg + ee + VN <= a.count;
+  };
+  const uint64_t step_b = static_cast<uint64_t>(gridDim.x) * (TE * ES);  // bytes from a tile to the next
+  const char* const in_r = a.in[r];
+  const char* in_t = in_r + (blockIdx.x * TE + static_cast<uint64_t>(t) * VN) * ES;  // this lane's vector of chunk 0
+  char* out_t = a.out[r] + (blockIdx.x * TE + static_cast<uint64_t>(t) * VN) * ES;
 
-  for (uint64_t tile = blockIdx.x; tile < a.tiles; tile += G) {
-    const uint64_t nt = tile + G;
-    const bool full = tile < a.full_tiles;
+  // copy step k's input of the tile `delta` bytes ahead into cell k: whole
+  // (mode 1), or zeros outside the chunk (mode 2); one commit group per cell,
+  // empty when there is no next tile (mode 0)
+  auto fill = [&](int k, int c, OFF off, int mode, uint64_t delta, uint64_t ee) {
+    if (mode == 1 || (mode == 2 && inside(c, ee))) cp_async16(mine + k * cells, in_t + delta + off, 16);
+    else if (mode == 2) cp_async16(mine + k * cells, in_r, 0);
+    cp_async_commit();
+  };
 
-    // own values of reduce-scatter step k (chunk c at byte offset off): the
-    // prefetched vector, or a ragged vector element by element; then the
-    // same step of the next tile is fetched into the freed registers
-    auto own = [&](uint4 (&pk)[U], int c, int64_t off, A (&v)[U][VN]) {
+  // the first tile's inputs, in reduce-scatter step order
+  {
+    const int mode = blockIdx.x < a.full_tiles ? 1 : 2;
+    const uint64_t e = blockIdx.x * TE + static_cast<uint64_t>(t) * VN;
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const uint64_t e = vec_elem(tile, u);
-        const uint64_t gi = static_cast<uint64_t>(c) * a.seg + e;
-        if (full || gi + VN <= chunk_end(c)) {
-          Vec<DT> w;
-          widen16<DT>(pk[u], w);
-#pragma unroll
-          for (int i = 0; i < VN; ++i) v[u][i] = w.v[i];
+    for (int k = 0; k < KMAX; ++k)
+      if (k < n) fill(k, chunk[k], offs[k], mode, 0, e);
+  }
+
+  for (uint64_t tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
+    const uint64_t nt = tile + gridDim.x;
+    const int next = nt >= a.tiles ? 0 : nt < a.full_tiles ? 1 : 2;  // no next tile / whole / checked
+    // Cell k is read at step k, between the barriers of hops k and k+1, and
+    // refilled with the next tile's step k after the barrier of hop k+1 (so
+    // the refill follows the read).  Every thread commits one group per cell,
+    // so the group of the cell read at any step has exactly n - 1 newer ones.
+    // fast_tag: this tile and the next are full in every chunk (the usual
+    // case): no checks and no choice of refill.
+    auto hops = [&](auto fast_tag) {
+      constexpr bool FAST = decltype(fast_tag)::value;
+      const bool full = FAST || tile < a.full_tiles;
+      const uint64_t e = tile * TE + static_cast<uint64_t>(t) * VN;
+      const uint64_t ne = e + static_cast<uint64_t>(gridDim.x) * TE;
+      auto refill = [&](int k, int c, OFF off) {
+        if constexpr (FAST) {
+          cp_async16(mine + k * cells, in_t + step_b + off, 16);
+          cp_async_commit();
         } else {
-          const uint64_t end = chunk_end(c);
-#pragma unroll
-          for (int i = 0; i < VN; ++i)
-            v[u][i] = gi + i < end ? widen1<DT>(*reinterpret_cast<const S*>(in_r + off + (e + i) * ES)) : A(0);
+          fill(k, c, off, next, step_b, ne);
         }
+      };
+      auto put = [&](int c, OFF off, const uint4& w) {  // this lane's rounded vector of chunk c (at off)
+        if (full || inside(c, e)) st16(out_t + off, w);
+      };
+      // reduce-scatter: N-1 hops of partials; step k adds chunk r-1-k of this rank
+      A p[VN];
+      {
+        wait_cells();
+        Vec<DT> w;
+        widen16<DT>(mine[0], w);
+#pragma unroll
+        for (int i = 0; i < VN; ++i) p[i] = w.v[i];
       }
-      load(nt, c, off, pk);
-    };
-    // store this lane's rounded vectors of chunk c (byte offset off)
-    auto put = [&](int c, int64_t off, const uint4 (&w)[U]) {
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const uint64_t e = vec_elem(tile, u);
-        char* const dst = out_r + off + e * ES;
-        if (full) {
-          st16(dst, w[u]);
-          continue;
-        }
-        const uint64_t gi = static_cast<uint64_t>(c) * a.seg + e;
-        const uint64_t end = chunk_end(c);
-        if (gi + VN <= end) {
-          st16(dst, w[u]);
-        } else {
-          const S* sv = reinterpret_cast<const S*>(&w[u]);
-#pragma unroll
-          for (int i = 0; i < VN; ++i)
-            if (gi + i < end) *reinterpret_cast<S*>(dst + i * ES) = sv[i];
-        }
-      }
-    };
-
-    // reduce-scatter: N-1 hops of partials; chunk r is complete at the end
-    A p[U][VN];
-    int c = c0;
-    int64_t off = off0;
-    own(pre[0], c, off, p);
-#pragma unroll
-    for (int k = 1; k < kRtMaxRanks; ++k) {
-      if (k >= n) break;
-#pragma unroll
-      for (int u = 0; u < U; ++u)
+      for (int k = 1; k < KMAX; ++k) {
+        if (k >= n) break;
 #pragma unroll
         for (int q = 0; q < NQ; ++q)
-          tx[bo + (u * NQ + q) * 32] = make_uint4(to_bits(p[u][4 * q]), to_bits(p[u][4 * q + 1]),
-                                                  to_bits(p[u][4 * q + 2]), to_bits(p[u][4 * q + 3]));
-      __syncthreads();
-#pragma unroll
-      for (int u = 0; u < U; ++u)
+          tx[bo + q * 32] = make_uint4(a_to_bits<DT>(p[4 * q]), a_to_bits<DT>(p[4 * q + 1]),
+                                       a_to_bits<DT>(p[4 * q + 2]), a_to_bits<DT>(p[4 * q + 3]));
+        __syncthreads();
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
-          const uint4 x = rx[bo + (u * NQ + q) * 32];
-          p[u][4 * q] = from_bits(x.x);
-          p[u][4 * q + 1] = from_bits(x.y);
-          p[u][4 * q + 2] = from_bits(x.z);
-          p[u][4 * q + 3] = from_bits(x.w);
+          const uint4 x = rx[bo + q * 32];
+          p[4 * q] = a_from_bits<DT>(x.x);
+          p[4 * q + 1] = a_from_bits<DT>(x.y);
+          p[4 * q + 2] = a_from_bits<DT>(x.z);
+          p[4 * q + 3] = a_from_bits<DT>(x.w);
         }
-      bo = bo == 0 ? other : 0;
-      c = dec(c);
-      off = down(off);
-      A x[U][VN];
-      own(pre[k], c, off, x);
+        bo = bo == 0 ? other : 0;
+        refill(k - 1, chunk[k - 1], offs[k - 1]);  // cell k-1 was read before this barrier
+        wait_cells();
+        Vec<DT> w;
+        widen16<DT>(mine[k * cells], w);
 #pragma unroll
-      for (int u = 0; u < U; ++u)
-#pragma unroll
-        for (int i = 0; i < VN; ++i) p[u][i] = op_step<OP>(p[u][i], x[u][i]);
-    }
-    // the one rounding, on rank r (c == r); the rounded value travels on
-    uint4 w[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
+        for (int i = 0; i < VN; ++i) p[i] = op_step<OP>(p[i], w.v[i]);
+      }
+      // the one rounding, on rank r (chunk r is offs[n-1]); the rounded value travels on
       Vec<DT> v;
 #pragma unroll
-      for (int i = 0; i < VN; ++i) v.v[i] = p[u][i];
-      w[u] = narrow16<DT>(v);
-    }
-    put(r, off_r, w);
-
-    // all-gather: N-1 hops; at hop j chunk r - j arrives, is stored and
-    // (but for the last hop) passed on
-    int cj = r;
-    int64_t offj = off_r;
-    for (int j = 1; j < n; ++j) {
+      for (int i = 0; i < VN; ++i) v.v[i] = p[i];
+      uint4 w = narrow16<DT>(v);
+      put(chunk_last, off_last, w);
+      // all-gather: N-1 hops; at hop j chunk r-j (offs[j-1]) arrives, is
+      // stored and (but for the last hop) passed on
 #pragma unroll
-      for (int u = 0; u < U; ++u) tx[bo + u * 32] = w[u];
-      __syncthreads();
-#pragma unroll
-      for (int u = 0; u < U; ++u) w[u] = rx[bo + u * 32];
-      bo = bo == 0 ? other : 0;
-      cj = dec(cj);
-      offj = down(offj);
-      put(cj, offj, w);
-    }
+      for (int j = 1; j < KMAX; ++j) {
+        if (j >= n) break;
+        tx[bo] = w;
+        __syncthreads();
+        w = rx[bo];
+        bo = bo == 0 ? other : 0;
+        if (j == 1) refill(n - 1, chunk_last, off_last);  // the last cell, read before this barrier
+        put(chunk[j - 1], offs[j - 1], w);
+      }
+    };
+    if (next == 1 && tile < a.full_tiles) hops(std::true_type{});
+    else hops(std::false_type{});
+    in_t += step_b;
+    out_t += step_b;
   }
+  cp_async_wait_n<0>();  // nothing of this CTA's is still being copied when it leaves
+  if (blockIdx.x == 0 && r == 0) ring_tail<DT, OP>(a, t);
 }
 
-template <int DT, int OP, int U, int MINB>
+template <int DT, int OP, int MINB, typename OFF, int NR>
 static int launch_ring_cta_t(RingCtaArgs a, cudaStream_t s) {
   constexpr int VN = Vec<DT>::kN;
   constexpr int NQ = VN / 4;
-  const uint64_t per_tile = 32ull * VN * U;
+  const uint64_t per_tile = 32ull * VN;
   a.tiles = std::max<uint64_t>(1, (a.seg + per_tile - 1) / per_tile);
   // the last chunk is the shortest (possibly empty): a tile is full in every
   // chunk when it is full in that one
   const uint64_t lead = static_cast<uint64_t>(a.n - 1) * a.seg;
   a.full_tiles = a.count > lead ? (a.count - lead) / per_tile : 0;
-  const size_t smem = 2ull * a.n * 32 * U * NQ * 16;
+  const size_t smem = (2ull * NQ + a.n) * a.n * 32 * 16;  // hop slots, then each thread's input cells
   static int smem_set[COLL_MAX_RANKS] = {0};  // per device ordinal: largest limit set so far
-  const int st = allow_dynamic_smem(reinterpret_cast<const void*>(k_ring_cta<DT, OP, U, MINB>), smem, smem_set);
+  const int st = allow_dynamic_smem(reinterpret_cast<const void*>(k_ring_cta<DT, OP, MINB, OFF, NR>), smem, smem_set);
   if (st != COLL_OK) return st;
   const uint64_t grid = std::min<uint64_t>(a.tiles, static_cast<uint64_t>(num_sms()) * MINB);
-  launch_pdl(k_ring_cta<DT, OP, U, MINB>, dim3(static_cast<unsigned>(grid)), dim3(32 * a.n), smem, s, a);
+  launch_pdl(k_ring_cta<DT, OP, MINB, OFF, NR>, dim3(static_cast<unsigned>(grid)), dim3(32 * a.n), smem, s, a);
   return launch_status(cudaGetLastError());
+}
+
+template <int DT, int OP>
+static int launch_ring_cta_op(const RingCtaArgs& a, cudaStream_t s) {
+  // byte offsets within one rank's buffer fit 32 bits below 4 GiB
+  const uint64_t span = static_cast<uint64_t>(a.n) * a.seg * Elem<DT>::kSize;
+  if (span >= (1ull << 32)) return launch_ring_cta_t<DT, OP, 3, uint64_t, 0>(a, s);
+  // eight ranks (the workloads' count) get the fully unrolled kernel
+  if (a.n == 8) return launch_ring_cta_t<DT, OP, 4, uint32_t, 8>(a, s);
+  return launch_ring_cta_t<DT, OP, 4, uint32_t, 0>(a, s);
 }
 
 template <int DT>
 static int launch_ring_cta_dt(const RingCtaArgs& a, coll_op_t op, cudaStream_t s) {
   switch (op) {
-    case COLL_SUM: return launch_ring_cta_t<DT, COLL_SUM, 1, 3>(a, s);
-    case COLL_MAX: return launch_ring_cta_t<DT, COLL_MAX, 1, 3>(a, s);
-    case COLL_MIN: return launch_ring_cta_t<DT, COLL_MIN, 1, 3>(a, s);
-    case COLL_PROD: return launch_ring_cta_t<DT, COLL_PROD, 1, 3>(a, s);
+    case COLL_SUM: return launch_ring_cta_op<DT, COLL_SUM>(a, s);
+    case COLL_MAX: return launch_ring_cta_op<DT, COLL_MAX>(a, s);
+    case COLL_MIN: return launch_ring_cta_op<DT, COLL_MIN>(a, s);
+    case COLL_PROD: return launch_ring_cta_op<DT, COLL_PROD>(a, s);
   }
   return COLL_ERR_UNSUPPORTED;
 }

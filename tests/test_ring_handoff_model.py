@@ -30,6 +30,12 @@ freely between barriers and checks that every read sees its own hop and that
 no store lands on a hop not yet read; with one buffer instead of two, some
 schedule breaks that.
 
+RING_CTA also stages each thread's own inputs in shared-memory cells with
+asynchronous copies, one commit group per cell: a deterministic model of one
+thread's program checks that the wait before every read leaves that cell's
+copy complete (n - 1 newer groups may still be in flight, never n), and that
+a refill never follows a read of the same cell without a barrier between.
+
 A random scheduler picks any enabled step; a receive is enabled when the
 hardware's test passes.  The checks are the claims above, and that every
 schedule finishes (no deadlock).
@@ -252,3 +258,86 @@ def test_cta_ring_double_buffer_under_random_schedules(n):
 
 def test_cta_ring_model_catches_a_single_buffer():
     assert not all(simulate_lockstep(4, tiles=2, buffers=1, seed=seed) for seed in range(200))
+
+
+def simulate_cells(n, tiles, pending_allowed):
+    """RING_CTA's own-input cells, one thread's program over `tiles` tiles.
+
+    Each thread copies every reduce-scatter step's input into its own cell
+    (cp.async, one commit group per cell) and reads cell k at step k.  The
+    prologue fills cells 0..n-1 for the first tile; in each tile, after the
+    barrier of hop k (k = 1..n-1) the thread refills cell k-1 for the next
+    tile, and after the first all-gather barrier cell n-1; before every read
+    it waits until at most `pending_allowed` groups are in flight.  Copies
+    complete in commit order, as late as the wait allows.  Returns False if a
+    read could see a cell whose copy for that (tile, step) has not completed,
+    or a refill could land before the cell's last read; True otherwise."""
+    groups = []          # (tile, cell) per committed group, in order
+    completed = 0        # groups known complete (the wait's guarantee)
+    cell_tile = {}       # cell -> tile whose data a completed group put there
+    last_read = {}       # cell -> event index of its last read
+    barrier_at = []      # event indices of barriers
+    ev = 0
+
+    def commit(tile, cell):
+        nonlocal ev
+        groups.append((tile, cell))
+        ev += 1
+
+    def wait(allowed):
+        nonlocal completed, ev
+        completed = max(completed, len(groups) - allowed)
+        for g in groups[:completed]:
+            cell_tile[g[1]] = g[0]
+        ev += 1
+
+    def read(tile, cell):
+        nonlocal ev
+        if cell_tile.get(cell) != tile:
+            return False
+        last_read[cell] = ev
+        ev += 1
+        return True
+
+    def barrier():
+        nonlocal ev
+        barrier_at.append(ev)
+        ev += 1
+
+    def refill(tile, cell):
+        # the refill must follow the cell's last read with a barrier in between
+        lr = last_read.get(cell)
+        if lr is not None and not any(lr < b for b in barrier_at):
+            return False
+        commit(tile, cell)
+        return True
+
+    for k in range(n):
+        commit(0, k)
+    for tile in range(tiles):
+        nxt = tile + 1  # a refill for a tile past the end is an empty group
+        wait(pending_allowed)
+        if not read(tile, 0):
+            return False
+        for k in range(1, n):
+            barrier()
+            if not refill(nxt, k - 1):
+                return False
+            wait(pending_allowed)
+            if not read(tile, k):
+                return False
+        for j in range(1, n):
+            barrier()
+            if j == 1 and not refill(nxt, n - 1):
+                return False
+    return True
+
+
+@pytest.mark.parametrize("n", [2, 3, 4, 5, 6, 7, 8])
+def test_cta_ring_cells_are_ready_when_read(n):
+    assert simulate_cells(n, tiles=4, pending_allowed=n - 1)
+
+
+def test_cta_ring_cell_model_catches_a_loose_wait():
+    # allowing n groups in flight lets a read see the previous tile's data
+    assert not simulate_cells(4, tiles=3, pending_allowed=4)
