@@ -121,7 +121,7 @@ def _dev(a: np.ndarray, dtype):
 
 
 FORM_NAMES = {1: "oneshot", 2: "twoshot", 4: "ring_ll", 5: "ring_cluster", 6: "ring_steps", 7: "twoshot_ll",
-              8: "ring_cta"}
+              8: "ring_cta", 9: "twoshot_ll128"}
 
 
 def tp_decode_cfg(n):
@@ -387,7 +387,7 @@ def build_ring_compare(M, oracle):
         send = [_dev(x, torch.bfloat16) for x in xs]
         for algo, aname, launches in ((M.RING_STEPS, "ring_steps", 2 * (n - 1)), (M.RING_LL, "ring_ll", 1),
                                       (M.RING_CLUSTER, "ring_cluster", 1), (M.RING_CTA, "ring_cta", 1),
-                                      (M.TWOSHOT_LL, "twoshot_ll", 1)):
+                                      (M.TWOSHOT_LL, "twoshot_ll", 1), (M.TWOSHOT_LL128, "twoshot_ll128", 1)):
             need = max(64, M.coll_all_reduce_workspace_size(n, count, torch.bfloat16, algo))
             ops.append(Op(f"all_reduce/{aname}",
                           lambda b, algo=algo: (lambda: M.coll_all_reduce(b["send"], b["recv"], algo=algo,
@@ -634,7 +634,7 @@ def build_allreduce_forms(M, oracle):
     ops = []
     forms = ((M.ONESHOT, "oneshot", None), (M.TWOSHOT, "twoshot", None), (M.RING_CTA, "ring_cta", None),
              (M.RING_CLUSTER, "ring_cluster", None), (M.TWOSHOT_LL, "twoshot_ll", 16 << 20),
-             (M.RING_LL, "ring_ll", 4 << 20))
+             (M.TWOSHOT_LL128, "twoshot_ll128", 64 << 20), (M.RING_LL, "ring_ll", 4 << 20))
     for n in FORMS_RANKS:
         for nbytes in FORMS_BYTES:
             count = nbytes // 2
@@ -658,11 +658,35 @@ def build_allreduce_forms(M, oracle):
     return ops, {"workload": "allreduce_forms_sweep", "virtual_ranks": list(FORMS_RANKS),
                  "bytes_per_rank": list(FORMS_BYTES), "dtype": "bf16",
                  "forms": ["oneshot", "twoshot", "ring_cta", "ring_cluster", "twoshot_ll <= 16 MiB",
-                           "ring_ll <= 4 MiB"]}
+                           "twoshot_ll128 <= 64 MiB", "ring_ll <= 4 MiB"]}
+
+
+def build_hbm_ceilings(M, oracle):
+    """Context for the movement kernels' fractions: what this GPU's HBM does
+    for a write-only stream (a fill), a read-only one (a sum) and a copy, on
+    4 GiB with torch's own kernels.  The collectives here mostly write far
+    more than they read (all_gather and dispatch write 8 bytes per byte read),
+    so the copy figure that the roofline uses is not their only ceiling."""
+    import torch
+    n = 1 << 30  # 4 GiB of fp32
+    a = torch.ones(n, device="cuda")
+    b = torch.empty(n, device="cuda")
+    nb = 4 * n
+    return [
+        Op("write_only_fill", lambda bf: (lambda: bf["b"].fill_(2.0)), {"b": b}, nb, 0,
+           {"op": "fill (torch)", "bytes": nb}, kernel="write_only_fill"),
+        Op("read_only_sum", lambda bf: (lambda: bf["a"].sum()), {"a": a}, nb, 0,
+           {"op": "sum (torch)", "bytes": nb}, kernel="read_only_sum"),
+        # an element-wise kernel: a captured copy_ of one dtype becomes a
+        # copy-engine transfer, which is not what the kernels here compete with
+        Op("copy", lambda bf: (lambda: torch.mul(bf["a"], 1.0, out=bf["b"])), {"a": a, "b": b}, 2 * nb, 0,
+           {"op": "copy (torch elementwise)", "bytes": 2 * nb}, kernel="copy"),
+    ], {"workload": "hbm_ceilings_4GiB", "note": "torch kernels, context only"}
 
 
 WORKLOADS = {
     "full_step": build_full_step,
+    "hbm_ceilings": build_hbm_ceilings,
     "allreduce_forms": build_allreduce_forms,
     "single_image": build_single_image,
     "ring_compare": build_ring_compare,
@@ -1436,7 +1460,7 @@ def main():
             "peak_source": f"{hbm_src} (MEASURED_PEAKS.json hbm_gbs, burst)",
             "share_of_step": round(d["time"] / total_s, 4), "traffic": traffic_for(dom, args.workload),
             "avg_call_us": round(avg_call * 1e6, 3),
-            "avg_launch_us": round(avg_call * 1e6 / launches_per_call, 3),
+            "avg_launch_us": round(avg_call * 1e6 / launches_per_call, 3) if launches_per_call else None,
             "algorithmic_bytes_per_call": round(d["bytes"] / d["calls"]),
             "note": "achieved = the op's algorithmic bytes / its device time; for a multi-launch op both are "
                     "spread evenly over its launches, so per launch the ratio is the same"}
