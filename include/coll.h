@@ -87,7 +87,8 @@ typedef enum {
   COLL_ALGO_RING_CLUSTER = 5, /* the same ring, ranks = CTAs of a cluster, hops over DSMEM */
   COLL_ALGO_RING_STEPS = 6,   /* the same ring, one stream-ordered launch per step */
   COLL_ALGO_TWOSHOT_LL = 7,   /* TWOSHOT in one launch, LL packets between ranks */
-  COLL_ALGO_RING_CTA = 8      /* the same ring, ranks = warp groups of one CTA, hops in shared memory */
+  COLL_ALGO_RING_CTA = 8,     /* the same ring, ranks = warp groups of one CTA, hops in shared memory */
+  COLL_ALGO_TWOSHOT_LL128 = 9 /* TWOSHOT in one launch, LL128 packets between ranks */
 } coll_algo_t;
 typedef enum { COLL_PROTO_SIMPLE = 0, COLL_PROTO_LL = 1, COLL_PROTO_LL128 = 2 } coll_proto_t;
 
@@ -232,6 +233,16 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    Buffers that are not
  *    16-byte aligned take the TWOSHOT kernel.  Needs N x (CTAs per SM) to
  *    fit on the GPU at once (COLL_ERR_UNSUPPORTED otherwise).
+ *  TWOSHOT_LL128 ([RLL] "Traditional LL Protocols": the [120 B data | 8 B
+ *    flag] line): TWOSHOT_LL with LL128 lines, 1.07 bytes per payload byte
+ *    instead of 2.  A warp moves 4 lines at a time; the 8 stores of a line
+ *    are not assumed to land together: its writer stores the data, fences
+ *    (gpu scope) and then the flag, and its reader polls the flag, fences,
+ *    and only then reads the data.  Bit-identical to TWOSHOT.  Workspace:
+ *    coll_all_reduce_workspace_size() bytes, 256-byte aligned, zero-filled
+ *    once, one call at a time, the same header (call counter, status pair,
+ *    COLL_TWOSHOT_LL_CALLS_PER_FILL calls per fill).  Unaligned buffers take
+ *    the TWOSHOT kernel.
  *  AUTO picks the form measured fastest on B200 for N and the bytes per rank
  *    (1 KiB .. 256 MiB per rank at 2, 3, 4 and 8 ranks, every one-launch
  *    form): ONESHOT for N == 3 up to 256 KiB and for N == 4 up to 64 KiB
@@ -245,8 +256,8 @@ COLL_API int coll_all_reduce(const void* const* send, void* const* recv, int nra
 COLL_API size_t coll_all_reduce_workspace_size(int nranks, size_t count, coll_dtype_t dtype,
                                       coll_algo_t algo);
 /* The form coll_all_reduce() runs for these arguments when nranks >= 2 and
- * count >= 1: ONESHOT, TWOSHOT, TWOSHOT_LL, RING_LL, RING_CLUSTER, RING_CTA
- * or RING_STEPS (AUTO and RING resolved, AUTO for a call that is not in
+ * count >= 1: ONESHOT, TWOSHOT, TWOSHOT_LL, TWOSHOT_LL128, RING_LL,
+ * RING_CLUSTER, RING_CTA or RING_STEPS (AUTO and RING resolved, AUTO for a call that is not in
  * place; `aligned` != 0 when every buffer is 16-byte aligned).  RING_STEPS launches 2(N-1) kernels, the others one.
  * Returns a negative COLL_ERR_* for an invalid rank count, dtype or algo.
  * Library introspection; the sources have no counterpart. */

@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libmvrcoll.so")
 
 BF16, FP16, FP32, INT32 = 0, 1, 2, 3
 SUM, MAX, MIN, PROD = 0, 1, 2, 3
-ALGO_AUTO, ONESHOT, TWOSHOT, RING, RING_LL, RING_CLUSTER, RING_STEPS, TWOSHOT_LL, RING_CTA = 0, 1, 2, 3, 4, 5, 6, 7, 8
+ALGO_AUTO, ONESHOT, TWOSHOT, RING, RING_LL, RING_CLUSTER, RING_STEPS, TWOSHOT_LL, RING_CTA, TWOSHOT_LL128 = range(10)
 SIMPLE, LL, LL128 = 0, 1, 2
 DEV_OK, DEV_FLAG_MISMATCH, DEV_TIMEOUT, DEV_SPLIT_OVERFLOW, DEV_BAD_ROUTE, DEV_EPOCH_WRAP = 0, 1, 2, 3, 4, 5
 RING_LL_CALLS_PER_FILL, TWOSHOT_LL_CALLS_PER_FILL = 1 << 25, 1 << 30  # calls one zero-filled workspace serves
@@ -33,7 +33,7 @@ _ESIZE = {BF16: 2, FP16: 2, FP32: 4, INT32: 4}
 OPS = {"sum": SUM, "max": MAX, "min": MIN, "prod": PROD}
 ALGOS = {"auto": ALGO_AUTO, "oneshot": ONESHOT, "twoshot": TWOSHOT, "ring": RING, "ring_ll": RING_LL,
          "ring_cluster": RING_CLUSTER, "ring_steps": RING_STEPS, "twoshot_ll": TWOSHOT_LL,
-         "ring_cta": RING_CTA}
+         "ring_cta": RING_CTA, "twoshot_ll128": TWOSHOT_LL128}
 PROTOS = {"simple": SIMPLE, "ll": LL, "ll128": LL128}
 
 
@@ -242,8 +242,9 @@ def coll_all_reduce_workspace_size(nranks: int, count: int, dtype: torch.dtype, 
 
 
 def coll_all_reduce_form(nranks: int, count: int, dtype: torch.dtype, algo=TWOSHOT, aligned: bool = True) -> int:
-    """The form coll_all_reduce() runs: ONESHOT, TWOSHOT, TWOSHOT_LL, RING_LL,
-    RING_CLUSTER, RING_CTA (one launch each) or RING_STEPS (2(N-1) launches)."""
+    """The form coll_all_reduce() runs: ONESHOT, TWOSHOT, TWOSHOT_LL, TWOSHOT_LL128,
+    RING_LL, RING_CLUSTER, RING_CTA (one launch each) or RING_STEPS (2(N-1)
+    launches)."""
     algo = ALGOS[algo] if isinstance(algo, str) else int(algo)
     rc = int(lib().coll_all_reduce_form(nranks, count, _DTYPES[dtype], algo, 1 if aligned else 0))
     if rc < 0:
@@ -253,9 +254,9 @@ def coll_all_reduce_form(nranks: int, count: int, dtype: torch.dtype, algo=TWOSH
 
 def coll_all_reduce(send, recv, op="sum", algo=TWOSHOT, workspace: torch.Tensor | None = None, stream=None):
     """``workspace``: a CUDA tensor passed through to the library when given.
-    RING, RING_STEPS, RING_LL and TWOSHOT_LL need one of at least
+    RING, RING_STEPS, RING_LL, TWOSHOT_LL and TWOSHOT_LL128 need one of at least
     coll_all_reduce_workspace_size() bytes (zero-filled before its first
-    RING_LL / TWOSHOT_LL use) and get a zeroed one allocated here when it
+    RING_LL / TWOSHOT_LL / TWOSHOT_LL128 use) and get a zeroed one allocated here when it
     is omitted;
     RING_CLUSTER uses one, when given, for its status pair and its fallback
     to RING_STEPS; RING_CTA only for that fallback."""
@@ -268,7 +269,7 @@ def coll_all_reduce(send, recv, op="sum", algo=TWOSHOT, workspace: torch.Tensor 
     if _same_numel(recv, "recv") != n:
         raise ValueError("send and recv sizes differ")
     ws_ptr, ws_bytes = None, 0
-    if workspace is None and algo in (RING, RING_LL, RING_STEPS, TWOSHOT_LL):
+    if workspace is None and algo in (RING, RING_LL, RING_STEPS, TWOSHOT_LL, TWOSHOT_LL128):
         need = coll_all_reduce_workspace_size(len(send), n, send[0].dtype, algo)
         workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=send[0].device)
     if workspace is not None:

@@ -357,19 +357,21 @@ size_t coll_all_reduce_workspace_size(int nranks, size_t count, coll_dtype_t dty
   if (algo == COLL_ALGO_RING || algo == COLL_ALGO_RING_STEPS) return 256 + ring_ws(count);
   if (algo == COLL_ALGO_RING_LL) return std::max(ring_ll_workspace(nranks, count, elem_size(dtype)), 256 + ring_ws(count));
   if (algo == COLL_ALGO_TWOSHOT_LL) return twoshot_ll_workspace(nranks, count, elem_size(dtype));
+  if (algo == COLL_ALGO_TWOSHOT_LL128) return twoshot_ll128_workspace(nranks, count, elem_size(dtype));
   return 0;
 }
 
 int coll_all_reduce_form(int nranks, size_t count, coll_dtype_t dtype, coll_algo_t algo, int aligned) {
   const int es = elem_size(dtype);
   if (!es || !valid_n(nranks)) return COLL_ERR_INVALID_ARG;
-  if (algo < COLL_ALGO_AUTO || algo > COLL_ALGO_RING_CTA) return COLL_ERR_UNSUPPORTED;
+  if (algo < COLL_ALGO_AUTO || algo > COLL_ALGO_TWOSHOT_LL128) return COLL_ERR_UNSUPPORTED;
   const bool vec = aligned != 0;
   switch (algo) {
     case COLL_ALGO_AUTO: return auto_form(nranks, count * es, false);
     case COLL_ALGO_RING: return ring_form(nranks, vec);
     case COLL_ALGO_RING_LL: return vec ? COLL_ALGO_RING_LL : COLL_ALGO_RING_STEPS;
     case COLL_ALGO_TWOSHOT_LL: return vec ? COLL_ALGO_TWOSHOT_LL : COLL_ALGO_TWOSHOT;
+    case COLL_ALGO_TWOSHOT_LL128: return vec ? COLL_ALGO_TWOSHOT_LL128 : COLL_ALGO_TWOSHOT;
     case COLL_ALGO_RING_CLUSTER:
       return vec && ring_cluster_supported(nranks) ? COLL_ALGO_RING_CLUSTER : COLL_ALGO_RING_STEPS;
     case COLL_ALGO_RING_CTA: return vec && ring_cta_supported(nranks) ? COLL_ALGO_RING_CTA : COLL_ALGO_RING_STEPS;
@@ -381,7 +383,7 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
                     coll_op_t op, coll_algo_t algo, void* workspace, size_t workspace_bytes, coll_stream_t stream) {
   const int es = elem_size(dtype);
   if (!es) return COLL_ERR_UNSUPPORTED;
-  if (!valid_op(op) || algo < COLL_ALGO_AUTO || algo > COLL_ALGO_RING_CTA) return COLL_ERR_UNSUPPORTED;
+  if (!valid_op(op) || algo < COLL_ALGO_AUTO || algo > COLL_ALGO_TWOSHOT_LL128) return COLL_ERR_UNSUPPORTED;
   if (!valid_n(nranks) || !all_nonnull(send, nranks) || !all_nonnull(recv, nranks)) return COLL_ERR_INVALID_ARG;
   const size_t bytes = count * es;
   if (bytes == 0) return COLL_OK;
@@ -396,8 +398,9 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
       if (overlap(recv[q], bytes, send[r], bytes) && !(q == r && recv[q] == send[r] && algo != COLL_ALGO_ONESHOT))
         return COLL_ERR_ALIAS;
   const bool ws_needed = algo == COLL_ALGO_RING || algo == COLL_ALGO_RING_LL || algo == COLL_ALGO_RING_STEPS ||
-                         algo == COLL_ALGO_TWOSHOT_LL;
-  const bool packet_ws = algo == COLL_ALGO_RING_LL || algo == COLL_ALGO_TWOSHOT_LL;  // LL FIFOs: 256-byte aligned
+                         algo == COLL_ALGO_TWOSHOT_LL || algo == COLL_ALGO_TWOSHOT_LL128;
+  const bool packet_ws = algo == COLL_ALGO_RING_LL || algo == COLL_ALGO_TWOSHOT_LL ||
+                         algo == COLL_ALGO_TWOSHOT_LL128;  // LL FIFOs: 256-byte aligned
   if (ws_needed && nranks > 1) {
     const size_t need = coll_all_reduce_workspace_size(nranks, count, dtype, algo);
     if (workspace == nullptr || workspace_bytes < need || (U(workspace) & (packet_ws ? 255 : 15)))
@@ -447,6 +450,19 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
       return launch_ring_ll(in, out, nranks, count, dtype, op, workspace, status, S(stream));
     }
     algo = COLL_ALGO_RING_STEPS;  // unaligned buffers: the stream-ordered steps, partials after the header
+  }
+  if (algo == COLL_ALGO_TWOSHOT_LL128) {
+    if (vec) {
+      const char* in[COLL_MAX_RANKS];
+      char* out[COLL_MAX_RANKS];
+      for (int r = 0; r < nranks; ++r) {
+        in[r] = static_cast<const char*>(send[r]);
+        out[r] = static_cast<char*>(recv[r]);
+      }
+      int* status = reinterpret_cast<int*>(static_cast<char*>(workspace) + 16);
+      return launch_twoshot_ll128(in, out, nranks, count, dtype, op, workspace, status, S(stream));
+    }
+    algo = COLL_ALGO_TWOSHOT;  // unaligned buffers: the plain two-shot kernel, the same result
   }
   if (algo == COLL_ALGO_TWOSHOT_LL) {
     if (vec) {

@@ -55,6 +55,9 @@ int launch_ring_steps(const char* const* in, char* const* out, int n, size_t cou
 size_t twoshot_ll_workspace(int n, size_t count, int es);
 int launch_twoshot_ll(const char* const* in, char* const* out, int n, size_t count, coll_dtype_t dt, coll_op_t op,
                       void* workspace, int* status, cudaStream_t s);
+size_t twoshot_ll128_workspace(int n, size_t count, int es);
+int launch_twoshot_ll128(const char* const* in, char* const* out, int n, size_t count, coll_dtype_t dt,
+                         coll_op_t op, void* workspace, int* status, cudaStream_t s);
 size_t ring_ll_workspace(int n, size_t count, int es);
 int launch_ring_ll(const char* const* in, char* const* out, int n, size_t count, coll_dtype_t dt, coll_op_t op,
                    void* workspace, int* status, cudaStream_t s);

@@ -99,6 +99,9 @@ def test_workspace_sizes():
     assert L.coll_all_reduce_workspace_size(8, 1000, M.BF16, M.TWOSHOT) == 0
     ws = L.coll_all_reduce_workspace_size(8, 1000, M.BF16, M.RING)
     assert ws >= 4000 and ws % 256 == 0
+    # TWOSHOT_LL128: header + two FIFOs of N x N segments in groups of 4 lines (480 payload B in 512 B)
+    seg = -(-(-(-1000 // 8)) // 8) * 8
+    assert L.coll_all_reduce_workspace_size(8, 1000, M.BF16, M.TWOSHOT_LL128) == 256 + 2 * 64 * -(-seg * 2 // 480) * 512
     assert L.coll_moe_route_workspace_size(8, 4096, 8, 256) > 0
     assert L.coll_moe_route_workspace_size(8, 4096, 8, 250) == 0  # experts not divisible by ranks
     assert L.coll_moe_route_workspace_size(8, 4096, 8, 2048) == 0  # too many experts
@@ -127,7 +130,9 @@ def test_all_reduce_form():
     assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING_CTA, 1) == M.RING_CTA
     assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING_CTA, 0) == M.RING_STEPS
     assert L.coll_all_reduce_form(9, 1000, M.BF16, M.RING_CTA, 1) == M.RING_STEPS
-    assert L.coll_all_reduce_form(8, 1000, M.BF16, 9, 1) == -2
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, M.TWOSHOT_LL128, 1) == M.TWOSHOT_LL128
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, M.TWOSHOT_LL128, 0) == M.TWOSHOT
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, 10, 1) == -2
     # RING and RING_STEPS: a 256-byte header, then 4 bytes of partial per element
     for algo in (M.RING, M.RING_STEPS):
         assert L.coll_all_reduce_workspace_size(8, 1000, M.BF16, algo) == 256 + 4096
@@ -160,7 +165,7 @@ def test_invalid_arguments_rejected_on_host():
     # unsupported dtype / op / algo
     assert L.coll_all_reduce(p, q, 4, 16, 9, M.SUM, M.TWOSHOT, None, 0, None) == -2
     assert L.coll_all_reduce(p, q, 4, 16, M.BF16, 9, M.TWOSHOT, None, 0, None) == -2
-    assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, 9, None, 0, None) == -2
+    assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, 10, None, 0, None) == -2
     assert L.coll_moe_combine(p, p, p, p, q, 4, 8, 2, 8, 16, M.INT32, 100, None, None) == -2
     # ring without workspace
     assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, M.RING, None, 0, None) == -5

@@ -1,5 +1,5 @@
-"""GPU: the call counter of the one-launch LL all-reduce forms (RING_LL,
-TWOSHOT_LL) cannot wrap silently.
+"""GPU: the call counter of the one-launch packet all-reduce forms (RING_LL,
+TWOSHOT_LL, TWOSHOT_LL128) cannot wrap silently.
 
 A line's flag carries the workspace's call counter in its upper bits (25 of
 them for RING_LL, 30 for TWOSHOT_LL), so after that many calls the flags
@@ -24,10 +24,11 @@ from gpu_util import from_dev, need_gpu, to_dev
 pytestmark = pytest.mark.gpu
 
 FORMS = [(M.RING_LL, M.RING_LL_CALLS_PER_FILL, oracle.all_reduce_ring),
-         (M.TWOSHOT_LL, M.TWOSHOT_LL_CALLS_PER_FILL, oracle.all_reduce_two_shot)]
+         (M.TWOSHOT_LL, M.TWOSHOT_LL_CALLS_PER_FILL, oracle.all_reduce_two_shot),
+         (M.TWOSHOT_LL128, M.TWOSHOT_LL_CALLS_PER_FILL, oracle.all_reduce_two_shot)]
 
 
-@pytest.mark.parametrize("algo,limit,ref", FORMS, ids=["ring_ll", "twoshot_ll"])
+@pytest.mark.parametrize("algo,limit,ref", FORMS, ids=["ring_ll", "twoshot_ll", "twoshot_ll128"])
 @pytest.mark.parametrize("n,count", [(4, 5000), (8, 65536 + 24)])
 def test_counter_stops_at_its_limit(algo, limit, ref, n, count):
     need_gpu()
