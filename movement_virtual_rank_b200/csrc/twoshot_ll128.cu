@@ -21,9 +21,9 @@
 // receiver trusts a 128-byte line once its flag is current, which relies on
 // the line arriving whole; on one GPU nothing makes the 8 lanes' stores of a
 // line land together, so the order is made explicit: every lane stores its
-// data, the warp synchronises, the flag lane fences (gpu scope) and only
-// then stores the flag; a reader's flag lanes poll the flags, fence, the
-// warp synchronises, and only then do the lanes read their data.  An owner
+// data, the warp synchronises, the flag lane fences (fence.acq_rel.gpu) and
+// only then stores the flag; a reader's flag lanes poll the flags, fence,
+// the warp synchronises, and only then do the lanes read their data.  An owner
 // writing one group to every rank stores all the data, fences once and then
 // stores all the flags; reading one group from every rank, it polls all the
 // flags, fences once and then reads all the data.  Message
@@ -67,9 +67,14 @@ __device__ __forceinline__ void t128_st16(char* p, const uint4& v) {
 __device__ __forceinline__ void t128_st8(char* p, uint32_t x, uint32_t y) {
   asm volatile("st.volatile.global.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(x), "r"(y) : "memory");
 }
+// flags: strong (relaxed, gpu scope) stores and loads, ordered against the
+// data by fence.acq_rel.gpu on the flag lane (the release and acquire
+// patterns of the PTX memory model; a warp barrier carries the order to and
+// from the lanes that move the data)
 __device__ __forceinline__ void t128_st64(char* p, uint64_t v) {
-  asm volatile("st.volatile.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
+__device__ __forceinline__ void t128_fence() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ uint4 t128_ld16(const char* p) {
   uint4 v;
   asm volatile("ld.volatile.global.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -85,7 +90,7 @@ __device__ __forceinline__ uint2 t128_ld8(const char* p) {
 }
 __device__ __forceinline__ uint64_t t128_ld64(const char* p) {
   uint64_t v;
-  asm volatile("ld.volatile.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
 __device__ __forceinline__ uint32_t t128_ld32(const uint32_t* p) {
@@ -136,7 +141,7 @@ __global__ void __launch_bounds__(kT128Threads) k_twoshot_ll128(const __grid_con
     else t128_st8(p, v.x, v.y);
     __syncwarp();
     if (j == 7) {
-      __threadfence();
+      t128_fence();
       t128_st64(p + 8, flag);
     }
   };
@@ -174,7 +179,7 @@ __global__ void __launch_bounds__(kT128Threads) k_twoshot_ll128(const __grid_con
     return make_uint4(d.x, d.y, 0, 0);
   };
   auto acquire = [&]() {  // after the flags: their writers' data is visible to the whole warp
-    __threadfence();
+    if (j == 7) t128_fence();
     __syncwarp();
   };
 
@@ -238,7 +243,7 @@ __global__ void __launch_bounds__(kT128Threads) k_twoshot_ll128(const __grid_con
     }
     __syncwarp();
     if (j == 7) {
-      __threadfence();
+      t128_fence();
       for (int q = 0; q < n; ++q)
         t128_st64(a.fifo_ag + ((static_cast<uint64_t>(q) * n + r) * a.gps + gi) * kGroupLines + 128 * l + 120, flag_ag);
     }
