@@ -121,7 +121,7 @@ def _dev(a: np.ndarray, dtype):
 
 
 FORM_NAMES = {1: "oneshot", 2: "twoshot", 4: "ring_ll", 5: "ring_cluster", 6: "ring_steps", 7: "twoshot_ll",
-              8: "ring_cta", 9: "twoshot_ll128"}
+              8: "ring_cta", 9: "twoshot_ll128", 10: "ring_lane"}
 
 
 def tp_decode_cfg(n):
@@ -374,8 +374,9 @@ def build_ring_compare(M, oracle):
     cooperative launch with LL packets between ranks (RING_LL) and as one
     launch of 8-CTA clusters with the hops over distributed shared memory
     (RING_CLUSTER) and as one launch whose CTAs hold all 8 ranks as warp
-    groups, the hops in shared memory (RING_CTA); the two-shot with LL packets fused into one cooperative
-    launch (TWOSHOT_LL); and the stream-ordered packet path of the LL sweep
+    groups, the hops in shared memory (RING_CTA) and as one launch whose warps hold all 8 ranks as lanes,
+    the hops by warp shuffles (RING_LANE); the two-shot with LL / LL128 packets fused into one cooperative
+    launch (TWOSHOT_LL, TWOSHOT_LL128); and the stream-ordered packet path of the LL sweep
     (per-rank LL pack, packetised two-shot, per-rank unpack)."""
     import torch
     n = 8
@@ -387,6 +388,7 @@ def build_ring_compare(M, oracle):
         send = [_dev(x, torch.bfloat16) for x in xs]
         for algo, aname, launches in ((M.RING_STEPS, "ring_steps", 2 * (n - 1)), (M.RING_LL, "ring_ll", 1),
                                       (M.RING_CLUSTER, "ring_cluster", 1), (M.RING_CTA, "ring_cta", 1),
+                                      (M.RING_LANE, "ring_lane", 1),
                                       (M.TWOSHOT_LL, "twoshot_ll", 1), (M.TWOSHOT_LL128, "twoshot_ll128", 1)):
             need = max(64, M.coll_all_reduce_workspace_size(n, count, torch.bfloat16, algo))
             ops.append(Op(f"all_reduce/{aname}",
@@ -419,7 +421,9 @@ def build_ring_compare(M, oracle):
                  "variants": ["ring_steps (launch per step)", "ring_ll (one launch, LL packets)",
                               "ring_cluster (one launch, cluster DSMEM hops)",
                               "ring_cta (one launch, ranks as warp groups, shared-memory hops)",
+                              "ring_lane (one launch, ranks as lanes, warp-shuffle hops)",
                               "twoshot_ll (one launch, LL packets, fused)",
+                              "twoshot_ll128 (one launch, LL128 packets, fused)",
                               "LL pack + packetised two-shot + unpack (stream-ordered)"]}
 
 
@@ -622,8 +626,8 @@ FORMS_BYTES = tuple(1 << k for k in range(10, 29, 2))  # 1 KiB .. 256 MiB per ra
 
 
 def build_allreduce_forms(M, oracle):
-    """Every one-launch all-reduce form (one-shot, two-shot, the CTA and
-    cluster rings, the fused LL two-shot and ring) on bf16 messages of 1 KiB
+    """Every one-launch all-reduce form (one-shot, two-shot, the lane, CTA
+    and cluster rings, the fused LL / LL128 two-shots and the LL ring) on bf16 messages of 1 KiB
     .. 256 MiB per rank at 2, 3, 4 and 8 virtual ranks: the measurements the
     AUTO choice rests on.  The LL forms move 4x the payload through L2 and
     stop at 16 MiB (two-shot) and 4 MiB (ring) per rank.  Inputs are seeded
@@ -632,7 +636,8 @@ def build_allreduce_forms(M, oracle):
     g = torch.Generator(device="cuda")
     g.manual_seed(W.SEED_BASE + 77)
     ops = []
-    forms = ((M.ONESHOT, "oneshot", None), (M.TWOSHOT, "twoshot", None), (M.RING_CTA, "ring_cta", None),
+    forms = ((M.ONESHOT, "oneshot", None), (M.TWOSHOT, "twoshot", None), (M.RING_LANE, "ring_lane", None),
+             (M.RING_CTA, "ring_cta", None),
              (M.RING_CLUSTER, "ring_cluster", None), (M.TWOSHOT_LL, "twoshot_ll", 16 << 20),
              (M.TWOSHOT_LL128, "twoshot_ll128", 64 << 20), (M.RING_LL, "ring_ll", 4 << 20))
     for n in FORMS_RANKS:
@@ -657,7 +662,7 @@ def build_allreduce_forms(M, oracle):
                               kernel=f"all_reduce/{aname}"))
     return ops, {"workload": "allreduce_forms_sweep", "virtual_ranks": list(FORMS_RANKS),
                  "bytes_per_rank": list(FORMS_BYTES), "dtype": "bf16",
-                 "forms": ["oneshot", "twoshot", "ring_cta", "ring_cluster", "twoshot_ll <= 16 MiB",
+                 "forms": ["oneshot", "twoshot", "ring_lane", "ring_cta", "ring_cluster", "twoshot_ll <= 16 MiB",
                            "twoshot_ll128 <= 64 MiB", "ring_ll <= 4 MiB"]}
 
 

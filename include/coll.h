@@ -88,7 +88,8 @@ typedef enum {
   COLL_ALGO_RING_STEPS = 6,   /* the same ring, one stream-ordered launch per step */
   COLL_ALGO_TWOSHOT_LL = 7,   /* TWOSHOT in one launch, LL packets between ranks */
   COLL_ALGO_RING_CTA = 8,     /* the same ring, ranks = warp groups of one CTA, hops in shared memory */
-  COLL_ALGO_TWOSHOT_LL128 = 9 /* TWOSHOT in one launch, LL128 packets between ranks */
+  COLL_ALGO_TWOSHOT_LL128 = 9, /* TWOSHOT in one launch, LL128 packets between ranks */
+  COLL_ALGO_RING_LANE = 10     /* the same ring, ranks = lanes of one warp, hops by warp shuffles */
 } coll_algo_t;
 typedef enum { COLL_PROTO_SIMPLE = 0, COLL_PROTO_LL = 1, COLL_PROTO_LL128 = 2 } coll_proto_t;
 
@@ -217,6 +218,15 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    the message tile by tile.  Needs 2 <= N <= 8 and 16-byte aligned
  *    buffers, with the same fallback as RING_CLUSTER; `workspace` is
  *    optional and unused (this form raises no device status).
+ *  RING_LANE: the RING schedule, chunk order and rounding (bit-identical
+ *    result) in one launch in which the N virtual ranks are N lanes of one
+ *    warp (a warp holds 32 / W such rings, W = N rounded up to a power of
+ *    two, each on its own 16-byte column of every chunk): each hop is a
+ *    warp shuffle from lane r to lane r+1, so the partials stay in
+ *    registers, no shared memory or barrier is used, and HBM sees each
+ *    input and output byte once.  Needs 2 <= N <= 8 and 16-byte aligned
+ *    buffers, with the same fallback as RING_CLUSTER; `workspace` is
+ *    optional and unused (this form raises no device status).
  *  TWOSHOT_LL ([RLL] "Traditional LL Protocols" and the "Pro5000 ?" two-shot,
  *    fused): the TWOSHOT segments and arithmetic (bit-identical result) in
  *    ONE cooperative launch.  Every rank writes each 16-byte group of its
@@ -257,7 +267,7 @@ COLL_API size_t coll_all_reduce_workspace_size(int nranks, size_t count, coll_dt
                                       coll_algo_t algo);
 /* The form coll_all_reduce() runs for these arguments when nranks >= 2 and
  * count >= 1: ONESHOT, TWOSHOT, TWOSHOT_LL, TWOSHOT_LL128, RING_LL,
- * RING_CLUSTER, RING_CTA or RING_STEPS (AUTO and RING resolved, AUTO for a call that is not in
+ * RING_CLUSTER, RING_CTA, RING_LANE or RING_STEPS (AUTO and RING resolved, AUTO for a call that is not in
  * place; `aligned` != 0 when every buffer is 16-byte aligned).  RING_STEPS launches 2(N-1) kernels, the others one.
  * Returns a negative COLL_ERR_* for an invalid rank count, dtype or algo.
  * Library introspection; the sources have no counterpart. */

@@ -22,7 +22,8 @@ LIB_PATH = os.path.join(_HERE, "libmvrcoll.so")
 
 BF16, FP16, FP32, INT32 = 0, 1, 2, 3
 SUM, MAX, MIN, PROD = 0, 1, 2, 3
-ALGO_AUTO, ONESHOT, TWOSHOT, RING, RING_LL, RING_CLUSTER, RING_STEPS, TWOSHOT_LL, RING_CTA, TWOSHOT_LL128 = range(10)
+(ALGO_AUTO, ONESHOT, TWOSHOT, RING, RING_LL, RING_CLUSTER, RING_STEPS, TWOSHOT_LL, RING_CTA, TWOSHOT_LL128,
+ RING_LANE) = range(11)
 SIMPLE, LL, LL128 = 0, 1, 2
 DEV_OK, DEV_FLAG_MISMATCH, DEV_TIMEOUT, DEV_SPLIT_OVERFLOW, DEV_BAD_ROUTE, DEV_EPOCH_WRAP = 0, 1, 2, 3, 4, 5
 RING_LL_CALLS_PER_FILL, TWOSHOT_LL_CALLS_PER_FILL = 1 << 25, 1 << 30  # calls one zero-filled workspace serves
@@ -33,7 +34,8 @@ _ESIZE = {BF16: 2, FP16: 2, FP32: 4, INT32: 4}
 OPS = {"sum": SUM, "max": MAX, "min": MIN, "prod": PROD}
 ALGOS = {"auto": ALGO_AUTO, "oneshot": ONESHOT, "twoshot": TWOSHOT, "ring": RING, "ring_ll": RING_LL,
          "ring_cluster": RING_CLUSTER, "ring_steps": RING_STEPS, "twoshot_ll": TWOSHOT_LL,
-         "ring_cta": RING_CTA, "twoshot_ll128": TWOSHOT_LL128}
+         "ring_cta": RING_CTA, "twoshot_ll128": TWOSHOT_LL128,
+         "ring_lane": RING_LANE}
 PROTOS = {"simple": SIMPLE, "ll": LL, "ll128": LL128}
 
 
@@ -243,8 +245,8 @@ def coll_all_reduce_workspace_size(nranks: int, count: int, dtype: torch.dtype, 
 
 def coll_all_reduce_form(nranks: int, count: int, dtype: torch.dtype, algo=TWOSHOT, aligned: bool = True) -> int:
     """The form coll_all_reduce() runs: ONESHOT, TWOSHOT, TWOSHOT_LL, TWOSHOT_LL128,
-    RING_LL, RING_CLUSTER, RING_CTA (one launch each) or RING_STEPS (2(N-1)
-    launches)."""
+    RING_LL, RING_CLUSTER, RING_CTA, RING_LANE (one launch each) or RING_STEPS
+    (2(N-1) launches)."""
     algo = ALGOS[algo] if isinstance(algo, str) else int(algo)
     rc = int(lib().coll_all_reduce_form(nranks, count, _DTYPES[dtype], algo, 1 if aligned else 0))
     if rc < 0:
@@ -259,7 +261,7 @@ def coll_all_reduce(send, recv, op="sum", algo=TWOSHOT, workspace: torch.Tensor 
     RING_LL / TWOSHOT_LL / TWOSHOT_LL128 use) and get a zeroed one allocated here when it
     is omitted;
     RING_CLUSTER uses one, when given, for its status pair and its fallback
-    to RING_STEPS; RING_CTA only for that fallback."""
+    to RING_STEPS; RING_CTA and RING_LANE only for that fallback."""
     algo = ALGOS[algo] if isinstance(algo, str) else int(algo)
     send = _ranks(send, "send", send[0].dtype)
     recv = _ranks(recv, "recv", send[0].dtype)

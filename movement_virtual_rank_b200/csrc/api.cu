@@ -364,7 +364,7 @@ size_t coll_all_reduce_workspace_size(int nranks, size_t count, coll_dtype_t dty
 int coll_all_reduce_form(int nranks, size_t count, coll_dtype_t dtype, coll_algo_t algo, int aligned) {
   const int es = elem_size(dtype);
   if (!es || !valid_n(nranks)) return COLL_ERR_INVALID_ARG;
-  if (algo < COLL_ALGO_AUTO || algo > COLL_ALGO_TWOSHOT_LL128) return COLL_ERR_UNSUPPORTED;
+  if (algo < COLL_ALGO_AUTO || algo > COLL_ALGO_RING_LANE) return COLL_ERR_UNSUPPORTED;
   const bool vec = aligned != 0;
   switch (algo) {
     case COLL_ALGO_AUTO: return auto_form(nranks, count * es, false);
@@ -375,6 +375,7 @@ int coll_all_reduce_form(int nranks, size_t count, coll_dtype_t dtype, coll_algo
     case COLL_ALGO_RING_CLUSTER:
       return vec && ring_cluster_supported(nranks) ? COLL_ALGO_RING_CLUSTER : COLL_ALGO_RING_STEPS;
     case COLL_ALGO_RING_CTA: return vec && ring_cta_supported(nranks) ? COLL_ALGO_RING_CTA : COLL_ALGO_RING_STEPS;
+    case COLL_ALGO_RING_LANE: return vec && ring_lane_supported(nranks) ? COLL_ALGO_RING_LANE : COLL_ALGO_RING_STEPS;
     default: return algo;
   }
 }
@@ -383,7 +384,7 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
                     coll_op_t op, coll_algo_t algo, void* workspace, size_t workspace_bytes, coll_stream_t stream) {
   const int es = elem_size(dtype);
   if (!es) return COLL_ERR_UNSUPPORTED;
-  if (!valid_op(op) || algo < COLL_ALGO_AUTO || algo > COLL_ALGO_TWOSHOT_LL128) return COLL_ERR_UNSUPPORTED;
+  if (!valid_op(op) || algo < COLL_ALGO_AUTO || algo > COLL_ALGO_RING_LANE) return COLL_ERR_UNSUPPORTED;
   if (!valid_n(nranks) || !all_nonnull(send, nranks) || !all_nonnull(recv, nranks)) return COLL_ERR_INVALID_ARG;
   const size_t bytes = count * es;
   if (bytes == 0) return COLL_OK;
@@ -414,10 +415,13 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
   for (int r = 0; r < nranks; ++r) vec = vec && al16(send[r]) && al16(recv[r]);
   const size_t seg = seg_elems(count, nranks, es);
   if (algo == COLL_ALGO_RING) algo = ring_form(nranks, vec);  // workspace checked above
-  if (algo == COLL_ALGO_RING_CLUSTER || algo == COLL_ALGO_RING_CTA) {
+  if (algo == COLL_ALGO_RING_CLUSTER || algo == COLL_ALGO_RING_CTA || algo == COLL_ALGO_RING_LANE) {
     const bool has_ws = workspace != nullptr && workspace_bytes >= 24;
     const bool cta = algo == COLL_ALGO_RING_CTA;
-    if (vec && (cta ? ring_cta_supported(nranks) : ring_cluster_supported(nranks))) {
+    const bool lane = algo == COLL_ALGO_RING_LANE;
+    if (vec && (lane  ? ring_lane_supported(nranks)
+                : cta ? ring_cta_supported(nranks)
+                      : ring_cluster_supported(nranks))) {
       if (has_ws && !al16(workspace)) return COLL_ERR_WORKSPACE;
       for (int r = 0; r < nranks && has_ws; ++r)
         if (overlap(workspace, 24, send[r], bytes) || overlap(workspace, 24, recv[r], bytes)) return COLL_ERR_ALIAS;
@@ -428,6 +432,7 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
         out[r] = static_cast<char*>(recv[r]);
       }
       int* status = has_ws ? reinterpret_cast<int*>(static_cast<char*>(workspace) + 16) : nullptr;
+      if (lane) return launch_ring_lane(in, out, nranks, count, dtype, op, S(stream));
       return cta ? launch_ring_cta(in, out, nranks, count, dtype, op, status, S(stream))
                  : launch_ring_cluster(in, out, nranks, count, dtype, op, status, S(stream));
     }

@@ -21,8 +21,9 @@
 // follows.  There is no spin-wait: a CTA-wide barrier cannot time out, and
 // the kernel waits on nothing outside its own CTA.
 //
-// Inputs are prefetched one tile ahead in registers: the vector of step k of
-// the next tile is loaded as soon as step k of this tile has used its own.
+// Inputs are staged one tile ahead in shared memory: each thread copies the
+// vector of step k of the next tile into its own 16-byte cell with cp.async
+// as soon as step k of this tile has read the cell.
 // Chunk boundaries are whole vectors, so every vector the hops carry lies
 // wholly inside its chunk or wholly outside it -- except the one that holds
 // the message's last count mod VN elements.  Those few elements (at most 7)
@@ -37,6 +38,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "ring_tail.cuh"
 
 namespace mvr {
 
@@ -59,31 +61,6 @@ template <int DT>
 __device__ __forceinline__ typename Elem<DT>::A a_from_bits(uint32_t w) {
   if constexpr (std::is_same<typename Elem<DT>::A, float>::value) return __uint_as_float(w);
   else return static_cast<typename Elem<DT>::A>(static_cast<int32_t>(w));
-}
-
-// The elements after the message's last whole vector (fewer than VN, all in
-// chunk ct): one thread each adds them in that chunk's ring order (ranks
-// ct+1, ..., n-1, 0, ..., ct) with the same partial type and the one rounding
-// at the end, and stores the result to every rank.  Each element is touched
-// by its own thread only, so in place is safe.
-template <int DT, int OP>
-__device__ void ring_tail(const RingCtaArgs& a, int lane) {
-  using S = typename Elem<DT>::S;
-  constexpr int VN = Vec<DT>::kN;
-  constexpr int ES = Elem<DT>::kSize;
-  const uint64_t vcount = a.count / VN * VN;
-  const uint64_t e = vcount + static_cast<uint64_t>(lane);
-  if (e >= a.count) return;
-  const int n = a.n;
-  const int ct = static_cast<int>(vcount / a.seg);
-  int q = ct + 1 == n ? 0 : ct + 1;
-  auto acc = widen1<DT>(*reinterpret_cast<const S*>(a.in[q] + e * ES));
-  for (int j = 1; j < n; ++j) {
-    q = q + 1 == n ? 0 : q + 1;
-    acc = op_step<OP>(acc, widen1<DT>(*reinterpret_cast<const S*>(a.in[q] + e * ES)));
-  }
-  const S o = narrow1<DT>(acc);
-  for (int r = 0; r < n; ++r) *reinterpret_cast<S*>(a.out[r] + e * ES) = o;
 }
 
 // cp.async of one 16-byte vector into shared memory: `bytes` (16 or 0) read

@@ -19,7 +19,8 @@ pytestmark = pytest.mark.gpu
 ALGOS = {M.ONESHOT: oracle.all_reduce_one_shot, M.TWOSHOT: oracle.all_reduce_two_shot,
          M.RING: oracle.all_reduce_ring, M.RING_LL: oracle.all_reduce_ring, M.RING_STEPS: oracle.all_reduce_ring,
          M.RING_CLUSTER: oracle.all_reduce_ring, M.TWOSHOT_LL: oracle.all_reduce_two_shot,
-         M.RING_CTA: oracle.all_reduce_ring}
+         M.RING_CTA: oracle.all_reduce_ring, M.RING_LANE: oracle.all_reduce_ring,
+         M.TWOSHOT_LL128: oracle.all_reduce_two_shot}
 
 
 def bits(a):
@@ -50,11 +51,11 @@ def test_fuzz_all_reduce(seed):
     in_place = algo != M.ONESHOT and bool(g.integers(0, 2))
     recv = send if in_place else [Guarded(count, dtype, offset=off * ((r + 1) % 2)) for r in range(n)]
     ws = None
-    if algo in (M.RING_CLUSTER, M.RING_CTA):  # a RING-sized workspace: the fallback for unaligned buffers or N > 8
+    if algo in (M.RING_CLUSTER, M.RING_CTA, M.RING_LANE):  # a RING-sized workspace: the fallback for unaligned buffers or N > 8
         need = M.coll_all_reduce_workspace_size(n, count, send[0].t.dtype, M.RING)
         ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
-    elif algo == M.TWOSHOT_LL:
-        need = M.coll_all_reduce_workspace_size(n, count, send[0].t.dtype, M.TWOSHOT_LL)
+    elif algo in (M.TWOSHOT_LL, M.TWOSHOT_LL128):
+        need = M.coll_all_reduce_workspace_size(n, count, send[0].t.dtype, algo)
         ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
     M.coll_all_reduce([b.t for b in send], [b.t for b in recv], op=op, algo=algo, workspace=ws)
     torch.cuda.synchronize()

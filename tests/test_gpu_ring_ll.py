@@ -128,12 +128,14 @@ def test_bounded_wait_times_out_and_context_survives():
     assert all(np.array_equal(g, w) for g, w in zip(got, want))
 
 
-# ------------------------------------------- cluster ring and CTA ring ----
+# ------------------------------------ cluster, CTA and lane rings ----
 # RING_CLUSTER (ranks = CTAs of a cluster, hops over distributed shared
-# memory) and RING_CTA (ranks = warp groups of one CTA, hops in its shared
-# memory) take the same tests.
+# memory), RING_CTA (ranks = warp groups of one CTA, hops in its shared
+# memory) and RING_LANE (ranks = lanes of one warp, hops by warp shuffles)
+# take the same tests.
 
-ONE_LAUNCH = pytest.mark.parametrize("algo", [M.RING_CLUSTER, M.RING_CTA], ids=["cluster", "cta"])
+ONE_LAUNCH = pytest.mark.parametrize("algo", [M.RING_CLUSTER, M.RING_CTA, M.RING_LANE],
+                                     ids=["cluster", "cta", "lane"])
 
 
 def run_cluster(xs, dtype, op, in_place=False, ws=None, algo=M.RING_CLUSTER):
@@ -145,7 +147,7 @@ def run_cluster(xs, dtype, op, in_place=False, ws=None, algo=M.RING_CLUSTER):
 
 
 @ONE_LAUNCH
-@pytest.mark.parametrize("n", [2, 3, 4, 5, 8])
+@pytest.mark.parametrize("n", [2, 3, 4, 5, 6, 7, 8])
 @pytest.mark.parametrize("count", [1, 9, 8 * 37 + 3, 65536 + 24, 300007])
 def test_ring_cluster_bf16_sum(algo, n, count):
     """Virtual ranks as the CTAs of a thread-block cluster, hops over
@@ -268,7 +270,7 @@ def test_ring_forms_agree(tokens, hidden):
     form = M.coll_all_reduce_form(n, count, torch.bfloat16, M.RING)
     assert form == M.RING_CTA
     want = oracle.all_reduce_ring(xs, 0, "bf16")
-    for algo in (M.RING, M.RING_STEPS, M.RING_CLUSTER, M.RING_CTA):
+    for algo in (M.RING, M.RING_STEPS, M.RING_CLUSTER, M.RING_CTA, M.RING_LANE):
         send = [to_dev(x, "bf16") for x in xs]
         recv = [torch.empty_like(t) for t in send]
         ws = torch.zeros(M.coll_all_reduce_workspace_size(n, count, torch.bfloat16, M.RING), dtype=torch.uint8,
