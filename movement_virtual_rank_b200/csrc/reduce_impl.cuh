@@ -5,8 +5,9 @@
 // Per element: acc = widen(x_0); acc = acc (op) widen(x_r) for r = 1..N-1 in
 // IEEE binary32 (no contraction: __fadd_rn / __fmul_rn); one rounding to the
 // storage type.  Each thread owns 16 bytes of every rank (8 bf16 lanes) and
-// issues all N loads before combining them, so N x 16 bytes per thread are in
-// flight; outputs are plain 16-byte stores.
+// issues its loads before combining them (all N for the rank counts compiled
+// as such, eight at a time for any other), so up to 8 x 16 bytes per thread
+// are in flight; outputs are plain 16-byte stores.
 //
 // Slices: blockIdx.x = part * nslices + slice.  For the two-shot all-reduce a
 // slice is owner s's segment ("From NCCL Ring LL to PCIe IPC AllReduce",
@@ -84,9 +85,21 @@ __global__ void __launch_bounds__(kThreads) k_reduce_vec(const __grid_constant__
 #pragma unroll
       for (int r = 1; r < NR; ++r) step16<DT, OP>(acc, x[r]);
     } else {
-      widen16<DT>(ld16(a.in[0] + byte), acc);
-#pragma unroll 4
-      for (int r = 1; r < n; ++r) step16<DT, OP>(acc, ld16(a.in[r] + byte));
+      // any rank count: loads issued eight at a time before they are
+      // combined (in rank order), so a thread waits once per eight ranks
+      constexpr int B = 8;
+      for (int r0 = 0; r0 < n; r0 += B) {
+        uint4 x[B];
+#pragma unroll
+        for (int i = 0; i < B; ++i)
+          if (r0 + i < n) x[i] = ld16(a.in[r0 + i] + byte);
+#pragma unroll
+        for (int i = 0; i < B; ++i) {
+          if (r0 + i >= n) break;
+          if (r0 + i == 0) widen16<DT>(x[0], acc);
+          else step16<DT, OP>(acc, x[i]);
+        }
+      }
     }
     const uint4 o = narrow16<DT>(acc);
     if constexpr (MODE == M_ALL) {
