@@ -82,7 +82,7 @@ typedef enum {
   COLL_ALGO_AUTO = 0,    /* the measured fastest: ONESHOT or TWOSHOT by ranks and size */
   COLL_ALGO_ONESHOT = 1, /* every rank reads all N inputs itself            */
   COLL_ALGO_TWOSHOT = 2, /* owner s reduces segment s, sends it to everyone */
-  COLL_ALGO_RING = 3,    /* 2(N-1) neighbour steps: RING_CTA, else RING_STEPS */
+  COLL_ALGO_RING = 3,    /* 2(N-1) neighbour steps: RING_LANE / RING_CTA, else RING_STEPS */
   COLL_ALGO_RING_LL = 4, /* the same ring in one launch, LL packets between ranks */
   COLL_ALGO_RING_CLUSTER = 5, /* the same ring, ranks = CTAs of a cluster, hops over DSMEM */
   COLL_ALGO_RING_STEPS = 6,   /* the same ring, one stream-ordered launch per step */
@@ -170,9 +170,11 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    c is accumulated in the order c+1, ..., N-1, 0, ..., c), and the N-1
  *    all-gather steps pass the finished chunks round.  Partials travel in
  *    fp32 (int32 for int32); the result may differ from the rank-order
- *    reduction by rounding only.  Runs as RING_CTA (one launch) when
- *    2 <= N <= 8 and every buffer is 16-byte aligned, and as RING_STEPS
- *    otherwise: the same result bit for bit.
+ *    reduction by rounding only.  When 2 <= N <= 8 and every buffer is
+ *    16-byte aligned it runs in one launch, as the form measured fastest on
+ *    B200: RING_LANE for N <= 3, for N == 4 up to 256 KiB and for N >= 5 up
+ *    to 16 KiB per rank, RING_CTA above; otherwise as RING_STEPS.  Every
+ *    form gives the same result bit for bit.
  *    coll_all_reduce_form() tells which.  `workspace`:
  *    coll_all_reduce_workspace_size() bytes, 16-byte aligned: a 256-byte
  *    header whose bytes 16..23 receive the status pair of the one-launch

@@ -329,11 +329,18 @@ int coll_reduce_scatter(const void* const* send, void* const* recv, int nranks, 
 }
 
 // ------------------------------------------------------------- AllReduce ----
-// RING runs as one launch of CTAs that each hold all ranks (RING_CTA) when
-// the buffers allow it: on B200 that measured faster than the cluster form
-// and the stream-ordered steps at every size tried (8 KB .. 32 MiB per rank)
-static coll_algo_t ring_form(int nranks, bool vec) {
-  return (vec && ring_cta_supported(nranks)) ? COLL_ALGO_RING_CTA : COLL_ALGO_RING_STEPS;
+// RING runs as the one-launch ring measured fastest on B200 for the rank
+// count and the bytes per rank (cold inputs, 1 KiB .. 256 MiB per rank at 2,
+// 3, 4 and 8 virtual ranks), when the buffers allow one: the ranks as lanes
+// of a warp (RING_LANE) at 2 and 3 ranks, at 4 ranks up to 256 KiB and at 5
+// and more up to 16 KiB; above those, where RING_LANE's per-rank 64-byte
+// accesses load the L1 data pipe, the ranks as warps of a CTA (RING_CTA).
+// The cluster form and the stream-ordered steps were slower at every size.
+// Every form gives the same bits.
+static coll_algo_t ring_form(int nranks, size_t bytes, bool vec) {
+  if (!vec || !ring_cta_supported(nranks)) return COLL_ALGO_RING_STEPS;
+  if (nranks <= 3 || (nranks == 4 && bytes <= (256u << 10)) || bytes <= (16u << 10)) return COLL_ALGO_RING_LANE;
+  return COLL_ALGO_RING_CTA;
 }
 
 // AUTO: the form measured fastest on B200 for the rank count and the bytes
@@ -368,7 +375,7 @@ int coll_all_reduce_form(int nranks, size_t count, coll_dtype_t dtype, coll_algo
   const bool vec = aligned != 0;
   switch (algo) {
     case COLL_ALGO_AUTO: return auto_form(nranks, count * es, false);
-    case COLL_ALGO_RING: return ring_form(nranks, vec);
+    case COLL_ALGO_RING: return ring_form(nranks, count * es, vec);
     case COLL_ALGO_RING_LL: return vec ? COLL_ALGO_RING_LL : COLL_ALGO_RING_STEPS;
     case COLL_ALGO_TWOSHOT_LL: return vec ? COLL_ALGO_TWOSHOT_LL : COLL_ALGO_TWOSHOT;
     case COLL_ALGO_TWOSHOT_LL128: return vec ? COLL_ALGO_TWOSHOT_LL128 : COLL_ALGO_TWOSHOT;
@@ -414,7 +421,7 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
   bool vec = true;
   for (int r = 0; r < nranks; ++r) vec = vec && al16(send[r]) && al16(recv[r]);
   const size_t seg = seg_elems(count, nranks, es);
-  if (algo == COLL_ALGO_RING) algo = ring_form(nranks, vec);  // workspace checked above
+  if (algo == COLL_ALGO_RING) algo = ring_form(nranks, bytes, vec);  // workspace checked above
   if (algo == COLL_ALGO_RING_CLUSTER || algo == COLL_ALGO_RING_CTA || algo == COLL_ALGO_RING_LANE) {
     const bool has_ws = workspace != nullptr && workspace_bytes >= 24;
     const bool cta = algo == COLL_ALGO_RING_CTA;

@@ -43,7 +43,8 @@ int main(void) {
   CHECK(coll_all_reduce_workspace_size(8, 1000, COLL_BF16, COLL_ALGO_TWOSHOT) == 0);
   CHECK(coll_all_reduce_workspace_size(8, 1000, COLL_BF16, COLL_ALGO_RING) >= 256 + 4000);
   CHECK(coll_all_reduce_form(8, 1000, COLL_BF16, COLL_ALGO_AUTO, 1) == COLL_ALGO_TWOSHOT);
-  CHECK(coll_all_reduce_form(8, 1000, COLL_BF16, COLL_ALGO_RING, 1) == COLL_ALGO_RING_CTA);
+  CHECK(coll_all_reduce_form(8, 1000, COLL_BF16, COLL_ALGO_RING, 1) == COLL_ALGO_RING_LANE);
+  CHECK(coll_all_reduce_form(8, 1 << 20, COLL_BF16, COLL_ALGO_RING, 1) == COLL_ALGO_RING_CTA);
   CHECK(coll_all_reduce_form(8, 1000, COLL_BF16, COLL_ALGO_RING, 0) == COLL_ALGO_RING_STEPS);
   CHECK(coll_all_reduce_form(9, 1000, COLL_BF16, COLL_ALGO_RING, 1) == COLL_ALGO_RING_STEPS);
   CHECK(coll_moe_route_workspace_size(8, 4096, 8, 256) > 0);

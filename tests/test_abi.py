@@ -107,15 +107,32 @@ def test_workspace_sizes():
     assert L.coll_moe_route_workspace_size(8, 4096, 8, 2048) == 0  # too many experts
 
 
+# RING's one-launch form by rank count: the largest bytes per rank at which
+# the lane ring (RING_LANE) was measured fastest (None: every size); above
+# it the CTA ring (RING_CTA)
+RING_LANE_UP_TO = {2: None, 3: None, 4: 256 << 10, 5: 16 << 10, 6: 16 << 10, 7: 16 << 10, 8: 16 << 10}
+
+
+def test_ring_form_by_ranks_and_size():
+    """RING picks RING_LANE or RING_CTA on the measured crossovers (host logic)."""
+    L = M.lib()
+    for n, up_to in RING_LANE_UP_TO.items():
+        for nbytes in (16, 1 << 10, 16 << 10, (16 << 10) + 16, 256 << 10, (256 << 10) + 16, 1 << 20, 256 << 20):
+            want = M.RING_LANE if up_to is None or nbytes <= up_to else M.RING_CTA
+            assert L.coll_all_reduce_form(n, nbytes // 2, M.BF16, M.RING, 1) == want, (n, nbytes)
+            assert L.coll_all_reduce_form(n, nbytes // 2, M.BF16, M.RING, 0) == M.RING_STEPS, (n, nbytes)
+
+
 def test_all_reduce_form():
     """Which form coll_all_reduce runs (host logic only, no device call)."""
     L = M.lib()
-    assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING, 1) == M.RING_CTA
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING, 1) == M.RING_LANE  # 2000 B per rank
     assert L.coll_all_reduce_form(8, 256 * 7168, M.BF16, M.RING, 1) == M.RING_CTA
-    assert L.coll_all_reduce_form(8, 1 << 30, M.FP32, M.RING, 1) == M.RING_CTA  # every size
+    assert L.coll_all_reduce_form(8, 1 << 30, M.FP32, M.RING, 1) == M.RING_CTA
     assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING, 0) == M.RING_STEPS  # unaligned
     assert L.coll_all_reduce_form(9, 1000, M.BF16, M.RING, 1) == M.RING_STEPS  # more ranks than a CTA holds
-    assert L.coll_all_reduce_form(2, 1000, M.BF16, M.RING, 1) == M.RING_CTA
+    assert L.coll_all_reduce_form(2, 1000, M.BF16, M.RING, 1) == M.RING_LANE
+    assert L.coll_all_reduce_form(2, 1 << 30, M.FP32, M.RING, 1) == M.RING_LANE
     assert L.coll_all_reduce_form(8, 5 << 20, M.BF16, M.RING_CLUSTER, 1) == M.RING_CLUSTER
     assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING_CLUSTER, 0) == M.RING_STEPS
     assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING_LL, 1) == M.RING_LL

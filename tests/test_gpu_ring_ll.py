@@ -261,14 +261,15 @@ def test_ring_cluster_back_to_back(algo):
 
 @pytest.mark.parametrize("tokens,hidden", [(1, 4096), (32, 7168), (160, 8192), (161, 8192), (256, 7168)])
 def test_ring_forms_agree(tokens, hidden):
-    """RING takes the one-launch CTA form for aligned buffers; every form
-    (CTA, cluster, stream-ordered steps) gives the same bits, and the
-    workspace header's status pair stays clear."""
+    """RING takes a one-launch form for aligned buffers (the lane ring up to
+    16 KiB per rank at 8 ranks, the CTA ring above); every form (lane, CTA,
+    cluster, stream-ordered steps) gives the same bits, and the workspace
+    header's status pair stays clear."""
     need_gpu()
     xs = W.tp_decode(tokens, hidden)
     n, count = len(xs), tokens * hidden
     form = M.coll_all_reduce_form(n, count, torch.bfloat16, M.RING)
-    assert form == M.RING_CTA
+    assert form == (M.RING_LANE if 2 * count <= 16 << 10 else M.RING_CTA)
     want = oracle.all_reduce_ring(xs, 0, "bf16")
     for algo in (M.RING, M.RING_STEPS, M.RING_CLUSTER, M.RING_CTA, M.RING_LANE):
         send = [to_dev(x, "bf16") for x in xs]
