@@ -220,11 +220,13 @@ def test_ring_cluster_fallbacks(algo):
 
 
 @pytest.mark.parametrize("n,count,dtype", [(2, 3_000_017, "bf16"), (5, 2_500_001, "bf16"), (8, 4_194_311, "bf16"),
-                                           (3, 2_000_003, "fp32"), (8, 1_048_583, "int32"), (7, 999_999, "fp16")])
+                                           (3, 2_000_003, "fp32"), (8, 1_048_583, "int32"), (7, 999_999, "fp16"),
+                                           (8, 3_000_000, "fp32"), (8, 2_500_002, "fp16"), (8, 5_000_011, "fp16")])
 @ONE_LAUNCH
 def test_ring_cluster_many_tiles(algo, n, count, dtype):
-    """Messages of many tiles per cluster (the clusters walk the tiles, two
-    slot sets alternating), with a ragged tail."""
+    """Messages of many tiles per CTA or cluster (the CTAs walk the tiles; at
+    8 ranks the CTA ring then prefetches its inputs into registers across
+    tile boundaries), with a ragged tail; odd counts run in place."""
     need_gpu()
     if dtype == "int32":
         g = W.rng(W.W_MISC, 0, salt=count)
@@ -232,7 +234,7 @@ def test_ring_cluster_many_tiles(algo, n, count, dtype):
     else:
         xs = W.ranks_values(W.W_MISC, n, count, dtype, "normal", salt=count % 977)
     ws = torch.zeros(64, dtype=torch.uint8, device="cuda")
-    got = run_cluster(xs, dtype, 0, in_place=(n % 2 == 1), ws=ws, algo=algo)
+    got = run_cluster(xs, dtype, 0, in_place=(count % 2 == 1), ws=ws, algo=algo)
     want = oracle.all_reduce_ring(xs, 0, dtype)
     for q in range(n):
         assert np.array_equal(bits(got[q]), bits(want[q])), q
