@@ -377,7 +377,7 @@ def build_ring_compare(M, oracle):
     groups, the hops in shared memory (RING_CTA) and as one launch whose warps hold all 8 ranks as lanes,
     the hops by warp shuffles (RING_LANE); the two-shot with LL / LL128 packets fused into one cooperative
     launch (TWOSHOT_LL, TWOSHOT_LL128); and the stream-ordered packet path of the LL sweep
-    (per-rank LL pack, packetised two-shot, per-rank unpack)."""
+    (LL pack of every rank, packetised two-shot, unpack of every rank: three launches)."""
     import torch
     n = 8
     ops = []
@@ -403,18 +403,16 @@ def build_ring_compare(M, oracle):
 
         def bind_ll(b, count=count):
             def run():
-                for r in range(n):
-                    M.coll_ll_pack(b["send"][r], b["pin"][r], M.LL, 1)
+                M.coll_ll_pack_ranks(b["send"], b["pin"], M.LL, 1)
                 M.coll_all_reduce_packed(b["pin"], b["pout"], count, torch.bfloat16, M.LL, 1)
-                for r in range(n):
-                    M.coll_ll_unpack(b["pout"][r], b["recv"][r], M.LL, 1)
+                M.coll_ll_unpack_ranks(b["pout"], b["recv"], M.LL, 1)
             return run
 
         ops.append(Op("all_reduce/ll_pack_ar_unpack", bind_ll,
                       {"send": send, "recv": [torch.empty_like(t) for t in send],
                        "pin": [torch.empty(pb, dtype=torch.uint8, device="cuda") for _ in range(n)],
                        "pout": [torch.empty(pb, dtype=torch.uint8, device="cuda") for _ in range(n)]},
-                      2 * n * S, 2 * n + 1, {"op": "all_reduce", "algo": "ll_pack_ar_unpack",
+                      2 * n * S, 3, {"op": "all_reduce", "algo": "ll_pack_ar_unpack",
                                              "shape": [tokens, hidden], "bytes_per_rank": S},
                       inputs=["send"], outputs=["recv"], kernel="all_reduce/ll_pack_ar_unpack"))
     return ops, {"workload": "ring_compare_8vr", "virtual_ranks": n, "shapes": W.tp_decode_shapes(),
@@ -424,7 +422,7 @@ def build_ring_compare(M, oracle):
                               "ring_lane (one launch, ranks as lanes, warp-shuffle hops)",
                               "twoshot_ll (one launch, LL packets, fused)",
                               "twoshot_ll128 (one launch, LL128 packets, fused)",
-                              "LL pack + packetised two-shot + unpack (stream-ordered)"]}
+                              "LL pack + packetised two-shot + unpack (stream-ordered, 3 launches)"]}
 
 
 def build_movement(M, oracle):
@@ -543,23 +541,23 @@ def _protocol_ops(M, nbytes, n=8):
         recv = [torch.empty_like(t) for t in send]
 
         def pack(b, proto=proto):
-            return lambda: [M.coll_ll_pack(b["send"][r], b["pin"][r], proto, 1) for r in range(n)]
+            return lambda: M.coll_ll_pack_ranks(b["send"], b["pin"], proto, 1)
 
         def reduce_packed(b, proto=proto):
             return lambda: M.coll_all_reduce_packed(b["pin"], b["pout"], count, torch.bfloat16, proto, 1)
 
         def unpack(b, proto=proto):
-            return lambda: [M.coll_ll_unpack(b["pout"][r], b["recv"][r], proto, 1) for r in range(n)]
+            return lambda: M.coll_ll_unpack_ranks(b["pout"], b["recv"], proto, 1)
 
         ops += [
-            Op(f"{pname}_pack/{tag}", pack, {"send": send, "pin": pin}, n * (nbytes + pb), n,
+            Op(f"{pname}_pack/{tag}", pack, {"send": send, "pin": pin}, n * (nbytes + pb), 1,
                {"op": f"{pname}_pack", "ranks": n, "bytes_per_rank": nbytes, "packed_bytes_per_rank": pb},
                inputs=["send"], kernel=f"{pname}_pack"),
             Op(f"all_reduce/{pname}/{tag}", reduce_packed, {"pin": pin, "pout": pout}, 2 * n * nbytes, 1,
                {"op": "all_reduce_packed", "proto": pname, "ranks": n, "bytes_per_rank": nbytes,
                 "line_bytes": 2 * n * pb, "note": "gbs counts payload bytes; the roofline counts line bytes"},
                kernel=f"all_reduce/{pname}", per_launch_bytes=2 * n * pb),
-            Op(f"{pname}_unpack/{tag}", unpack, {"pout": pout, "recv": recv}, n * (pb + nbytes), n,
+            Op(f"{pname}_unpack/{tag}", unpack, {"pout": pout, "recv": recv}, n * (pb + nbytes), 1,
                {"op": f"{pname}_unpack", "ranks": n, "bytes_per_rank": nbytes, "packed_bytes_per_rank": pb},
                outputs=["recv"], kernel=f"{pname}_unpack"),
         ]

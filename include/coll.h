@@ -330,6 +330,19 @@ COLL_API int coll_ll_pack(const void* src, void* packed, size_t bytes, coll_prot
 COLL_API int coll_ll_unpack(const void* packed, void* dst, size_t bytes, coll_proto_t proto,
                    uint64_t step, int* d_status, coll_stream_t stream);
 
+/* The same two codecs for the equally long messages of all N virtual ranks
+ * in one launch ([RLL] "Pro5000 ?": every rank encodes its own message
+ * before the exchange and decodes the result after it): rank r's `bytes`
+ * bytes at src[r] into packed[r], or packed[r] into dst[r].  Each result is
+ * bit-identical to the one-rank call on that rank's buffers.  No message may
+ * overlap any packet buffer, and the buffers written (packed[] for pack,
+ * dst[] for unpack) must be disjoint; every packed[r] 16-byte aligned.
+ * Unpack counts flag mismatches over all ranks into d_status[1]. */
+COLL_API int coll_ll_pack_ranks(const void* const* src, void* const* packed, int nranks, size_t bytes,
+                                coll_proto_t proto, uint64_t step, coll_stream_t stream);
+COLL_API int coll_ll_unpack_ranks(const void* const* packed, void* const* dst, int nranks, size_t bytes,
+                                  coll_proto_t proto, uint64_t step, int* d_status, coll_stream_t stream);
+
 /* Packetised AllReduce: packed_in[r] are rank r's packets (proto, `count`
  * elements of payload, flag = step).  The kernel checks every input line's
  * flag (mismatches counted as above, over all ranks), reduces the payload in

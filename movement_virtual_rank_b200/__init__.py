@@ -69,6 +69,8 @@ _SIGS = {
     "coll_packed_bytes": (_SZ, [_SZ, _I]),
     "coll_ll_pack": (_I, [_VP, _VP, _SZ, _I, _U64, _VP]),
     "coll_ll_unpack": (_I, [_VP, _VP, _SZ, _I, _U64, _VP, _VP]),
+    "coll_ll_pack_ranks": (_I, [_PP, _PP, _I, _SZ, _I, _U64, _VP]),
+    "coll_ll_unpack_ranks": (_I, [_PP, _PP, _I, _SZ, _I, _U64, _VP, _VP]),
     "coll_all_reduce_packed": (_I, [_PP, _PP, _I, _SZ, _I, _I, _I, _U64, _VP, _VP]),
     "coll_moe_route": (_I, [_PP, _I, _I, _I, _I, _VP, _VP, _VP, _PP, _VP, _VP, _SZ, _VP]),
     "coll_moe_route_dedup": (_I, [_PP, _I, _I, _I, _I, _VP, _VP, _VP, _PP, _VP, _VP, _SZ, _VP]),
@@ -392,6 +394,47 @@ def coll_ll_unpack(packed: torch.Tensor, dst: torch.Tensor, proto, step: int, st
     with torch.cuda.device(dst.device):
         _check("coll_ll_unpack", lib().coll_ll_unpack(packed.data_ptr(), dst.data_ptr(), nbytes, proto, step, st,
                                                       _stream(stream)))
+
+
+def coll_ll_pack_ranks(src, packed, proto, step: int, nbytes: int | None = None, stream=None):
+    """Encode every rank's message (``src[r]`` into ``packed[r]``) in one launch."""
+    proto = PROTOS[proto] if isinstance(proto, str) else int(proto)
+    src = _ranks(src, "src")
+    packed = _ranks(packed, "packed")
+    if len(src) != len(packed):
+        raise ValueError("src and packed must list the same ranks")
+    nbytes = _nbytes(src[0]) if nbytes is None else nbytes
+    for t in src:
+        if _nbytes(t) < nbytes:
+            raise ValueError("src buffer too small")
+    for t in packed:
+        if _nbytes(t) < coll_packed_bytes(nbytes, proto):
+            raise ValueError("packed buffer too small")
+    (ps, _ks), (pp, _kp) = _ptrs(src), _ptrs(packed)
+    with torch.cuda.device(src[0].device):
+        _check("coll_ll_pack_ranks", lib().coll_ll_pack_ranks(ps, pp, len(src), nbytes, proto, step, _stream(stream)))
+
+
+def coll_ll_unpack_ranks(packed, dst, proto, step: int, status: torch.Tensor | None = None,
+                         nbytes: int | None = None, stream=None):
+    """Decode every rank's packets (``packed[r]`` into ``dst[r]``) in one launch."""
+    proto = PROTOS[proto] if isinstance(proto, str) else int(proto)
+    packed = _ranks(packed, "packed")
+    dst = _ranks(dst, "dst")
+    if len(packed) != len(dst):
+        raise ValueError("packed and dst must list the same ranks")
+    nbytes = _nbytes(dst[0]) if nbytes is None else nbytes
+    for t in dst:
+        if _nbytes(t) < nbytes:
+            raise ValueError("dst buffer too small")
+    for t in packed:
+        if _nbytes(t) < coll_packed_bytes(nbytes, proto):
+            raise ValueError("packed buffer too small")
+    st = None if status is None else _cuda(status, "status").data_ptr()
+    (pp, _kp), (pd, _kd) = _ptrs(packed), _ptrs(dst)
+    with torch.cuda.device(dst[0].device):
+        _check("coll_ll_unpack_ranks", lib().coll_ll_unpack_ranks(pp, pd, len(dst), nbytes, proto, step, st,
+                                                                  _stream(stream)))
 
 
 def coll_all_reduce_packed(packed_in, packed_out, count: int, dtype: torch.dtype, proto, step: int, op="sum",

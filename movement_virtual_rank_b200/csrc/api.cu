@@ -641,20 +641,67 @@ static bool valid_step(coll_proto_t proto, uint64_t step) {
 }
 
 int coll_ll_pack(const void* src, void* packed, size_t bytes, coll_proto_t proto, uint64_t step, coll_stream_t stream) {
-  if (proto != COLL_PROTO_LL && proto != COLL_PROTO_LL128) return COLL_ERR_UNSUPPORTED;
-  if (src == nullptr || packed == nullptr || !valid_step(proto, step) || !al16(packed)) return COLL_ERR_INVALID_ARG;
-  if (bytes == 0) return COLL_OK;
-  if (overlap(src, bytes, packed, coll_packed_bytes(bytes, proto))) return COLL_ERR_ALIAS;
-  return launch_ll_pack(src, packed, bytes, proto, step, S(stream));
+  return coll_ll_pack_ranks(&src, &packed, 1, bytes, proto, step, stream);
 }
 
 int coll_ll_unpack(const void* packed, void* dst, size_t bytes, coll_proto_t proto, uint64_t step, int* d_status,
                    coll_stream_t stream) {
+  return coll_ll_unpack_ranks(&packed, &dst, 1, bytes, proto, step, d_status, stream);
+}
+
+// the n messages (`mbytes` each) and the n packet buffers (`pbytes` each):
+// no message overlaps any packet buffer, and the written side's buffers are
+// disjoint
+static int codec_check(const void* const* msgs, const void* const* pkts, int n, size_t mbytes, size_t pbytes,
+                       bool pack) {
+  for (int r = 0; r < n; ++r)
+    if (!al16(pkts[r])) return COLL_ERR_INVALID_ARG;
+  for (int r = 0; r < n; ++r)
+    for (int q = 0; q < n; ++q) {
+      if (overlap(msgs[r], mbytes, pkts[q], pbytes)) return COLL_ERR_ALIAS;
+      if (q != r && (pack ? overlap(pkts[r], pbytes, pkts[q], pbytes) : overlap(msgs[r], mbytes, msgs[q], mbytes)))
+        return COLL_ERR_ALIAS;
+    }
+  return COLL_OK;
+}
+
+int coll_ll_pack_ranks(const void* const* src, void* const* packed, int nranks, size_t bytes, coll_proto_t proto,
+                       uint64_t step, coll_stream_t stream) {
   if (proto != COLL_PROTO_LL && proto != COLL_PROTO_LL128) return COLL_ERR_UNSUPPORTED;
-  if (dst == nullptr || packed == nullptr || !valid_step(proto, step) || !al16(packed)) return COLL_ERR_INVALID_ARG;
+  if (!valid_n(nranks) || !all_nonnull(src, nranks) || !all_nonnull(packed, nranks) || !valid_step(proto, step))
+    return COLL_ERR_INVALID_ARG;
+  const int c = codec_check(src, packed, nranks, bytes, coll_packed_bytes(bytes, proto), true);
+  if (c != COLL_OK) return c;
   if (bytes == 0) return COLL_OK;
-  if (overlap(dst, bytes, packed, coll_packed_bytes(bytes, proto))) return COLL_ERR_ALIAS;
-  return launch_ll_unpack(packed, dst, bytes, proto, step, d_status, S(stream));
+  CodecArgs a{};
+  for (int r = 0; r < nranks; ++r) {
+    a.in[r] = static_cast<const uint8_t*>(src[r]);
+    a.out[r] = static_cast<uint8_t*>(packed[r]);
+  }
+  a.bytes = bytes;
+  a.step = step;
+  a.n = nranks;
+  return launch_ll_pack(a, proto, S(stream));
+}
+
+int coll_ll_unpack_ranks(const void* const* packed, void* const* dst, int nranks, size_t bytes, coll_proto_t proto,
+                         uint64_t step, int* d_status, coll_stream_t stream) {
+  if (proto != COLL_PROTO_LL && proto != COLL_PROTO_LL128) return COLL_ERR_UNSUPPORTED;
+  if (!valid_n(nranks) || !all_nonnull(packed, nranks) || !all_nonnull(dst, nranks) || !valid_step(proto, step))
+    return COLL_ERR_INVALID_ARG;
+  const int c = codec_check(dst, packed, nranks, bytes, coll_packed_bytes(bytes, proto), false);
+  if (c != COLL_OK) return c;
+  if (bytes == 0) return COLL_OK;
+  CodecArgs a{};
+  for (int r = 0; r < nranks; ++r) {
+    a.in[r] = static_cast<const uint8_t*>(packed[r]);
+    a.out[r] = static_cast<uint8_t*>(dst[r]);
+  }
+  a.bytes = bytes;
+  a.step = step;
+  a.n = nranks;
+  a.status = d_status;
+  return launch_ll_unpack(a, proto, S(stream));
 }
 
 int coll_all_reduce_packed(const void* const* packed_in, void* const* packed_out, int nranks, size_t count,

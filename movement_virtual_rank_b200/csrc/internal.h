@@ -101,10 +101,18 @@ struct GatherRowsArgs {
 int launch_gather_rows(const GatherRowsArgs& a, cudaStream_t s);
 
 // --------------------------------------------------------------- packets ----
-int launch_ll_pack(const void* src, void* packed, size_t bytes, int proto, uint64_t step,
-                   cudaStream_t s);
-int launch_ll_unpack(const void* packed, void* dst, size_t bytes, int proto, uint64_t step,
-                     int* status, cudaStream_t s);
+// One codec launch encodes (pack) or decodes (unpack) the equally long
+// messages of n virtual ranks, blockIdx.y selecting the rank.
+struct CodecArgs {
+  const uint8_t* in[kMaxRanksH];  // messages (pack) or packets (unpack)
+  uint8_t* out[kMaxRanksH];       // packets (pack) or messages (unpack)
+  uint64_t bytes;                 // message bytes per rank
+  uint64_t step;                  // the flag
+  int n;
+  int* status;                    // unpack: flag mismatches (may be null)
+};
+int launch_ll_pack(const CodecArgs& a, int proto, cudaStream_t s);
+int launch_ll_unpack(const CodecArgs& a, int proto, cudaStream_t s);
 
 struct PackedReduceArgs {
   const char* in[kMaxRanksH];

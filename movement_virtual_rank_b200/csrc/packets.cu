@@ -54,11 +54,17 @@ __device__ __forceinline__ void store8_any(uint8_t* dst, uint64_t off, uint64_t 
 }
 
 // ------------------------------------------------------------------ LL ----
+//
+// Every codec kernel serves the n ranks of one call: CTA row blockIdx.y
+// takes ranks blockIdx.y, blockIdx.y + gridDim.y, ..., walking each rank's
+// message with a grid-stride loop.  The launcher gives every rank its own row
+// (gridDim.y = n), so all ranks are in flight at once: measured on one B200
+// against one rank after the other (gridDim.y = 1), as fast at 16 MiB per
+// rank and 1-2.5% faster at 256 MiB, and 9-21% faster than one launch per
+// rank at 16 MiB.  The alignment arguments hold for every rank's pointers.
 
-__global__ void __launch_bounds__(kThreads) k_ll_pack(const uint8_t* __restrict__ src, uint8_t* __restrict__ packed,
-                                                      uint64_t bytes, uint32_t flag, int src_al16) {
-  pdl_wait();
-  pdl_trigger();
+__device__ __forceinline__ void ll_pack_rank(const uint8_t* __restrict__ src, uint8_t* __restrict__ packed,
+                                             uint64_t bytes, uint32_t flag, int src_al16) {
   const uint64_t nlines = (bytes + 3) / 4;
   const uint64_t ngroups = nlines / 4;  // groups of 4 lines = 16 message bytes
   const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
@@ -81,26 +87,30 @@ __global__ void __launch_bounds__(kThreads) k_ll_pack(const uint8_t* __restrict_
     st8(packed + 8 * L, make_uint2(load_word_tail(src, 4 * L, bytes), flag));
 }
 
-__global__ void __launch_bounds__(kThreads) k_ll_unpack(const uint8_t* __restrict__ packed, uint8_t* __restrict__ dst,
-                                                        uint64_t bytes, uint32_t flag, int dst_al16, int* status) {
+__global__ void __launch_bounds__(kThreads) k_ll_pack(const __grid_constant__ CodecArgs a, int src_al16) {
   pdl_wait();
   pdl_trigger();
+  for (int r = blockIdx.y; r < a.n; r += gridDim.y) ll_pack_rank(a.in[r], a.out[r], a.bytes, static_cast<uint32_t>(a.step), src_al16);
+}
+
+__device__ __forceinline__ int ll_unpack_rank(const uint8_t* __restrict__ packed, uint8_t* __restrict__ dst,
+                                              uint64_t bytes, uint32_t flag, int dst_al16) {
   const uint64_t nlines = (bytes + 3) / 4;
   const uint64_t ngroups = nlines / 4;
   const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
   const uint64_t t0 = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   int bad = 0;
   for (uint64_t g = t0; g < ngroups; g += stride) {
-    const uint4 a = ld16(packed + 32 * g);
-    const uint4 b = ld16(packed + 32 * g + 16);
-    bad += (a.y != flag) + (a.w != flag) + (b.y != flag) + (b.w != flag);
+    const uint4 x0 = ld16(packed + 32 * g);
+    const uint4 x1 = ld16(packed + 32 * g + 16);
+    bad += (x0.y != flag) + (x0.w != flag) + (x1.y != flag) + (x1.w != flag);
     if (dst_al16 && 16 * g + 16 <= bytes) {
-      st16(dst + 16 * g, make_uint4(a.x, a.z, b.x, b.z));
+      st16(dst + 16 * g, make_uint4(x0.x, x0.z, x1.x, x1.z));
     } else {
-      store_bytes(dst, 16 * g, bytes, a.x);
-      store_bytes(dst, 16 * g + 4, bytes, a.z);
-      store_bytes(dst, 16 * g + 8, bytes, b.x);
-      store_bytes(dst, 16 * g + 12, bytes, b.z);
+      store_bytes(dst, 16 * g, bytes, x0.x);
+      store_bytes(dst, 16 * g + 4, bytes, x0.z);
+      store_bytes(dst, 16 * g + 8, bytes, x1.x);
+      store_bytes(dst, 16 * g + 12, bytes, x1.z);
     }
   }
   for (uint64_t L = 4 * ngroups + t0; L < nlines; L += stride) {
@@ -108,7 +118,16 @@ __global__ void __launch_bounds__(kThreads) k_ll_unpack(const uint8_t* __restric
     bad += (v.y != flag);
     store_bytes(dst, 4 * L, bytes, v.x);
   }
-  report_warp(status, COLL_DEV_FLAG_MISMATCH, bad);
+  return bad;
+}
+
+__global__ void __launch_bounds__(kThreads) k_ll_unpack(const __grid_constant__ CodecArgs a, int dst_al16) {
+  pdl_wait();
+  pdl_trigger();
+  int bad = 0;
+  for (int r = blockIdx.y; r < a.n; r += gridDim.y)
+    bad += ll_unpack_rank(a.in[r], a.out[r], a.bytes, static_cast<uint32_t>(a.step), dst_al16);
+  report_warp(a.status, COLL_DEV_FLAG_MISMATCH, bad);
 }
 
 // --------------------------------------------------------------- LL128 ----
@@ -122,11 +141,9 @@ __global__ void __launch_bounds__(kThreads) k_ll_unpack(const uint8_t* __restric
 constexpr int kGroupBytes = 480;  // 4 lines of payload
 constexpr int kWarps = kThreads / 32;
 
-__global__ void __launch_bounds__(kThreads) k_ll128_pack(const uint8_t* __restrict__ src, uint8_t* __restrict__ packed,
-                                                         uint64_t bytes, uint64_t step, int src_al8, int src_al16) {
-  __shared__ __align__(16) uint8_t stage[kWarps][2][kGroupBytes];
-  pdl_wait();
-  pdl_trigger();
+__device__ __forceinline__ void ll128_pack_rank(const uint8_t* __restrict__ src, uint8_t* __restrict__ packed,
+                                                uint64_t bytes, uint64_t step, int src_al8, int src_al16,
+                                                uint8_t (*stage)[2][kGroupBytes]) {
   const uint64_t nlines = (bytes + 119) / 120;
   uint64_t first = 0;  // first line of the 8-threads-per-line part
   if (src_al16) {
@@ -171,12 +188,17 @@ __global__ void __launch_bounds__(kThreads) k_ll128_pack(const uint8_t* __restri
   }
 }
 
-__global__ void __launch_bounds__(kThreads) k_ll128_unpack(const uint8_t* __restrict__ packed, uint8_t* __restrict__ dst,
-                                                           uint64_t bytes, uint64_t step, int dst_al8, int dst_al16,
-                                                           int* status) {
+__global__ void __launch_bounds__(kThreads) k_ll128_pack(const __grid_constant__ CodecArgs a, int src_al8,
+                                                         int src_al16) {
   __shared__ __align__(16) uint8_t stage[kWarps][2][kGroupBytes];
   pdl_wait();
   pdl_trigger();
+  for (int r = blockIdx.y; r < a.n; r += gridDim.y) ll128_pack_rank(a.in[r], a.out[r], a.bytes, a.step, src_al8, src_al16, stage);
+}
+
+__device__ __forceinline__ int ll128_unpack_rank(const uint8_t* __restrict__ packed, uint8_t* __restrict__ dst,
+                                                 uint64_t bytes, uint64_t step, int dst_al8, int dst_al16,
+                                                 uint8_t (*stage)[2][kGroupBytes]) {
   const uint64_t nlines = (bytes + 119) / 120;
   int bad = 0;
   uint64_t first = 0;
@@ -222,7 +244,18 @@ __global__ void __launch_bounds__(kThreads) k_ll128_unpack(const uint8_t* __rest
       bad += (f != step);
     }
   }
-  report_warp(status, COLL_DEV_FLAG_MISMATCH, bad);
+  return bad;
+}
+
+__global__ void __launch_bounds__(kThreads) k_ll128_unpack(const __grid_constant__ CodecArgs a, int dst_al8,
+                                                           int dst_al16) {
+  __shared__ __align__(16) uint8_t stage[kWarps][2][kGroupBytes];
+  pdl_wait();
+  pdl_trigger();
+  int bad = 0;
+  for (int r = blockIdx.y; r < a.n; r += gridDim.y)
+    bad += ll128_unpack_rank(a.in[r], a.out[r], a.bytes, a.step, dst_al8, dst_al16, stage);
+  report_warp(a.status, COLL_DEV_FLAG_MISMATCH, bad);
 }
 
 // ------------------------------------------------ bulk-copy LL pack path ----
@@ -238,13 +271,16 @@ __global__ void __launch_bounds__(kThreads) k_ll128_unpack(const uint8_t* __rest
 constexpr int kPackStages = 4;
 constexpr uint32_t kPackMsg = 4096, kPackPkt = 8192;
 
-__global__ void __launch_bounds__(32) k_ll_pack_tma(const unsigned char* __restrict__ src,
-                                                    unsigned char* __restrict__ packed, uint64_t tiles, uint32_t flag) {
+__global__ void __launch_bounds__(32) k_ll_pack_tma(const __grid_constant__ CodecArgs a, uint64_t tiles) {
   extern __shared__ __align__(128) unsigned char smem[];  // [stage]{in[kPackMsg], out[kPackPkt]}
   __shared__ __align__(8) uint64_t bar[kPackStages];
   constexpr uint32_t kStage = kPackMsg + kPackPkt;
   pdl_wait();
   pdl_trigger();
+  const uint32_t flag = static_cast<uint32_t>(a.step);
+  const unsigned char* __restrict__ src = a.in[blockIdx.y];  // one rank per CTA row
+  unsigned char* __restrict__ packed = a.out[blockIdx.y];
+  const uint64_t total = tiles;
   const int lane = threadIdx.x;
   if (lane == 0) {
     for (int st = 0; st < kPackStages; ++st) mbar_init(&bar[st], 1);
@@ -257,10 +293,10 @@ __global__ void __launch_bounds__(32) k_ll_pack_tma(const unsigned char* __restr
     bulk_load(smem + st * kStage, src + t * kPackMsg, kPackMsg, &bar[st]);
   };
   int inflight = 0;
-  for (int st = 0; st < kPackStages && blockIdx.x + st * stride < tiles; ++st, ++inflight)
+  for (int st = 0; st < kPackStages && blockIdx.x + st * stride < total; ++st, ++inflight)
     if (lane == 0) issue(blockIdx.x + st * stride, st);
   int i = 0;
-  for (uint64_t t = blockIdx.x; t < tiles; t += stride, ++i) {
+  for (uint64_t t = blockIdx.x; t < total; t += stride, ++i) {
     const int st = i % kPackStages;
     const uint32_t par = (i / kPackStages) & 1;
     int ok = 1;
@@ -292,7 +328,7 @@ __global__ void __launch_bounds__(32) k_ll_pack_tma(const unsigned char* __restr
       bulk_store(packed + t * kPackPkt, out, kPackPkt);
       bulk_commit();
       const uint64_t nxt = t + kPackStages * stride;
-      if (nxt < tiles) {
+      if (nxt < total) {
         issue(nxt, st);
         ++inflight;
       }
@@ -302,55 +338,80 @@ __global__ void __launch_bounds__(32) k_ll_pack_tma(const unsigned char* __restr
   if (lane == 0) bulk_wait_all();
 }
 
-int launch_ll_pack(const void* src, void* packed, size_t bytes, int proto, uint64_t step, cudaStream_t s) {
-  if (bytes == 0) return COLL_OK;
-  const auto* sp = static_cast<const uint8_t*>(src);
-  auto* pp = static_cast<uint8_t*>(packed);
-  if (proto == COLL_PROTO_LL && ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(packed)) & 15) == 0) {
+// The codec grid for n ranks of `units` work items each: one CTA row per
+// rank, at most 8 CTAs per SM in all
+static dim3 codec_grid(uint64_t units, int n) {
+  const unsigned gy = static_cast<unsigned>(n);
+  uint64_t gx = (units + kThreads - 1) / kThreads;
+  uint64_t cap = static_cast<uint64_t>(num_sms()) * 8 / gy;
+  if (cap < 1) cap = 1;
+  if (gx > cap) gx = cap;
+  if (gx < 1) gx = 1;
+  return dim3(static_cast<unsigned>(gx), gy);
+}
+
+// every message pointer's low bits, and every packet pointer's
+static void codec_bits(const CodecArgs& a, uintptr_t& msg, uintptr_t& pkt, bool pack) {
+  msg = pkt = 0;
+  for (int r = 0; r < a.n; ++r) {
+    msg |= reinterpret_cast<uintptr_t>(pack ? static_cast<const void*>(a.in[r]) : static_cast<const void*>(a.out[r]));
+    pkt |= reinterpret_cast<uintptr_t>(pack ? static_cast<const void*>(a.out[r]) : static_cast<const void*>(a.in[r]));
+  }
+}
+
+int launch_ll_pack(const CodecArgs& a0, int proto, cudaStream_t s) {
+  if (a0.bytes == 0 || a0.n < 1) return COLL_OK;
+  CodecArgs a = a0;
+  uintptr_t msg, pkt;
+  codec_bits(a, msg, pkt, true);
+  const dim3 block(kThreads);
+  if (proto == COLL_PROTO_LL && ((msg | pkt) & 15) == 0) {
     // whole tiles through the bulk-copy path when every CTA gets at least 4, the rest below
-    const unsigned grid = static_cast<unsigned>(num_sms()) * 4;  // 4 x 48 KB of stages per SM
-    const uint64_t tiles = bytes / kPackMsg;
-    if (tiles >= 4ull * grid) {
+    // 4 x 48 KB of stages per SM, shared by the ranks (one CTA row each)
+    unsigned gx = static_cast<unsigned>(num_sms()) * 4 / static_cast<unsigned>(a.n);
+    if (gx < 1) gx = 1;
+    const uint64_t tiles = a.bytes / kPackMsg;  // per rank
+    if (tiles >= 4ull * gx) {
       const size_t smem = static_cast<size_t>(kPackStages) * (kPackMsg + kPackPkt);
       static int smem_set[COLL_MAX_RANKS] = {0};  // per device ordinal: largest limit set so far
       const int ok = allow_dynamic_smem(reinterpret_cast<const void*>(k_ll_pack_tma), smem, smem_set);
       if (ok != COLL_OK) return ok;
-      launch_pdl(k_ll_pack_tma, dim3(grid), dim3(32), smem, s, sp, pp, tiles, static_cast<uint32_t>(step));
+      launch_pdl(k_ll_pack_tma, dim3(gx, a.n), dim3(32), smem, s, a, tiles);
       const int st = launch_status(cudaGetLastError());
       if (st != COLL_OK) return st;
-      sp += tiles * kPackMsg;
-      pp += tiles * kPackPkt;
-      bytes -= tiles * kPackMsg;
-      if (bytes == 0) return COLL_OK;
+      for (int r = 0; r < a.n; ++r) {
+        a.in[r] += tiles * kPackMsg;
+        a.out[r] += tiles * kPackPkt;
+      }
+      a.bytes -= tiles * kPackMsg;
+      if (a.bytes == 0) return COLL_OK;
     }
   }
   if (proto == COLL_PROTO_LL) {
-    const uint64_t nlines = (bytes + 3) / 4;
-    launch_pdl(k_ll_pack, dim3(grid_units(nlines / 4 + 1)), dim3(kThreads), 0, s, sp, pp, bytes, static_cast<uint32_t>(step),
-                                                               (reinterpret_cast<uintptr_t>(src) & 15) == 0);
+    const uint64_t nlines = (a.bytes + 3) / 4;
+    launch_pdl(k_ll_pack, codec_grid(nlines / 4 + 1, a.n), block, 0, s, a,
+               static_cast<int>((msg & 15) == 0));
   } else {
-    const uint64_t nlines = (bytes + 119) / 120;
-    const int al16 = ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(packed)) & 15) == 0;
-    launch_pdl(k_ll128_pack, dim3(grid_units(nlines * 8)), dim3(kThreads), 0, s, sp, pp, bytes, step,
-               static_cast<int>((reinterpret_cast<uintptr_t>(src) & 7) == 0), al16);
+    const uint64_t nlines = (a.bytes + 119) / 120;
+    launch_pdl(k_ll128_pack, codec_grid(nlines * 8, a.n), block, 0, s, a,
+               static_cast<int>((msg & 7) == 0), static_cast<int>(((msg | pkt) & 15) == 0));
   }
   return launch_status(cudaGetLastError());
 }
 
-int launch_ll_unpack(const void* packed, void* dst, size_t bytes, int proto, uint64_t step, int* status,
-                     cudaStream_t s) {
-  if (bytes == 0) return COLL_OK;
-  const auto* pp = static_cast<const uint8_t*>(packed);
-  auto* dp = static_cast<uint8_t*>(dst);
+int launch_ll_unpack(const CodecArgs& a, int proto, cudaStream_t s) {
+  if (a.bytes == 0 || a.n < 1) return COLL_OK;
+  uintptr_t msg, pkt;
+  codec_bits(a, msg, pkt, false);
+  const dim3 block(kThreads);
   if (proto == COLL_PROTO_LL) {
-    const uint64_t nlines = (bytes + 3) / 4;
-    launch_pdl(k_ll_unpack, dim3(grid_units(nlines / 4 + 1)), dim3(kThreads), 0, s, pp, dp, bytes, static_cast<uint32_t>(step),
-                                                                 (reinterpret_cast<uintptr_t>(dst) & 15) == 0, status);
+    const uint64_t nlines = (a.bytes + 3) / 4;
+    launch_pdl(k_ll_unpack, codec_grid(nlines / 4 + 1, a.n), block, 0, s, a,
+               static_cast<int>((msg & 15) == 0));
   } else {
-    const uint64_t nlines = (bytes + 119) / 120;
-    const int al16 = ((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(packed)) & 15) == 0;
-    launch_pdl(k_ll128_unpack, dim3(grid_units(nlines * 8)), dim3(kThreads), 0, s, pp, dp, bytes, step,
-               static_cast<int>((reinterpret_cast<uintptr_t>(dst) & 7) == 0), al16, status);
+    const uint64_t nlines = (a.bytes + 119) / 120;
+    launch_pdl(k_ll128_unpack, codec_grid(nlines * 8, a.n), block, 0, s, a,
+               static_cast<int>((msg & 7) == 0), static_cast<int>(((msg | pkt) & 15) == 0));
   }
   return launch_status(cudaGetLastError());
 }

@@ -221,6 +221,18 @@ def test_invalid_arguments_rejected_on_host():
     assert L.coll_ll_unpack(BASE, BASE + 0x100000, 64, M.LL, 0, None, None) == -1
     assert L.coll_ll_pack(BASE, BASE + 0x100000, 64, 7, 1, None) == -2
     assert L.coll_all_reduce_packed(p, q, 4, 16, M.BF16, M.SUM, M.LL128, 0, None, None) == -1
+    # the N-rank codecs: the same checks per rank, plus overlap between ranks
+    assert L.coll_ll_pack_ranks(p, q, 4, 64, M.LL, 0, None) == -1
+    assert L.coll_ll_pack_ranks(p, q, 0, 64, M.LL, 1, None) == -1
+    assert L.coll_ll_pack_ranks(p, q, 4, 64, 7, 1, None) == -2
+    assert L.coll_ll_unpack_ranks(q, p, 4, 64, M.LL128, 0, None, None) == -1
+    q8, _k8 = _arr([BASE + 0x10000000 + i * 0x100000 + (8 if i == 2 else 0) for i in range(4)])
+    assert L.coll_ll_pack_ranks(p, q8, 4, 64, M.LL, 1, None) == -1  # a packet buffer not 16-byte aligned
+    qo, _ko = _arr([BASE + 0x10000000 + i * 0x40 for i in range(4)])  # packets 64 B apart, 128 B long
+    assert L.coll_ll_pack_ranks(p, qo, 4, 64, M.LL, 1, None) == -3
+    assert L.coll_ll_pack_ranks(p, p, 4, 64, M.LL, 1, None) == -3  # message and packet buffer overlap
+    po, _kpo = _arr([BASE + i * 0x20 for i in range(4)])  # decoded messages 32 B apart, 64 B long
+    assert L.coll_ll_unpack_ranks(q, po, 4, 64, M.LL, 1, None, None) == -3
     # MoE shapes
     assert L.coll_moe_route(p, 4, 16, 0, 8, BASE, BASE, BASE, q, None, BASE, 1 << 20, None) == -1
     assert L.coll_moe_route(p, 4, 16, 2, 6, BASE, BASE, BASE, q, None, BASE, 1 << 20, None) == -1
@@ -276,6 +288,8 @@ def test_zero_counts_are_noops_on_host():
     assert L.coll_broadcast(p, 4, 0, M.INT32, 1, None) == 0
     assert L.coll_all_gather(p, q, 4, 0, M.BF16, None) == 0
     assert L.coll_ll_pack(BASE, BASE + 0x100000, 0, M.LL, 1, None) == 0
+    assert L.coll_ll_pack_ranks(p, q, 4, 0, M.LL128, 1, None) == 0
+    assert L.coll_ll_unpack_ranks(q, p, 4, 0, M.LL, 1, None, None) == 0
     # a single rank in place does nothing
     assert L.coll_all_reduce(p, p, 1, 100, M.BF16, M.SUM, M.TWOSHOT, None, 0, None) == 0
     assert L.coll_broadcast(p, 1, 100, M.BF16, 0, None) == 0

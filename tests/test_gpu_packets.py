@@ -225,3 +225,72 @@ def test_unpack_counts_bad_flags_bulk_path(proto):
     torch.cuda.synchronize()
     assert st.tolist() == [M.DEV_FLAG_MISMATCH, int(bad_lines.size)]
     assert torch.equal(out, torch.from_numpy(msg).cuda())  # the data are written all the same
+
+
+@pytest.mark.parametrize("proto", [M.LL, M.LL128])
+@pytest.mark.parametrize("n,nbytes", [(1, 1000), (3, 1), (3, 121), (8, 4097), (8, 65536 + 12), (5, (1 << 20) + 7),
+                                      (8, 16 << 20), (8, (16 << 20) + 120 * 3 + 5), (2, 10_000_000),
+                                      (2, (64 << 20) + 4097)])
+@pytest.mark.parametrize("unaligned_rank", [None, 1])
+def test_pack_unpack_ranks(proto, n, nbytes, unaligned_rank):
+    """All ranks' messages in one launch (a CTA row per rank): every rank's
+    packets are the oracle's encoding of its own message, the round trip is
+    exact, and no byte outside a buffer is touched.  One rank's message at an
+    odd offset sends every rank down the unaligned code."""
+    need_gpu()
+    if unaligned_rank is not None and unaligned_rank >= n:
+        pytest.skip("fewer ranks")
+    step = 0x2468_1357 + n if proto == M.LL else (0x77 << 48) + nbytes
+    pb = M.coll_packed_bytes(nbytes, proto)
+    msgs = [u8(nbytes, 31 * r + nbytes % 997) for r in range(n)]
+    offs = [1 if r == unaligned_rank else 0 for r in range(n)]
+    raws = [torch.zeros(nbytes + 64, dtype=torch.uint8, device="cuda") for _ in range(n)]
+    src = [raws[r][offs[r]:offs[r] + nbytes] for r in range(n)]
+    for r in range(n):
+        src[r].copy_(torch.from_numpy(msgs[r]).cuda())
+    pk_raw = [torch.full((pb + 64,), 0xEE, dtype=torch.uint8, device="cuda") for _ in range(n)]
+    packed = [t[:pb] for t in pk_raw]
+    M.coll_ll_pack_ranks(src, packed, proto, step)
+    torch.cuda.synchronize()
+    for r in range(n):
+        assert np.array_equal(packed[r].cpu().numpy(), oracle.pack(msgs[r], proto, step)), r
+        assert (pk_raw[r][pb:] == 0xEE).all(), r
+    out_raw = [torch.full((nbytes + 64,), 0x33, dtype=torch.uint8, device="cuda") for _ in range(n)]
+    dst = [out_raw[r][offs[r] + 3:offs[r] + 3 + nbytes] for r in range(n)]
+    st = status_tensor()
+    M.coll_ll_unpack_ranks(packed, dst, proto, step, status=st)
+    torch.cuda.synchronize()
+    for r in range(n):
+        assert np.array_equal(dst[r].cpu().numpy(), msgs[r]), r
+        o = out_raw[r].cpu().numpy()
+        assert (o[:offs[r] + 3] == 0x33).all() and (o[offs[r] + 3 + nbytes:] == 0x33).all(), r
+    assert st.tolist() == [0, 0]
+
+
+@pytest.mark.parametrize("proto", [M.LL, M.LL128])
+def test_unpack_ranks_counts_bad_flags(proto):
+    """Corrupted flags in several ranks' packets are counted exactly, summed
+    over the ranks, and every rank's data is still written."""
+    need_gpu()
+    n, nbytes, step = 4, (1 << 20) + 333, 5
+    line = 8 if proto == M.LL else 128
+    flag_at = 4 if proto == M.LL else 120
+    msgs = [u8(nbytes, 500 + r) for r in range(n)]
+    total = 0
+    packed = []
+    for r in range(n):
+        pk = oracle.pack(msgs[r], proto, step)
+        if r in (1, 3):
+            g = W.rng(W.W_MISC, 4, salt=r)
+            lines = np.unique(g.integers(0, pk.size // line, 40 + r))
+            for L in lines:
+                pk[L * line + flag_at] ^= 0x10
+            total += lines.size
+        packed.append(torch.from_numpy(pk).cuda())
+    dst = [torch.empty(nbytes, dtype=torch.uint8, device="cuda") for _ in range(n)]
+    st = status_tensor()
+    M.coll_ll_unpack_ranks(packed, dst, proto, step, status=st)
+    torch.cuda.synchronize()
+    assert st.tolist() == [M.DEV_FLAG_MISMATCH, total]
+    for r in range(n):
+        assert np.array_equal(dst[r].cpu().numpy(), msgs[r]), r
