@@ -31,7 +31,7 @@ from .numerics import (  # noqa: F401
 )
 from .collectives import (  # noqa: F401
     broadcast, gather, reduce, scatter, reduce_scatter, all_reduce,
-    all_reduce_one_shot, all_reduce_two_shot, all_reduce_ring, all_gather,
+    all_reduce_one_shot, all_reduce_two_shot, all_reduce_ring, all_reduce_ring_wire, all_gather,
     all_to_all, all_to_all_v, segment_elems,
 )
 from .moe import moe_route, moe_route_dedup, moe_dispatch, moe_combine, moe_permute_send  # noqa: F401

@@ -171,6 +171,41 @@ def all_reduce_ring(xs, op: int, dtype: str, trace=None):
     return outs
 
 
+def all_reduce_ring_wire(xs, op: int, dtype: str):
+    """The same ring (chunk order and the 2(N-1) steps of ``all_reduce_ring``)
+    with the partial travelling in the buffers' own type: every rank that
+    receives a chunk's partial widens it, combines its own values in the
+    arithmetic type, and rounds the result back to the storage type before
+    passing it on, as a ring whose messages carry the buffer dtype does.
+
+    Reading: the pages fix no wire type for the ring (NCCL's ring kernel is
+    only named in "From NCCL Ring LL ..."); this is the variant in which
+    every hop rounds, reported beside the fp32-partial ring.  For fp32 and
+    int32 the storage and arithmetic types agree, and for MAX / MIN rounding
+    a winner's own bits is exact, so there it equals ``all_reduce_ring``.
+    """
+    n = len(xs)
+    count = xs[0].size
+    seg = segment_elems(count, n, dtype)
+    bounds = [(min(c * seg, count), min((c + 1) * seg, count)) for c in range(n)]
+    outs = [np.empty_like(np.asarray(xs[0])) for _ in range(n)]
+    if n == 1:
+        outs[0][:] = np.asarray(xs[0])
+        return outs
+    # rank c+1 starts chunk c with its own (storage-type) values
+    msg = [np.array(np.asarray(xs[(c + 1) % n])[lo:hi], copy=True) for c, (lo, hi) in enumerate(bounds)]
+    for k in range(1, n):  # reduce-scatter steps: each hop delivers a storage-type message
+        for c, (lo, hi) in enumerate(bounds):
+            r = (c + 1 + k) % n
+            msg[c] = narrow(combine(widen(msg[c], dtype), widen(np.asarray(xs[r])[lo:hi], dtype), op, dtype), dtype)
+    for c, (lo, hi) in enumerate(bounds):  # complete on rank c
+        outs[c][lo:hi] = msg[c]
+    for j in range(1, n):  # all-gather steps, as in all_reduce_ring
+        for c, (lo, hi) in enumerate(bounds):
+            outs[(c + j) % n][lo:hi] = outs[(c + j - 1) % n][lo:hi]
+    return outs
+
+
 # ---------------------------------------------------------- AllGather ----
 
 def all_gather(xs):

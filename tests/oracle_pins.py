@@ -401,6 +401,99 @@ def pin_ring_schedule():
     assert float(oracle.all_reduce(vals, SUM, "fp32")[0][0]) == 1.0
 
 
+def pin_ring_wire_hand_example():
+    """The per-hop-rounding ring on one bf16 element, worked by hand.  With 3
+    ranks and 1 element only chunk 0 holds data, accumulated in the ring
+    order: rank 1's value, then rank 2's, then rank 0's.  bf16 keeps 8
+    significant bits, so next to 1 the spacing is 2^-7 and 1 + 2^-8 is a tie
+    that rounds to even, to 1.  With t = 2^-8, ranks (x0, x1, x2):
+      (t, 1, t): 1 + t -> 1, then 1 + t -> 1; the fp32-partial ring keeps
+                 1 + 2t = 1 + 2^-7 exactly and rounds once to it;
+      (t, t, 1): t + 1 -> 1, then 1 + t -> 1 (rank order would give
+                 t + t = 2^-7 exactly, then 1 + 2^-7);
+      (1, t, t): t + t = 2^-7 exactly, then 2^-7 + 1 = 1 + 2^-7, which bf16
+                 holds: both rings agree."""
+    t = 2.0 ** -8
+    cases = [((t, 1.0, t), 1.0, 1.0 + 2.0 ** -7),   # x0, x1, x2 -> wire, fp32 ring
+             ((t, t, 1.0), 1.0, 1.0 + 2.0 ** -7),
+             ((1.0, t, t), 1.0 + 2.0 ** -7, 1.0 + 2.0 ** -7)]
+    for vals, want_wire, want_ring in cases:
+        xs = [bf16([v]) for v in vals]
+        wire = oracle.all_reduce_ring_wire(xs, SUM, "bf16")
+        ring = oracle.all_reduce_ring(xs, SUM, "bf16")
+        for q in range(3):
+            assert float(bf16_to_float(wire[q])[0]) == want_wire, (vals, q)
+            assert float(bf16_to_float(ring[q])[0]) == want_ring, (vals, q)
+
+
+def _bf16_rne_fraction(q: fractions.Fraction) -> fractions.Fraction:
+    """A rational rounded to the nearest bf16 value, ties to even (finite,
+    normal range), from the definition: 8 significant bits."""
+    if q == 0:
+        return fractions.Fraction(0)
+    sign = -1 if q < 0 else 1
+    a = abs(q)
+    e = math.floor(math.log2(a))
+    if fractions.Fraction(2) ** e > a:
+        e -= 1
+    elif fractions.Fraction(2) ** (e + 1) <= a:
+        e += 1
+    ulp = fractions.Fraction(2) ** (e - 7)
+    m = a / ulp  # in [128, 256)
+    lo = math.floor(m)
+    rem = m - lo
+    if rem > fractions.Fraction(1, 2) or (rem == fractions.Fraction(1, 2) and lo % 2 == 1):
+        lo += 1
+    return sign * lo * ulp
+
+
+def pin_ring_wire_exact_rational():
+    """Random bf16 inputs on 2..8 ranks: every element equals the chunk's
+    ring-order sum with a round to bf16 after every addition, computed in
+    exact rationals (no float arithmetic in the reference)."""
+    g = W.rng(W.W_MISC, 11, salt=3)
+    for n in range(2, 9):
+        count = 40
+        xs = [bf16(g.uniform(-4, 4, count).astype(np.float32)) for _ in range(n)]
+        got = oracle.all_reduce_ring_wire(xs, SUM, "bf16")
+        seg = oracle.segment_elems(count, n, "bf16")
+        vals = [[fractions.Fraction(float(v)) for v in bf16_to_float(x)] for x in xs]
+        for e in range(count):
+            c = e // seg
+            acc = vals[(c + 1) % n][e]
+            for k in range(1, n):
+                acc = _bf16_rne_fraction(acc + vals[(c + 1 + k) % n][e])
+            for q in range(n):
+                assert fractions.Fraction(float(bf16_to_float(got[q][e:e + 1])[0])) == acc, (n, e, q)
+
+
+def pin_ring_wire_reduces_to_ring():
+    """Where rounding to the storage type changes nothing the two rings
+    agree bit for bit: fp32 and int32 (storage = arithmetic type), MAX / MIN
+    (the winner's own bits), and 2 ranks (one addition, one rounding)."""
+    for dtype in ("fp32", "int32"):
+        for op in (SUM, PROD, MAX, MIN):
+            for n in (2, 3, 5, 8):
+                if dtype == "int32":
+                    g = W.rng(W.W_MISC, 12, salt=n + 10 * op)
+                    xs = [g.integers(-1000, 1000, 333, dtype=np.int64).astype(np.int32) for _ in range(n)]
+                else:
+                    xs = W.ranks_values(W.W_MISC, n, 333, dtype, "uniform" if op == PROD else "normal", salt=n + op)
+                a = oracle.all_reduce_ring_wire(xs, op, dtype)
+                b = oracle.all_reduce_ring(xs, op, dtype)
+                for q in range(n):
+                    assert np.array_equal(np.asarray(a[q]).view(np.uint32), np.asarray(b[q]).view(np.uint32))
+    for dtype in ("bf16", "fp16"):
+        for op in (MAX, MIN):
+            xs = W.ranks_values(W.W_MISC, 6, 1001, dtype, "normal", salt=op)
+            assert all(np.array_equal(a, b) for a, b in zip(oracle.all_reduce_ring_wire(xs, op, dtype),
+                                                            oracle.all_reduce_ring(xs, op, dtype)))
+        for op in (SUM, PROD):
+            xs = W.ranks_values(W.W_MISC, 2, 1001, dtype, "uniform", salt=op + 7)
+            assert all(np.array_equal(a, b) for a, b in zip(oracle.all_reduce_ring_wire(xs, op, dtype),
+                                                            oracle.all_reduce_ring(xs, op, dtype)))
+
+
 def pin_all_to_all_v_roundtrip():
     for n in (1, 2, 5, 8):
         row = 3

@@ -232,6 +232,22 @@ def m_ring_partials_in_storage_type(mp):
     mp.setattr(C, "combine", f)
 
 
+def m_ring_wire_without_hop_rounding(mp):
+    """the storage-type ring carries fp32 partials after all (rounds once)"""
+    _patch(mp, "all_reduce_ring_wire", lambda xs, op, dtype: C.all_reduce_ring(xs, op, dtype))
+
+
+def m_ring_wire_rank_order(mp):
+    """the storage-type ring rounds at every step but adds in rank order 0..N-1"""
+    def f(xs, op, dtype):
+        n = len(xs)
+        acc = np.array(np.asarray(xs[0]), copy=True)
+        for r in range(1, n):
+            acc = NUM.narrow(NUM.combine(NUM.widen(acc, dtype), NUM.widen(np.asarray(xs[r]), dtype), op, dtype), dtype)
+        return [np.array(acc, copy=True) for _ in range(n)]
+    _patch(mp, "all_reduce_ring_wire", f)
+
+
 def m_segment_unaligned(mp):
     _patch(mp, "segment_elems", lambda count, n, dtype: -(-count // n) + 1)
 
