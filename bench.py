@@ -121,7 +121,7 @@ def _dev(a: np.ndarray, dtype):
 
 
 FORM_NAMES = {1: "oneshot", 2: "twoshot", 4: "ring_ll", 5: "ring_cluster", 6: "ring_steps", 7: "twoshot_ll",
-              8: "ring_cta", 9: "twoshot_ll128", 10: "ring_lane"}
+              8: "ring_cta", 9: "twoshot_ll128", 10: "ring_lane", 11: "ring_wire"}
 
 
 def tp_decode_cfg(n):
@@ -388,7 +388,7 @@ def build_ring_compare(M, oracle):
         send = [_dev(x, torch.bfloat16) for x in xs]
         for algo, aname, launches in ((M.RING_STEPS, "ring_steps", 2 * (n - 1)), (M.RING_LL, "ring_ll", 1),
                                       (M.RING_CLUSTER, "ring_cluster", 1), (M.RING_CTA, "ring_cta", 1),
-                                      (M.RING_LANE, "ring_lane", 1),
+                                      (M.RING_LANE, "ring_lane", 1), (M.RING_WIRE, "ring_wire", 1),
                                       (M.TWOSHOT_LL, "twoshot_ll", 1), (M.TWOSHOT_LL128, "twoshot_ll128", 1)):
             need = max(64, M.coll_all_reduce_workspace_size(n, count, torch.bfloat16, algo))
             ops.append(Op(f"all_reduce/{aname}",
@@ -420,6 +420,7 @@ def build_ring_compare(M, oracle):
                               "ring_cluster (one launch, cluster DSMEM hops)",
                               "ring_cta (one launch, ranks as warp groups, shared-memory hops)",
                               "ring_lane (one launch, ranks as lanes, warp-shuffle hops)",
+                              "ring_wire (the CTA ring with partials rounded to bf16 at every hop: a different result)",
                               "twoshot_ll (one launch, LL packets, fused)",
                               "twoshot_ll128 (one launch, LL128 packets, fused)",
                               "LL pack + packetised two-shot + unpack (stream-ordered, 3 launches)"]}
@@ -667,7 +668,8 @@ def build_allreduce_forms(M, oracle):
 def build_hbm_ceilings(M, oracle):
     """Context for the movement kernels' fractions: what this GPU's HBM does
     for a write-only stream (a fill), a read-only one (a sum) and a copy, on
-    4 GiB with torch's own kernels.  The collectives here mostly write far
+    4 GiB, and for a 1 -> 8 fan-out and an 8 -> 1 fan-in of 128 MiB, with
+    torch's own kernels.  The collectives here mostly write far
     more than they read (all_gather and dispatch write 8 bytes per byte read),
     so the copy figure that the roofline uses is not their only ceiling."""
     import torch
@@ -675,6 +677,9 @@ def build_hbm_ceilings(M, oracle):
     a = torch.ones(n, device="cuda")
     b = torch.empty(n, device="cuda")
     nb = 4 * n
+    small = 128 << 20  # bytes
+    s_small = torch.ones(small // 2, dtype=torch.bfloat16, device="cuda")
+    d_big = torch.empty(8, small // 2, dtype=torch.bfloat16, device="cuda")
     return [
         Op("write_only_fill", lambda bf: (lambda: bf["b"].fill_(2.0)), {"b": b}, nb, 0,
            {"op": "fill (torch)", "bytes": nb}, kernel="write_only_fill"),
@@ -684,6 +689,15 @@ def build_hbm_ceilings(M, oracle):
         # copy-engine transfer, which is not what the kernels here compete with
         Op("copy", lambda bf: (lambda: torch.mul(bf["a"], 1.0, out=bf["b"])), {"a": a, "b": b}, 2 * nb, 0,
            {"op": "copy (torch elementwise)", "bytes": 2 * nb}, kernel="copy"),
+        # the all_gather / dispatch mix (one byte read, eight written) and the
+        # combine / reduce_scatter mix (eight read, one written), at the
+        # default step's all_gather size: 128 MiB <-> 8 x 128 MiB of bf16
+        Op("fan_out_1to8", lambda bf: (lambda: bf["d"].copy_(bf["s"].expand(8, -1))),
+           {"s": s_small, "d": d_big}, small + 8 * small, 0,
+           {"op": "1 -> 8 broadcast copy (torch elementwise)", "bytes": 9 * small}, kernel="fan_out_1to8"),
+        Op("fan_in_8to1", lambda bf: (lambda: torch.sum(bf["d"], 0, out=bf["s"])),
+           {"s": s_small, "d": d_big}, small + 8 * small, 0,
+           {"op": "8 -> 1 sum (torch)", "bytes": 9 * small}, kernel="fan_in_8to1"),
     ], {"workload": "hbm_ceilings_4GiB", "note": "torch kernels, context only"}
 
 

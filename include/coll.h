@@ -89,7 +89,8 @@ typedef enum {
   COLL_ALGO_TWOSHOT_LL = 7,   /* TWOSHOT in one launch, LL packets between ranks */
   COLL_ALGO_RING_CTA = 8,     /* the same ring, ranks = warp groups of one CTA, hops in shared memory */
   COLL_ALGO_TWOSHOT_LL128 = 9, /* TWOSHOT in one launch, LL128 packets between ranks */
-  COLL_ALGO_RING_LANE = 10     /* the same ring, ranks = lanes of one warp, hops by warp shuffles */
+  COLL_ALGO_RING_LANE = 10,    /* the same ring, ranks = lanes of one warp, hops by warp shuffles */
+  COLL_ALGO_RING_WIRE = 11     /* the ring's order, partials rounded to the buffer type at every hop */
 } coll_algo_t;
 typedef enum { COLL_PROTO_SIMPLE = 0, COLL_PROTO_LL = 1, COLL_PROTO_LL128 = 2 } coll_proto_t;
 
@@ -229,6 +230,16 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    input and output byte once.  Needs 2 <= N <= 8 and 16-byte aligned
  *    buffers, with the same fallback as RING_CLUSTER; `workspace` is
  *    optional and unused (this form raises no device status).
+ *  RING_WIRE: the RING schedule and chunk order with a different result:
+ *    every reduce-scatter hop carries the partial rounded to the buffers'
+ *    type (a ring whose messages carry the buffer dtype), so each receiver
+ *    widens it, combines its own values in fp32 and rounds again.  For bf16
+ *    / fp16 SUM and PROD the result differs from RING's by those extra
+ *    roundings (no bound is promised); for fp32, int32, MAX and MIN it is
+ *    RING's bit for bit.  Runs as RING_CTA with half the hop bytes for
+ *    bf16 / fp16; needs 2 <= N <= 8 and 16-byte aligned buffers
+ *    (COLL_ERR_UNSUPPORTED otherwise: there is no stream-ordered form);
+ *    `workspace` is ignored.
  *  TWOSHOT_LL ([RLL] "Traditional LL Protocols" and the "Pro5000 ?" two-shot,
  *    fused): the TWOSHOT segments and arithmetic (bit-identical result) in
  *    ONE cooperative launch.  Every rank writes each 16-byte group of its
@@ -269,10 +280,12 @@ COLL_API size_t coll_all_reduce_workspace_size(int nranks, size_t count, coll_dt
                                       coll_algo_t algo);
 /* The form coll_all_reduce() runs for these arguments when nranks >= 2 and
  * count >= 1: ONESHOT, TWOSHOT, TWOSHOT_LL, TWOSHOT_LL128, RING_LL,
- * RING_CLUSTER, RING_CTA, RING_LANE or RING_STEPS (AUTO and RING resolved, AUTO for a call that is not in
- * place; `aligned` != 0 when every buffer is 16-byte aligned).  RING_STEPS launches 2(N-1) kernels, the others one.
- * Returns a negative COLL_ERR_* for an invalid rank count, dtype or algo.
- * Library introspection; the sources have no counterpart. */
+ * RING_CLUSTER, RING_CTA, RING_LANE, RING_WIRE or RING_STEPS (AUTO and RING
+ * resolved, AUTO for a call that is not in place; `aligned` != 0 when every
+ * buffer is 16-byte aligned).  RING_STEPS launches 2(N-1) kernels, the
+ * others one.  Returns a negative COLL_ERR_* for an invalid rank count,
+ * dtype or algo, and COLL_ERR_UNSUPPORTED for a RING_WIRE call that cannot
+ * run.  Library introspection; the sources have no counterpart. */
 COLL_API int coll_all_reduce_form(int nranks, size_t count, coll_dtype_t dtype, coll_algo_t algo,
                                   int aligned);
 

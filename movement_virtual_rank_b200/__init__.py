@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libmvrcoll.so")
 BF16, FP16, FP32, INT32 = 0, 1, 2, 3
 SUM, MAX, MIN, PROD = 0, 1, 2, 3
 (ALGO_AUTO, ONESHOT, TWOSHOT, RING, RING_LL, RING_CLUSTER, RING_STEPS, TWOSHOT_LL, RING_CTA, TWOSHOT_LL128,
- RING_LANE) = range(11)
+ RING_LANE, RING_WIRE) = range(12)
 SIMPLE, LL, LL128 = 0, 1, 2
 DEV_OK, DEV_FLAG_MISMATCH, DEV_TIMEOUT, DEV_SPLIT_OVERFLOW, DEV_BAD_ROUTE, DEV_EPOCH_WRAP = 0, 1, 2, 3, 4, 5
 RING_LL_CALLS_PER_FILL, TWOSHOT_LL_CALLS_PER_FILL = 1 << 25, 1 << 30  # calls one zero-filled workspace serves
@@ -35,7 +35,7 @@ OPS = {"sum": SUM, "max": MAX, "min": MIN, "prod": PROD}
 ALGOS = {"auto": ALGO_AUTO, "oneshot": ONESHOT, "twoshot": TWOSHOT, "ring": RING, "ring_ll": RING_LL,
          "ring_cluster": RING_CLUSTER, "ring_steps": RING_STEPS, "twoshot_ll": TWOSHOT_LL,
          "ring_cta": RING_CTA, "twoshot_ll128": TWOSHOT_LL128,
-         "ring_lane": RING_LANE}
+         "ring_lane": RING_LANE, "ring_wire": RING_WIRE}
 PROTOS = {"simple": SIMPLE, "ll": LL, "ll128": LL128}
 
 
@@ -247,8 +247,8 @@ def coll_all_reduce_workspace_size(nranks: int, count: int, dtype: torch.dtype, 
 
 def coll_all_reduce_form(nranks: int, count: int, dtype: torch.dtype, algo=TWOSHOT, aligned: bool = True) -> int:
     """The form coll_all_reduce() runs: ONESHOT, TWOSHOT, TWOSHOT_LL, TWOSHOT_LL128,
-    RING_LL, RING_CLUSTER, RING_CTA, RING_LANE (one launch each) or RING_STEPS
-    (2(N-1) launches)."""
+    RING_LL, RING_CLUSTER, RING_CTA, RING_LANE, RING_WIRE (one launch each) or
+    RING_STEPS (2(N-1) launches)."""
     algo = ALGOS[algo] if isinstance(algo, str) else int(algo)
     rc = int(lib().coll_all_reduce_form(nranks, count, _DTYPES[dtype], algo, 1 if aligned else 0))
     if rc < 0:

@@ -371,7 +371,7 @@ size_t coll_all_reduce_workspace_size(int nranks, size_t count, coll_dtype_t dty
 int coll_all_reduce_form(int nranks, size_t count, coll_dtype_t dtype, coll_algo_t algo, int aligned) {
   const int es = elem_size(dtype);
   if (!es || !valid_n(nranks)) return COLL_ERR_INVALID_ARG;
-  if (algo < COLL_ALGO_AUTO || algo > COLL_ALGO_RING_LANE) return COLL_ERR_UNSUPPORTED;
+  if (algo < COLL_ALGO_AUTO || algo > COLL_ALGO_RING_WIRE) return COLL_ERR_UNSUPPORTED;
   const bool vec = aligned != 0;
   switch (algo) {
     case COLL_ALGO_AUTO: return auto_form(nranks, count * es, false);
@@ -383,6 +383,7 @@ int coll_all_reduce_form(int nranks, size_t count, coll_dtype_t dtype, coll_algo
       return vec && ring_cluster_supported(nranks) ? COLL_ALGO_RING_CLUSTER : COLL_ALGO_RING_STEPS;
     case COLL_ALGO_RING_CTA: return vec && ring_cta_supported(nranks) ? COLL_ALGO_RING_CTA : COLL_ALGO_RING_STEPS;
     case COLL_ALGO_RING_LANE: return vec && ring_lane_supported(nranks) ? COLL_ALGO_RING_LANE : COLL_ALGO_RING_STEPS;
+    case COLL_ALGO_RING_WIRE: return vec && ring_cta_supported(nranks) ? COLL_ALGO_RING_WIRE : COLL_ERR_UNSUPPORTED;
     default: return algo;
   }
 }
@@ -391,7 +392,7 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
                     coll_op_t op, coll_algo_t algo, void* workspace, size_t workspace_bytes, coll_stream_t stream) {
   const int es = elem_size(dtype);
   if (!es) return COLL_ERR_UNSUPPORTED;
-  if (!valid_op(op) || algo < COLL_ALGO_AUTO || algo > COLL_ALGO_RING_LANE) return COLL_ERR_UNSUPPORTED;
+  if (!valid_op(op) || algo < COLL_ALGO_AUTO || algo > COLL_ALGO_RING_WIRE) return COLL_ERR_UNSUPPORTED;
   if (!valid_n(nranks) || !all_nonnull(send, nranks) || !all_nonnull(recv, nranks)) return COLL_ERR_INVALID_ARG;
   const size_t bytes = count * es;
   if (bytes == 0) return COLL_OK;
@@ -422,6 +423,16 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
   for (int r = 0; r < nranks; ++r) vec = vec && al16(send[r]) && al16(recv[r]);
   const size_t seg = seg_elems(count, nranks, es);
   if (algo == COLL_ALGO_RING) algo = ring_form(nranks, bytes, vec);  // workspace checked above
+  if (algo == COLL_ALGO_RING_WIRE) {  // one launch only: there is no stream-ordered form with rounded partials
+    if (!vec || !ring_cta_supported(nranks)) return COLL_ERR_UNSUPPORTED;
+    const char* in[COLL_MAX_RANKS];
+    char* out[COLL_MAX_RANKS];
+    for (int r = 0; r < nranks; ++r) {
+      in[r] = static_cast<const char*>(send[r]);
+      out[r] = static_cast<char*>(recv[r]);
+    }
+    return launch_ring_cta(in, out, nranks, count, dtype, op, true, S(stream));
+  }
   if (algo == COLL_ALGO_RING_CLUSTER || algo == COLL_ALGO_RING_CTA || algo == COLL_ALGO_RING_LANE) {
     const bool has_ws = workspace != nullptr && workspace_bytes >= 24;
     const bool cta = algo == COLL_ALGO_RING_CTA;
@@ -440,7 +451,7 @@ int coll_all_reduce(const void* const* send, void* const* recv, int nranks, size
       }
       int* status = has_ws ? reinterpret_cast<int*>(static_cast<char*>(workspace) + 16) : nullptr;
       if (lane) return launch_ring_lane(in, out, nranks, count, dtype, op, S(stream));
-      return cta ? launch_ring_cta(in, out, nranks, count, dtype, op, status, S(stream))
+      return cta ? launch_ring_cta(in, out, nranks, count, dtype, op, false, S(stream))
                  : launch_ring_cluster(in, out, nranks, count, dtype, op, status, S(stream));
     }
     // no one-launch form: the stream-ordered steps, given a RING-sized workspace

@@ -69,7 +69,7 @@ bool ring_lane_supported(int n);
 int launch_ring_lane(const char* const* in, char* const* out, int n, size_t count, coll_dtype_t dt, coll_op_t op,
                      cudaStream_t s);
 int launch_ring_cta(const char* const* in, char* const* out, int n, size_t count, coll_dtype_t dt, coll_op_t op,
-                    int* status, cudaStream_t s);
+                    bool wire, cudaStream_t s);
 int launch_wait_flag(const uint32_t* flag, uint32_t expect, uint32_t budget_us, int* status, cudaStream_t s);
 
 // ---------------------------------------------------------------- copies ----

@@ -84,13 +84,16 @@ __device__ __forceinline__ void cp_async_wait_n() {
 
 // NR: the rank count at compile time (its loops unrolled and its waits
 // immediate), or 0 for any count in 2..8.  D: the register prefetch distance
-// in steps, or 0 for the cp.async cells.
-template <int DT, int OP, int MINB, typename OFF, int NR, int D>
+// in steps, or 0 for the cp.async cells.  WIRE: the reduce-scatter hops carry
+// the partial rounded to the storage type (RING_WIRE) instead of fp32 /
+// int32 (RING): each receiver widens it, adds its own values and rounds
+// again before passing it on.
+template <int DT, int OP, int MINB, typename OFF, int NR, int D, bool WIRE>
 __global__ void __launch_bounds__(kRtMaxRanks * 32, MINB) k_ring_cta(const __grid_constant__ RingCtaArgs a) {
   static_assert(D == 0 || (NR > 0 && NR % D == 0), "register slots repeat every tile");
   using A = typename Elem<DT>::A;
   constexpr int VN = Vec<DT>::kN;  // elements per 16-byte vector
-  constexpr int NQ = VN / 4;       // 16-byte pieces of a vector's fp32 / int32 partials
+  constexpr int NQ = WIRE ? 1 : VN / 4;  // 16-byte pieces a reduce-scatter hop carries per lane
   constexpr int ES = Elem<DT>::kSize;
   constexpr uint64_t TE = 32ull * VN;    // elements of one chunk per tile
   constexpr uint32_t kSlotU4 = 32 * NQ;  // one warp's hop slot, in 16-byte units
@@ -241,18 +244,29 @@ __global__ void __launch_bounds__(kRtMaxRanks * 32, MINB) k_ring_cta(const __gri
 #pragma unroll
       for (int k = 1; k < KMAX; ++k) {
         if (k >= n) break;
+        if constexpr (WIRE) {
+          Vec<DT> v;
 #pragma unroll
-        for (int q = 0; q < NQ; ++q)
-          tx[bo + q * 32] = make_uint4(a_to_bits<DT>(p[4 * q]), a_to_bits<DT>(p[4 * q + 1]),
-                                       a_to_bits<DT>(p[4 * q + 2]), a_to_bits<DT>(p[4 * q + 3]));
-        __syncthreads();
+          for (int i = 0; i < VN; ++i) v.v[i] = p[i];
+          tx[bo] = narrow16<DT>(v);  // the hop's rounding
+          __syncthreads();
+          widen16<DT>(rx[bo], v);
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-          const uint4 x = rx[bo + q * 32];
-          p[4 * q] = a_from_bits<DT>(x.x);
-          p[4 * q + 1] = a_from_bits<DT>(x.y);
-          p[4 * q + 2] = a_from_bits<DT>(x.z);
-          p[4 * q + 3] = a_from_bits<DT>(x.w);
+          for (int i = 0; i < VN; ++i) p[i] = v.v[i];
+        } else {
+#pragma unroll
+          for (int q = 0; q < NQ; ++q)
+            tx[bo + q * 32] = make_uint4(a_to_bits<DT>(p[4 * q]), a_to_bits<DT>(p[4 * q + 1]),
+                                         a_to_bits<DT>(p[4 * q + 2]), a_to_bits<DT>(p[4 * q + 3]));
+          __syncthreads();
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) {
+            const uint4 x = rx[bo + q * 32];
+            p[4 * q] = a_from_bits<DT>(x.x);
+            p[4 * q + 1] = a_from_bits<DT>(x.y);
+            p[4 * q + 2] = a_from_bits<DT>(x.z);
+            p[4 * q + 3] = a_from_bits<DT>(x.w);
+          }
         }
         bo = bo == 0 ? other : 0;
         Vec<DT> w;
@@ -294,7 +308,7 @@ __global__ void __launch_bounds__(kRtMaxRanks * 32, MINB) k_ring_cta(const __gri
     out_t += step_b;
   }
   cp_async_wait_n<0>();  // nothing of this CTA's is still being copied when it leaves
-  if (blockIdx.x == 0 && r == 0) ring_tail<DT, OP>(a, t);
+  if (blockIdx.x == 0 && r == 0) ring_tail<DT, OP, WIRE>(a, t);
 }
 
 template <int DT>
@@ -303,10 +317,10 @@ static uint64_t ring_cta_tiles(uint64_t seg) {
   return std::max<uint64_t>(1, (seg + per_tile - 1) / per_tile);
 }
 
-template <int DT, int OP, int MINB, typename OFF, int NR, int D>
+template <int DT, int OP, int MINB, typename OFF, int NR, int D, bool WIRE>
 static int launch_ring_cta_t(RingCtaArgs a, cudaStream_t s) {
   constexpr int VN = Vec<DT>::kN;
-  constexpr int NQ = VN / 4;
+  constexpr int NQ = WIRE ? 1 : VN / 4;
   const uint64_t per_tile = 32ull * VN;
   a.tiles = ring_cta_tiles<DT>(a.seg);
   // the last chunk is the shortest (possibly empty): a tile is full in every
@@ -317,37 +331,49 @@ static int launch_ring_cta_t(RingCtaArgs a, cudaStream_t s) {
   const size_t smem = (2ull * NQ + (D > 0 ? 0 : a.n)) * a.n * 32 * 16;
   static int smem_set[COLL_MAX_RANKS] = {0};  // per device ordinal: largest limit set so far
   const int st =
-      allow_dynamic_smem(reinterpret_cast<const void*>(k_ring_cta<DT, OP, MINB, OFF, NR, D>), smem, smem_set);
+      allow_dynamic_smem(reinterpret_cast<const void*>(k_ring_cta<DT, OP, MINB, OFF, NR, D, WIRE>), smem, smem_set);
   if (st != COLL_OK) return st;
   const uint64_t grid = std::min<uint64_t>(a.tiles, static_cast<uint64_t>(num_sms()) * MINB);
-  launch_pdl(k_ring_cta<DT, OP, MINB, OFF, NR, D>, dim3(static_cast<unsigned>(grid)), dim3(32 * a.n), smem, s, a);
+  launch_pdl(k_ring_cta<DT, OP, MINB, OFF, NR, D, WIRE>, dim3(static_cast<unsigned>(grid)), dim3(32 * a.n), smem, s,
+             a);
   return launch_status(cudaGetLastError());
 }
 
-template <int DT, int OP>
+template <int DT, int OP, bool WIRE>
 static int launch_ring_cta_op(const RingCtaArgs& a, cudaStream_t s) {
   // byte offsets within one rank's buffer fit 32 bits below 4 GiB
   const uint64_t span = static_cast<uint64_t>(a.n) * a.seg * Elem<DT>::kSize;
-  if (span >= (1ull << 32)) return launch_ring_cta_t<DT, OP, 3, uint64_t, 0, 0>(a, s);
+  if (span >= (1ull << 32)) return launch_ring_cta_t<DT, OP, 3, uint64_t, 0, 0, WIRE>(a, s);
   // eight ranks (the workloads' count) get the fully unrolled kernel: with
   // register prefetch when a CTA walks several tiles (measured on B200 at
   // 3.5 MiB per rank: 12.97 against 13.64 us; 256 MiB: 717 against 764 us),
   // with the cells when every CTA holds one tile (1 MiB: 5.21 against 5.47)
   if (a.n == 8) {
     const uint64_t slots = static_cast<uint64_t>(num_sms()) * 4;
-    if (ring_cta_tiles<DT>(a.seg) > slots) return launch_ring_cta_t<DT, OP, 4, uint32_t, 8, 4>(a, s);
-    return launch_ring_cta_t<DT, OP, 4, uint32_t, 8, 0>(a, s);
+    if (ring_cta_tiles<DT>(a.seg) > slots) return launch_ring_cta_t<DT, OP, 4, uint32_t, 8, 4, WIRE>(a, s);
+    return launch_ring_cta_t<DT, OP, 4, uint32_t, 8, 0, WIRE>(a, s);
   }
-  return launch_ring_cta_t<DT, OP, 4, uint32_t, 0, 0>(a, s);
+  return launch_ring_cta_t<DT, OP, 4, uint32_t, 0, 0, WIRE>(a, s);
+}
+
+// Rounding a partial to the storage type changes nothing for fp32 / int32
+// (storage = arithmetic type) or for MAX / MIN (the winner's own bits), so
+// RING_WIRE runs the fp32 ring's kernels there.
+template <int DT, int OP>
+static int launch_ring_cta_wire(const RingCtaArgs& a, bool wire, cudaStream_t s) {
+  if constexpr ((DT == COLL_BF16 || DT == COLL_FP16) && (OP == COLL_SUM || OP == COLL_PROD)) {
+    if (wire) return launch_ring_cta_op<DT, OP, true>(a, s);
+  }
+  return launch_ring_cta_op<DT, OP, false>(a, s);
 }
 
 template <int DT>
-static int launch_ring_cta_dt(const RingCtaArgs& a, coll_op_t op, cudaStream_t s) {
+static int launch_ring_cta_dt(const RingCtaArgs& a, coll_op_t op, bool wire, cudaStream_t s) {
   switch (op) {
-    case COLL_SUM: return launch_ring_cta_op<DT, COLL_SUM>(a, s);
-    case COLL_MAX: return launch_ring_cta_op<DT, COLL_MAX>(a, s);
-    case COLL_MIN: return launch_ring_cta_op<DT, COLL_MIN>(a, s);
-    case COLL_PROD: return launch_ring_cta_op<DT, COLL_PROD>(a, s);
+    case COLL_SUM: return launch_ring_cta_wire<DT, COLL_SUM>(a, wire, s);
+    case COLL_MAX: return launch_ring_cta_wire<DT, COLL_MAX>(a, wire, s);
+    case COLL_MIN: return launch_ring_cta_wire<DT, COLL_MIN>(a, wire, s);
+    case COLL_PROD: return launch_ring_cta_wire<DT, COLL_PROD>(a, wire, s);
   }
   return COLL_ERR_UNSUPPORTED;
 }
@@ -355,8 +381,7 @@ static int launch_ring_cta_dt(const RingCtaArgs& a, coll_op_t op, cudaStream_t s
 bool ring_cta_supported(int n) { return n >= 2 && n <= kRtMaxRanks; }
 
 int launch_ring_cta(const char* const* in, char* const* out, int n, size_t count, coll_dtype_t dt, coll_op_t op,
-                    int* status, cudaStream_t s) {
-  (void)status;  // nothing in this form waits, so it never raises a status
+                    bool wire, cudaStream_t s) {
   RingCtaArgs a{};
   for (int r = 0; r < n; ++r) {
     a.in[r] = in[r];
@@ -368,10 +393,10 @@ int launch_ring_cta(const char* const* in, char* const* out, int n, size_t count
   a.count = count;
   a.n = n;
   switch (dt) {
-    case COLL_BF16: return launch_ring_cta_dt<COLL_BF16>(a, op, s);
-    case COLL_FP16: return launch_ring_cta_dt<COLL_FP16>(a, op, s);
-    case COLL_FP32: return launch_ring_cta_dt<COLL_FP32>(a, op, s);
-    case COLL_INT32: return launch_ring_cta_dt<COLL_INT32>(a, op, s);
+    case COLL_BF16: return launch_ring_cta_dt<COLL_BF16>(a, op, wire, s);
+    case COLL_FP16: return launch_ring_cta_dt<COLL_FP16>(a, op, wire, s);
+    case COLL_FP32: return launch_ring_cta_dt<COLL_FP32>(a, op, wire, s);
+    case COLL_INT32: return launch_ring_cta_dt<COLL_INT32>(a, op, wire, s);
   }
   return COLL_ERR_UNSUPPORTED;
 }

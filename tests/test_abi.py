@@ -153,7 +153,11 @@ def test_all_reduce_form():
     assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING_LANE, 0) == M.RING_STEPS
     assert L.coll_all_reduce_form(9, 1000, M.BF16, M.RING_LANE, 1) == M.RING_STEPS
     assert L.coll_all_reduce_form(3, 1000, M.BF16, M.RING_LANE, 1) == M.RING_LANE
-    assert L.coll_all_reduce_form(8, 1000, M.BF16, 11, 1) == -2
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING_WIRE, 1) == M.RING_WIRE
+    assert L.coll_all_reduce_form(2, 1 << 30, M.FP32, M.RING_WIRE, 1) == M.RING_WIRE
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, M.RING_WIRE, 0) == -2  # no stream-ordered form
+    assert L.coll_all_reduce_form(9, 1000, M.BF16, M.RING_WIRE, 1) == -2
+    assert L.coll_all_reduce_form(8, 1000, M.BF16, 12, 1) == -2
     # RING and RING_STEPS: a 256-byte header, then 4 bytes of partial per element
     for algo in (M.RING, M.RING_STEPS):
         assert L.coll_all_reduce_workspace_size(8, 1000, M.BF16, algo) == 256 + 4096
@@ -186,7 +190,7 @@ def test_invalid_arguments_rejected_on_host():
     # unsupported dtype / op / algo
     assert L.coll_all_reduce(p, q, 4, 16, 9, M.SUM, M.TWOSHOT, None, 0, None) == -2
     assert L.coll_all_reduce(p, q, 4, 16, M.BF16, 9, M.TWOSHOT, None, 0, None) == -2
-    assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, 11, None, 0, None) == -2
+    assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, 12, None, 0, None) == -2
     assert L.coll_moe_combine(p, p, p, p, q, 4, 8, 2, 8, 16, M.INT32, 100, None, None) == -2
     # ring without workspace
     assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, M.RING, None, 0, None) == -5
@@ -203,6 +207,8 @@ def test_invalid_arguments_rejected_on_host():
     assert L.coll_all_reduce(p, q, 4, 1 << 16, M.BF16, M.SUM, M.RING_CTA, BASE + 0x100, 64, None) == -3
     assert L.coll_all_reduce(p9, q9, 9, 16, M.BF16, M.SUM, M.RING_LANE, None, 0, None) == -2
     assert L.coll_all_reduce(pu, q, 4, 16, M.BF16, M.SUM, M.RING_LANE, None, 0, None) == -2
+    assert L.coll_all_reduce(p9, q9, 9, 16, M.BF16, M.SUM, M.RING_WIRE, None, 0, None) == -2
+    assert L.coll_all_reduce(pu, q, 4, 16, M.BF16, M.SUM, M.RING_WIRE, None, 0, None) == -2
     assert L.coll_all_reduce(p, q, 4, 16, M.BF16, M.SUM, M.RING_LANE, BASE + 0x50000008, 64, None) == -5
     # fused LL two-shot: workspace missing, too small, or not 256-byte aligned
     need = L.coll_all_reduce_workspace_size(4, 16, M.BF16, M.TWOSHOT_LL)
