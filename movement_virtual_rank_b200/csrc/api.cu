@@ -3,6 +3,7 @@
 // kernel.  No entry point allocates memory or synchronises the stream.
 #include <algorithm>
 #include <atomic>
+#include <mutex>
 #include <cstdio>
 #include <cstring>
 #include <vector>
@@ -54,6 +55,35 @@ int num_sms() {
   if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
   cache[dev].store(v, std::memory_order_relaxed);
   return v;
+}
+
+// CTAs of `fn` that fit on the whole GPU at once (occupancy API), cached per
+// kernel and device.  A grid-stride kernel launched with more CTAs than fit
+// runs its extra CTAs as a short second wave after the first has finished
+// its share, so the element kernels' grids are capped here.
+int resident_ctas(const void* fn, int threads, size_t smem) {
+  struct Entry {
+    const void* fn;
+    int dev, threads, per_sm;
+  };
+  static Entry table[256];
+  static int used = 0;
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) dev = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+      if (table[i].fn == fn && table[i].dev == dev && table[i].threads == threads) return table[i].per_sm * num_sms();
+  }
+  int v = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, fn, threads, smem) != cudaSuccess || v <= 0) {
+    (void)cudaGetLastError();
+    return num_sms() * 8;  // the grids' own cap; the launch reports any real error
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (used < 256) table[used++] = Entry{fn, dev, threads, v};
+  return v * num_sms();
 }
 
 int elem_size(coll_dtype_t dt) {

@@ -14,6 +14,7 @@ constexpr int kMaxRanksH = COLL_MAX_RANKS;
 constexpr int kBlockThreads = 256;  // threads per CTA of the element-wise kernels
 
 int num_sms();                      // SM count of the current device (cached)
+int resident_ctas(const void* fn, int threads, size_t smem);  // CTAs of fn that fit at once on the device
 int elem_size(coll_dtype_t dt);     // 2 or 4, 0 for an unknown dtype
 int launch_status(cudaError_t e);   // COLL_OK or COLL_ERR_CUDA (remembers the error text)
 // Raise `fn`'s dynamic shared memory limit to at least `bytes` on the current

@@ -513,10 +513,13 @@ static int launch_combine_dt(const MoeMoveArgs& a, cudaStream_t s) {
   const int64_t rows = static_cast<int64_t>(a.n) * a.tokens;
   uint64_t bits = a.row_bytes;
   for (int r = 0; r < a.n; ++r) bits |= reinterpret_cast<uintptr_t>(a.x[r]) | reinterpret_cast<uintptr_t>(a.y[r]);
-  const unsigned grid = move_grid(rows);
-  if ((bits & 15) == 0 && a.topk == 8) launch_pdl(k_moe_combine<DT, true, 8>, dim3(grid), dim3(kMoveThreads), 0, s, a);
-  else if ((bits & 15) == 0) launch_pdl(k_moe_combine<DT, true, 0>, dim3(grid), dim3(kMoveThreads), 0, s, a);
-  else launch_pdl(k_moe_combine<DT, false, 0>, dim3(grid), dim3(kMoveThreads), 0, s, a);
+  void (*fn)(MoeMoveArgs) = (bits & 15) == 0 && a.topk == 8 ? k_moe_combine<DT, true, 8>
+                            : (bits & 15) == 0                ? k_moe_combine<DT, true, 0>
+                                                              : k_moe_combine<DT, false, 0>;
+  // a CTA per token row, no more CTAs than fit at once
+  const int64_t cap = resident_ctas(reinterpret_cast<const void*>(fn), kMoveThreads, 0);
+  const unsigned grid = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(rows, cap)));
+  launch_pdl(fn, dim3(grid), dim3(kMoveThreads), 0, s, a);
   return launch_status(cudaGetLastError());
 }
 

@@ -19,9 +19,10 @@
 
 namespace mvr {
 
-static unsigned grid_units(uint64_t units) {
+// CTAs for `units` threads' work of kernel `fn`: no more than fit at once
+static unsigned grid_units(uint64_t units, const void* fn) {
   uint64_t want = (units + kThreads - 1) / kThreads;
-  const uint64_t cap = static_cast<uint64_t>(num_sms()) * 8;
+  const uint64_t cap = static_cast<uint64_t>(resident_ctas(fn, kThreads, 0));
   if (want > cap) want = cap;
   if (want < 1) want = 1;
   return static_cast<unsigned>(want);
@@ -339,11 +340,11 @@ __global__ void __launch_bounds__(32) k_ll_pack_tma(const __grid_constant__ Code
 }
 
 // The codec grid for n ranks of `units` work items each: one CTA row per
-// rank, at most 8 CTAs per SM in all
-static dim3 codec_grid(uint64_t units, int n) {
+// rank, no more CTAs in all than fit at once
+static dim3 codec_grid(uint64_t units, int n, const void* fn) {
   const unsigned gy = static_cast<unsigned>(n);
   uint64_t gx = (units + kThreads - 1) / kThreads;
-  uint64_t cap = static_cast<uint64_t>(num_sms()) * 8 / gy;
+  uint64_t cap = static_cast<uint64_t>(resident_ctas(fn, kThreads, 0)) / gy;
   if (cap < 1) cap = 1;
   if (gx > cap) gx = cap;
   if (gx < 1) gx = 1;
@@ -389,11 +390,11 @@ int launch_ll_pack(const CodecArgs& a0, int proto, cudaStream_t s) {
   }
   if (proto == COLL_PROTO_LL) {
     const uint64_t nlines = (a.bytes + 3) / 4;
-    launch_pdl(k_ll_pack, codec_grid(nlines / 4 + 1, a.n), block, 0, s, a,
+    launch_pdl(k_ll_pack, codec_grid(nlines / 4 + 1, a.n, reinterpret_cast<const void*>(k_ll_pack)), block, 0, s, a,
                static_cast<int>((msg & 15) == 0));
   } else {
     const uint64_t nlines = (a.bytes + 119) / 120;
-    launch_pdl(k_ll128_pack, codec_grid(nlines * 8, a.n), block, 0, s, a,
+    launch_pdl(k_ll128_pack, codec_grid(nlines * 8, a.n, reinterpret_cast<const void*>(k_ll128_pack)), block, 0, s, a,
                static_cast<int>((msg & 7) == 0), static_cast<int>(((msg | pkt) & 15) == 0));
   }
   return launch_status(cudaGetLastError());
@@ -406,11 +407,11 @@ int launch_ll_unpack(const CodecArgs& a, int proto, cudaStream_t s) {
   const dim3 block(kThreads);
   if (proto == COLL_PROTO_LL) {
     const uint64_t nlines = (a.bytes + 3) / 4;
-    launch_pdl(k_ll_unpack, codec_grid(nlines / 4 + 1, a.n), block, 0, s, a,
+    launch_pdl(k_ll_unpack, codec_grid(nlines / 4 + 1, a.n, reinterpret_cast<const void*>(k_ll_unpack)), block, 0, s, a,
                static_cast<int>((msg & 15) == 0));
   } else {
     const uint64_t nlines = (a.bytes + 119) / 120;
-    launch_pdl(k_ll128_unpack, codec_grid(nlines * 8, a.n), block, 0, s, a,
+    launch_pdl(k_ll128_unpack, codec_grid(nlines * 8, a.n, reinterpret_cast<const void*>(k_ll128_unpack)), block, 0, s, a,
                static_cast<int>((msg & 7) == 0), static_cast<int>(((msg | pkt) & 15) == 0));
   }
   return launch_status(cudaGetLastError());
@@ -576,13 +577,21 @@ static int launch_ar_packed_t(const PackedReduceArgs& a, int proto, cudaStream_t
   // the 8-rank sum (the workloads' rank count) issues its eight loads at once
   const bool eight = a.n == 8 && OP == COLL_SUM;
   if (proto == COLL_PROTO_LL) {
-    const dim3 grid(grid_units(a.nlines / 2 + 1));
-    if (eight) launch_pdl(k_ar_ll<DT, OP, 8>, grid, dim3(kThreads), 0, s, a);
-    else launch_pdl(k_ar_ll<DT, OP, 0>, grid, dim3(kThreads), 0, s, a);
+    if (eight)
+      launch_pdl(k_ar_ll<DT, OP, 8>, dim3(grid_units(a.nlines / 2 + 1, reinterpret_cast<const void*>(k_ar_ll<DT, OP, 8>))),
+                 dim3(kThreads), 0, s, a);
+    else
+      launch_pdl(k_ar_ll<DT, OP, 0>, dim3(grid_units(a.nlines / 2 + 1, reinterpret_cast<const void*>(k_ar_ll<DT, OP, 0>))),
+                 dim3(kThreads), 0, s, a);
   } else {
-    const dim3 grid(grid_units(a.nlines * 8));
-    if (eight) launch_pdl(k_ar_ll128<DT, OP, 8>, grid, dim3(kThreads), 0, s, a);
-    else launch_pdl(k_ar_ll128<DT, OP, 0>, grid, dim3(kThreads), 0, s, a);
+    if (eight)
+      launch_pdl(k_ar_ll128<DT, OP, 8>,
+                 dim3(grid_units(a.nlines * 8, reinterpret_cast<const void*>(k_ar_ll128<DT, OP, 8>))), dim3(kThreads), 0,
+                 s, a);
+    else
+      launch_pdl(k_ar_ll128<DT, OP, 0>,
+                 dim3(grid_units(a.nlines * 8, reinterpret_cast<const void*>(k_ar_ll128<DT, OP, 0>))), dim3(kThreads), 0,
+                 s, a);
   }
   return launch_status(cudaGetLastError());
 }

@@ -18,6 +18,8 @@
 // one tile close together in time, so the repeated reads hit L2).
 #pragma once
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -212,22 +214,26 @@ __global__ void __launch_bounds__(kThreads) k_ring_rs(const __grid_constant__ Ri
 
 template <int DT, int OP, int NR>
 int launch_reduce_nr(const ReduceArgs& a, int mode, bool vec, int bps, cudaStream_t s) {
-  const dim3 grid(static_cast<unsigned>(a.nslices * bps));
+  void (*fn)(ReduceArgs) = nullptr;
   if (vec) {
     switch (mode) {
-      case M_ALL: launch_pdl(k_reduce_vec<DT, OP, NR, M_ALL>, dim3(grid), dim3(kThreads), 0, s, a); break;
-      case M_BLOCK: launch_pdl(k_reduce_vec<DT, OP, NR, M_BLOCK>, dim3(grid), dim3(kThreads), 0, s, a); break;
-      case M_SAME: launch_pdl(k_reduce_vec<DT, OP, NR, M_SAME>, dim3(grid), dim3(kThreads), 0, s, a); break;
-      default: launch_pdl(k_reduce_vec<DT, OP, NR, M_ONESHOT>, dim3(grid), dim3(kThreads), 0, s, a); break;
+      case M_ALL: fn = k_reduce_vec<DT, OP, NR, M_ALL>; break;
+      case M_BLOCK: fn = k_reduce_vec<DT, OP, NR, M_BLOCK>; break;
+      case M_SAME: fn = k_reduce_vec<DT, OP, NR, M_SAME>; break;
+      default: fn = k_reduce_vec<DT, OP, NR, M_ONESHOT>; break;
     }
   } else {
     switch (mode) {
-      case M_ALL: launch_pdl(k_reduce_scalar<DT, OP, M_ALL>, dim3(grid), dim3(kThreads), 0, s, a); break;
-      case M_BLOCK: launch_pdl(k_reduce_scalar<DT, OP, M_BLOCK>, dim3(grid), dim3(kThreads), 0, s, a); break;
-      case M_SAME: launch_pdl(k_reduce_scalar<DT, OP, M_SAME>, dim3(grid), dim3(kThreads), 0, s, a); break;
-      default: launch_pdl(k_reduce_scalar<DT, OP, M_ONESHOT>, dim3(grid), dim3(kThreads), 0, s, a); break;
+      case M_ALL: fn = k_reduce_scalar<DT, OP, M_ALL>; break;
+      case M_BLOCK: fn = k_reduce_scalar<DT, OP, M_BLOCK>; break;
+      case M_SAME: fn = k_reduce_scalar<DT, OP, M_SAME>; break;
+      default: fn = k_reduce_scalar<DT, OP, M_ONESHOT>; break;
     }
   }
+  // no more CTAs than fit at once (the slices stay interleaved: a multiple of nslices)
+  const int res = resident_ctas(reinterpret_cast<const void*>(fn), kThreads, 0);
+  if (static_cast<int64_t>(a.nslices) * bps > res) bps = std::max(1, res / a.nslices);
+  launch_pdl(fn, dim3(static_cast<unsigned>(a.nslices * bps)), dim3(kThreads), 0, s, a);
   return launch_status(cudaGetLastError());
 }
 
