@@ -135,7 +135,9 @@ def test_ll_sweep_sizes(log2):
     packed output compared on the device with the packed Simple result, and
     every line of it against the oracle's packetised all-reduce.  The oracle
     runs on chunks of whole lines (each line of the result depends only on
-    the same line of every rank's packets), so host memory stays bounded."""
+    the same line of every rank's packets), so host memory stays bounded.
+    Every rank's Simple output equals rank 0's, and the one-launch codecs for
+    all ranks give the one-rank calls' bytes, encoding and decoding."""
     need_gpu()
     n, nbytes = 8, 1 << log2
     count = nbytes // 2
@@ -143,12 +145,20 @@ def test_ll_sweep_sizes(log2):
     send = [to_dev(x, "bf16") for x in xs]
     simple = [torch.empty_like(t) for t in send]
     M.coll_all_reduce(send, simple, algo=M.TWOSHOT)
+    for q in range(1, n):
+        assert torch.equal(simple[q].view(torch.int16), simple[0].view(torch.int16)), q
     for proto in (M.LL, M.LL128):
         step = log2 + 1
         pb = M.coll_packed_bytes(nbytes, proto)
         packed = [torch.empty(pb, dtype=torch.uint8, device="cuda") for _ in range(n)]
         for r in range(n):
             M.coll_ll_pack(send[r], packed[r], proto, step)
+        together = [torch.empty(pb, dtype=torch.uint8, device="cuda") for _ in range(n)]
+        M.coll_ll_pack_ranks(send, together, proto, step)
+        torch.cuda.synchronize()
+        for r in range(n):
+            assert torch.equal(together[r], packed[r]), r
+        del together
         out = [torch.empty(pb, dtype=torch.uint8, device="cuda") for _ in range(n)]
         st = status_tensor()
         M.coll_all_reduce_packed(packed, out, count, torch.bfloat16, proto, step, status=st)
@@ -161,7 +171,13 @@ def test_ll_sweep_sizes(log2):
         for q in range(n):
             assert torch.equal(out[q], ref)
         assert torch.equal(dec.view(torch.int16), simple[0].view(torch.int16))
-        del packed, ref, dec
+        decs = [torch.empty_like(send[0]) for _ in range(n)]
+        M.coll_ll_unpack_ranks(out, decs, proto, step, status=st)
+        torch.cuda.synchronize()
+        assert st.tolist() == [0, 0]
+        for q in range(n):
+            assert torch.equal(decs[q].view(torch.int16), simple[0].view(torch.int16)), q
+        del packed, ref, dec, decs
         line = 8 if proto == M.LL else 128
         per = 2 if proto == M.LL else 60  # bf16 elements of payload per line
         nl = pb // line
