@@ -45,6 +45,10 @@ int main(void) {
   CHECK(coll_all_reduce_form(8, 1000, COLL_BF16, COLL_ALGO_AUTO, 1) == COLL_ALGO_TWOSHOT);
   CHECK(coll_all_reduce_form(8, 1000, COLL_BF16, COLL_ALGO_RING, 1) == COLL_ALGO_RING_LANE);
   CHECK(coll_all_reduce_form(8, 1 << 20, COLL_BF16, COLL_ALGO_RING, 1) == COLL_ALGO_RING_CTA);
+  CHECK(coll_all_reduce_form(8, 1000, COLL_BF16, COLL_ALGO_RING_WIRE, 1) == COLL_ALGO_RING_WIRE);
+  CHECK(coll_all_reduce_form(8, 1000, COLL_BF16, COLL_ALGO_RING_WIRE, 0) == COLL_ERR_UNSUPPORTED);
+  CHECK(coll_ll_pack_ranks(NULL, NULL, 4, 16, COLL_PROTO_LL, 1, NULL) == COLL_ERR_INVALID_ARG);
+  CHECK(coll_ll_unpack_ranks(NULL, NULL, 4, 16, COLL_PROTO_LL128, 1, NULL, NULL) == COLL_ERR_INVALID_ARG);
   CHECK(coll_all_reduce_form(8, 1000, COLL_BF16, COLL_ALGO_RING, 0) == COLL_ALGO_RING_STEPS);
   CHECK(coll_all_reduce_form(9, 1000, COLL_BF16, COLL_ALGO_RING, 1) == COLL_ALGO_RING_STEPS);
   CHECK(coll_moe_route_workspace_size(8, 4096, 8, 256) > 0);
