@@ -263,7 +263,9 @@ def coll_all_reduce(send, recv, op="sum", algo=TWOSHOT, workspace: torch.Tensor 
     RING_LL / TWOSHOT_LL / TWOSHOT_LL128 use) and get a zeroed one allocated here when it
     is omitted;
     RING_CLUSTER uses one, when given, for its status pair and its fallback
-    to RING_STEPS; RING_CTA and RING_LANE only for that fallback."""
+    to RING_STEPS; RING_CTA and RING_LANE only for that fallback; RING_WIRE
+    ignores it (it has no fallback: unaligned buffers or more than 8 ranks
+    raise)."""
     algo = ALGOS[algo] if isinstance(algo, str) else int(algo)
     send = _ranks(send, "send", send[0].dtype)
     recv = _ranks(recv, "recv", send[0].dtype)
