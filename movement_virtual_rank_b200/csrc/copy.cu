@@ -35,11 +35,10 @@ static int pick_unit(uint64_t bits) {
   return 1;
 }
 
+// one unit per thread for each of `slices` slices, the slices interleaved
 static unsigned grid_for(uint64_t units, int slices) {
-  uint64_t want = (units + kThreads - 1) / kThreads;
-  const uint64_t cap = std::max<uint64_t>(1, static_cast<uint64_t>(num_sms()) * 8 / std::max(1, slices));
-  want = std::min(want, cap);
-  return static_cast<unsigned>(std::max<uint64_t>(1, want) * slices);
+  const uint64_t per = std::min<uint64_t>(stream_grid(units, kThreads), kMaxStreamGrid / std::max(1, slices));
+  return static_cast<unsigned>(per * slices);
 }
 
 // ------------------------------------------------------------- fan-out ----
@@ -339,11 +338,8 @@ int launch_copy_jobs(const CopyJob* jobs, int njobs, cudaStream_t s) {
                               : U == 4  ? k_copy_jobs<4>
                               : U == 2  ? k_copy_jobs<2>
                                         : k_copy_jobs<1>;
-    // about one unit per thread (latency first), no more CTAs than fit at once
-    uint64_t want = (acc + kThreads - 1) / kThreads;
-    want = std::min<uint64_t>(std::max<uint64_t>(want, 1),
-                              static_cast<uint64_t>(resident_ctas(reinterpret_cast<const void*>(fn), kThreads, 0)));
-    launch_pdl(fn, dim3(static_cast<unsigned>(want)), dim3(kThreads), 0, s, args);
+    // about one unit per thread, CTAs launched in order
+    launch_pdl(fn, dim3(static_cast<unsigned>(stream_grid(acc, kThreads))), dim3(kThreads), 0, s, args);
     const int st = launch_status(cudaGetLastError());
     if (st != COLL_OK) return st;
   }

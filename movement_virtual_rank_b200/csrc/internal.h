@@ -15,6 +15,8 @@ constexpr int kBlockThreads = 256;  // threads per CTA of the element-wise kerne
 
 int num_sms();                      // SM count of the current device (cached)
 int resident_ctas(const void* fn, int threads, size_t smem);  // CTAs of fn that fit at once on the device
+constexpr uint64_t kMaxStreamGrid = 1ull << 30;  // CTAs of one streaming launch at most
+uint64_t stream_grid(uint64_t units, int threads);  // one work item per thread, at most kMaxStreamGrid CTAs
 int elem_size(coll_dtype_t dt);     // 2 or 4, 0 for an unknown dtype
 int launch_status(cudaError_t e);   // COLL_OK or COLL_ERR_CUDA (remembers the error text)
 // Raise `fn`'s dynamic shared memory limit to at least `bytes` on the current

@@ -516,9 +516,8 @@ static int launch_combine_dt(const MoeMoveArgs& a, cudaStream_t s) {
   void (*fn)(MoeMoveArgs) = (bits & 15) == 0 && a.topk == 8 ? k_moe_combine<DT, true, 8>
                             : (bits & 15) == 0                ? k_moe_combine<DT, true, 0>
                                                               : k_moe_combine<DT, false, 0>;
-  // a CTA per token row, no more CTAs than fit at once
-  const int64_t cap = resident_ctas(reinterpret_cast<const void*>(fn), kMoveThreads, 0);
-  const unsigned grid = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(rows, cap)));
+  // a CTA per token row, launched in order
+  const unsigned grid = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(rows, kMaxStreamGrid)));
   launch_pdl(fn, dim3(grid), dim3(kMoveThreads), 0, s, a);
   return launch_status(cudaGetLastError());
 }

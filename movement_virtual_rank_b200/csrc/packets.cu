@@ -19,14 +19,8 @@
 
 namespace mvr {
 
-// CTAs for `units` threads' work of kernel `fn`: no more than fit at once
-static unsigned grid_units(uint64_t units, const void* fn) {
-  uint64_t want = (units + kThreads - 1) / kThreads;
-  const uint64_t cap = static_cast<uint64_t>(resident_ctas(fn, kThreads, 0));
-  if (want > cap) want = cap;
-  if (want < 1) want = 1;
-  return static_cast<unsigned>(want);
-}
+// CTAs for `units` threads' work: one work item per thread
+static unsigned grid_units(uint64_t units) { return static_cast<unsigned>(stream_grid(units, kThreads)); }
 
 // little-endian bytes [off, off+len) of src, zero beyond `bytes`, as a u32/u64
 __device__ __forceinline__ uint32_t load_word_tail(const uint8_t* src, uint64_t off, uint64_t bytes) {
@@ -340,7 +334,8 @@ __global__ void __launch_bounds__(32) k_ll_pack_tma(const __grid_constant__ Code
 }
 
 // The codec grid for n ranks of `units` work items each: one CTA row per
-// rank, no more CTAs in all than fit at once
+// rank, no more CTAs in all than fit at once (the warps walk several line
+// groups each; one work item per thread measured 20-60% slower here)
 static dim3 codec_grid(uint64_t units, int n, const void* fn) {
   const unsigned gy = static_cast<unsigned>(n);
   uint64_t gx = (units + kThreads - 1) / kThreads;
@@ -578,19 +573,19 @@ static int launch_ar_packed_t(const PackedReduceArgs& a, int proto, cudaStream_t
   const bool eight = a.n == 8 && OP == COLL_SUM;
   if (proto == COLL_PROTO_LL) {
     if (eight)
-      launch_pdl(k_ar_ll<DT, OP, 8>, dim3(grid_units(a.nlines / 2 + 1, reinterpret_cast<const void*>(k_ar_ll<DT, OP, 8>))),
+      launch_pdl(k_ar_ll<DT, OP, 8>, dim3(grid_units(a.nlines / 2 + 1)),
                  dim3(kThreads), 0, s, a);
     else
-      launch_pdl(k_ar_ll<DT, OP, 0>, dim3(grid_units(a.nlines / 2 + 1, reinterpret_cast<const void*>(k_ar_ll<DT, OP, 0>))),
+      launch_pdl(k_ar_ll<DT, OP, 0>, dim3(grid_units(a.nlines / 2 + 1)),
                  dim3(kThreads), 0, s, a);
   } else {
     if (eight)
       launch_pdl(k_ar_ll128<DT, OP, 8>,
-                 dim3(grid_units(a.nlines * 8, reinterpret_cast<const void*>(k_ar_ll128<DT, OP, 8>))), dim3(kThreads), 0,
+                 dim3(grid_units(a.nlines * 8)), dim3(kThreads), 0,
                  s, a);
     else
       launch_pdl(k_ar_ll128<DT, OP, 0>,
-                 dim3(grid_units(a.nlines * 8, reinterpret_cast<const void*>(k_ar_ll128<DT, OP, 0>))), dim3(kThreads), 0,
+                 dim3(grid_units(a.nlines * 8)), dim3(kThreads), 0,
                  s, a);
   }
   return launch_status(cudaGetLastError());

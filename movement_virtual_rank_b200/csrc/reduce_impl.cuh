@@ -230,9 +230,14 @@ int launch_reduce_nr(const ReduceArgs& a, int mode, bool vec, int bps, cudaStrea
       default: fn = k_reduce_scalar<DT, OP, M_ONESHOT>; break;
     }
   }
-  // no more CTAs than fit at once (the slices stay interleaved: a multiple of nslices)
-  const int res = resident_ctas(reinterpret_cast<const void*>(fn), kThreads, 0);
-  if (static_cast<int64_t>(a.nslices) * bps > res) bps = std::max(1, res / a.nslices);
+  // one vector per thread (blocks_per_slice), the slices interleaved; the
+  // one-shot keeps a resident grid, so that the N readers of a tile run
+  // together and L2 serves the repeats (a full grid measured 17.4 -> 20.1 us
+  // at 8 x 3.5 MiB)
+  if (mode == M_ONESHOT) {
+    const int res = resident_ctas(reinterpret_cast<const void*>(fn), kThreads, 0);
+    if (static_cast<int64_t>(a.nslices) * bps > res) bps = std::max(1, res / a.nslices);
+  }
   launch_pdl(fn, dim3(static_cast<unsigned>(a.nslices * bps)), dim3(kThreads), 0, s, a);
   return launch_status(cudaGetLastError());
 }
