@@ -58,11 +58,10 @@ int num_sms() {
 }
 
 // CTAs of `fn` that fit on the whole GPU at once (occupancy API), cached per
-// kernel and device: the grid of the kernels that walk their data with a
-// resident grid (the packet codecs, whose warps take several line groups per
-// pass, and the one-shot all-reduce, whose N readers of a tile must run
-// together for L2 to serve the repeats).  A larger grid would run its extra
-// CTAs as a short second wave after the first had finished its share.
+// kernel and device: the grid of a kernel that walks its data with a resident
+// grid (the one-shot all-reduce, whose N readers of a tile must run together
+// for L2 to serve the repeats).  A larger grid would run its extra CTAs as a
+// short second wave after the first had finished its share.
 int resident_ctas(const void* fn, int threads, size_t smem) {
   struct Entry {
     const void* fn;

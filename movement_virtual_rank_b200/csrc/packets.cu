@@ -334,16 +334,15 @@ __global__ void __launch_bounds__(32) k_ll_pack_tma(const __grid_constant__ Code
 }
 
 // The codec grid for n ranks of `units` work items each: one CTA row per
-// rank, no more CTAs in all than fit at once (the warps walk several line
-// groups each; one work item per thread measured 20-60% slower here)
-static dim3 codec_grid(uint64_t units, int n, const void* fn) {
-  const unsigned gy = static_cast<unsigned>(n);
-  uint64_t gx = (units + kThreads - 1) / kThreads;
-  uint64_t cap = static_cast<uint64_t>(resident_ctas(fn, kThreads, 0)) / gy;
-  if (cap < 1) cap = 1;
-  if (gx > cap) gx = cap;
-  if (gx < 1) gx = 1;
-  return dim3(static_cast<unsigned>(gx), gy);
+// rank, about eight work items per thread, the CTAs launched in order.  The
+// warps walk several line groups each (for LL128, two per pass), so one item
+// per thread (20-60% slower) gives a CTA too little work, and a resident grid
+// walking the data with a stride measured 7-14% slower for the LL128 codecs
+// at 16 and 256 MiB per rank (LL128 pack at 8 x 256 MiB: 757 -> 651 us).
+static dim3 codec_grid(uint64_t units, int n) {
+  constexpr uint64_t kItemsPerThread = 8;
+  return dim3(static_cast<unsigned>(stream_grid((units + kItemsPerThread - 1) / kItemsPerThread, kThreads)),
+              static_cast<unsigned>(n));
 }
 
 // every message pointer's low bits, and every packet pointer's
@@ -385,11 +384,11 @@ int launch_ll_pack(const CodecArgs& a0, int proto, cudaStream_t s) {
   }
   if (proto == COLL_PROTO_LL) {
     const uint64_t nlines = (a.bytes + 3) / 4;
-    launch_pdl(k_ll_pack, codec_grid(nlines / 4 + 1, a.n, reinterpret_cast<const void*>(k_ll_pack)), block, 0, s, a,
+    launch_pdl(k_ll_pack, codec_grid(nlines / 4 + 1, a.n), block, 0, s, a,
                static_cast<int>((msg & 15) == 0));
   } else {
     const uint64_t nlines = (a.bytes + 119) / 120;
-    launch_pdl(k_ll128_pack, codec_grid(nlines * 8, a.n, reinterpret_cast<const void*>(k_ll128_pack)), block, 0, s, a,
+    launch_pdl(k_ll128_pack, codec_grid(nlines * 8, a.n), block, 0, s, a,
                static_cast<int>((msg & 7) == 0), static_cast<int>(((msg | pkt) & 15) == 0));
   }
   return launch_status(cudaGetLastError());
@@ -402,11 +401,11 @@ int launch_ll_unpack(const CodecArgs& a, int proto, cudaStream_t s) {
   const dim3 block(kThreads);
   if (proto == COLL_PROTO_LL) {
     const uint64_t nlines = (a.bytes + 3) / 4;
-    launch_pdl(k_ll_unpack, codec_grid(nlines / 4 + 1, a.n, reinterpret_cast<const void*>(k_ll_unpack)), block, 0, s, a,
+    launch_pdl(k_ll_unpack, codec_grid(nlines / 4 + 1, a.n), block, 0, s, a,
                static_cast<int>((msg & 15) == 0));
   } else {
     const uint64_t nlines = (a.bytes + 119) / 120;
-    launch_pdl(k_ll128_unpack, codec_grid(nlines * 8, a.n, reinterpret_cast<const void*>(k_ll128_unpack)), block, 0, s, a,
+    launch_pdl(k_ll128_unpack, codec_grid(nlines * 8, a.n), block, 0, s, a,
                static_cast<int>((msg & 7) == 0), static_cast<int>(((msg | pkt) & 15) == 0));
   }
   return launch_status(cudaGetLastError());
