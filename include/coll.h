@@ -217,8 +217,8 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    result) in one launch in which every CTA holds all N virtual ranks,
  *    one warp each: each hop is a store into a shared-memory slot of the
  *    same SM and one CTA-wide barrier, so the partials never leave the SM
- *    and nothing waits on another CTA.  The CTAs (up to four per SM) walk
- *    the message tile by tile.  Needs 2 <= N <= 8 and 16-byte aligned
+ *    and nothing waits on another CTA.  The grid has one CTA per tile of
+ *    the message, launched in order.  Needs 2 <= N <= 8 and 16-byte aligned
  *    buffers, with the same fallback as RING_CLUSTER; `workspace` is
  *    optional and unused (this form raises no device status).
  *  RING_LANE: the RING schedule, chunk order and rounding (bit-identical

@@ -7,7 +7,7 @@
 // in "From NCCL Ring LL to PCIe IPC AllReduce"), so the result is
 // bit-identical.  A CTA holds all N ranks, one warp each (lane t of warp r
 // plays rank r for one 16-byte vector of every chunk of a tile of 32 vectors
-// per chunk); the CTAs of the grid walk the tiles with a stride.
+// per chunk); each CTA of the grid takes one tile.
 //
 // Hops.  The ring of one tile is 2N-2 hops: N-1 reduce-scatter hops that
 // carry the fp32 / int32 partials (laid out piece-major, so that each
@@ -21,15 +21,13 @@
 // follows.  There is no spin-wait: a CTA-wide barrier cannot time out, and
 // the kernel waits on nothing outside its own CTA.
 //
-// Inputs come in one of two ways (template parameter D).  D = 0: they are
-// staged one tile ahead in shared memory: each thread copies the vector of
-// step k of the next tile into its own 16-byte cell with cp.async as soon as
-// step k of this tile has read the cell; a CTA's first tile has all N copies
-// in flight at once, which suits a CTA that holds one tile.  D > 0 (N a
-// multiple of D): each thread loads its inputs into D registers, step k + D
-// issued as soon as step k has used its own, across tile boundaries; this
-// keeps the cells' shared-memory traffic off the pipe that the hops load,
-// which suits a CTA that walks several tiles.
+// Inputs are staged in shared memory: each thread copies the vector of every
+// reduce-scatter step of its tile into its own 16-byte cell with cp.async,
+// all N copies in flight at once, and a CTA that walks a further tile
+// refills cell k with that tile's step k as soon as step k has read it.  The
+// grid has one CTA per tile, launched in order (a CTA walks further tiles
+// only beyond 2^30 of them): measured faster than a resident grid walking
+// the tiles, with the next tile's inputs in the cells or in registers.
 // Chunk boundaries are whole vectors, so every vector the hops carry lies
 // wholly inside its chunk or wholly outside it -- except the one that holds
 // the message's last count mod VN elements.  Those few elements (at most 7)
@@ -83,14 +81,12 @@ __device__ __forceinline__ void cp_async_wait_n() {
 }
 
 // NR: the rank count at compile time (its loops unrolled and its waits
-// immediate), or 0 for any count in 2..8.  D: the register prefetch distance
-// in steps, or 0 for the cp.async cells.  WIRE: the reduce-scatter hops carry
+// immediate), or 0 for any count in 2..8.  WIRE: the reduce-scatter hops carry
 // the partial rounded to the storage type (RING_WIRE) instead of fp32 /
 // int32 (RING): each receiver widens it, adds its own values and rounds
 // again before passing it on.
-template <int DT, int OP, int MINB, typename OFF, int NR, int D, bool WIRE>
+template <int DT, int OP, int MINB, typename OFF, int NR, bool WIRE>
 __global__ void __launch_bounds__(kRtMaxRanks * 32, MINB) k_ring_cta(const __grid_constant__ RingCtaArgs a) {
-  static_assert(D == 0 || (NR > 0 && NR % D == 0), "register slots repeat every tile");
   using A = typename Elem<DT>::A;
   constexpr int VN = Vec<DT>::kN;  // elements per 16-byte vector
   constexpr int NQ = WIRE ? 1 : VN / 4;  // 16-byte pieces a reduce-scatter hop carries per lane
@@ -169,28 +165,13 @@ __global__ void __launch_bounds__(kRtMaxRanks * 32, MINB) k_ring_cta(const __gri
     cp_async_commit();
   };
 
-  // D > 0: step k's input of the tile `delta` bytes ahead into register slot
-  // k mod D: whole (mode 1), or zero outside the chunk (mode 2).  A load that
-  // is L2-coherent (not the read-only path), since in place a later tile of
-  // this CTA writes what an earlier one read.
-  uint4 xin[D > 0 ? D : 1];
-  auto load = [&](int slot, OFF off, int mode, uint64_t delta, int c, uint64_t ee) {
-    if (mode == 1 || (mode == 2 && inside(c, ee))) xin[slot] = __ldcg(reinterpret_cast<const uint4*>(in_t + delta + off));
-    else xin[slot] = make_uint4(0, 0, 0, 0);
-  };
-
   // the first tile's inputs, in reduce-scatter step order
   {
     const int mode = blockIdx.x < a.full_tiles ? 1 : 2;
     const uint64_t e = blockIdx.x * TE + static_cast<uint64_t>(t) * VN;
-    if constexpr (D > 0) {
 #pragma unroll
-      for (int k = 0; k < D; ++k) load(k, offs[k], mode, 0, chunk[k], e);
-    } else {
-#pragma unroll
-      for (int k = 0; k < KMAX; ++k)
-        if (k < n) fill(k, chunk[k], offs[k], mode, 0, e);
-    }
+    for (int k = 0; k < KMAX; ++k)
+      if (k < n) fill(k, chunk[k], offs[k], mode, 0, e);
   }
 
   for (uint64_t tile = blockIdx.x; tile < a.tiles; tile += gridDim.x) {
@@ -218,28 +199,14 @@ __global__ void __launch_bounds__(kRtMaxRanks * 32, MINB) k_ring_cta(const __gri
       auto put = [&](int c, OFF off, const uint4& w) {  // this lane's rounded vector of chunk c (at off)
         if (full || inside(c, e)) st16(out_t + off, w);
       };
-      // D > 0: after step k, the load of step k + D (of this tile, or of the
-      // next once past the last step) into the slot step k has just used
-      auto issue = [&](int k) {
-        if constexpr (D > 0) {
-          const int s2 = k + D;
-          if (s2 < NR) load(k % D, offs[s2], full ? 1 : 2, 0, chunk[s2], e);
-          else if (next != 0) load(k % D, offs[s2 - NR], FAST ? 1 : next, step_b, chunk[s2 - NR], ne);
-        }
-      };
       // reduce-scatter: N-1 hops of partials; step k adds chunk r-1-k of this rank
       A p[VN];
       {
+        wait_cells();
         Vec<DT> w;
-        if constexpr (D > 0) {
-          widen16<DT>(xin[0], w);
-        } else {
-          wait_cells();
-          widen16<DT>(mine[0], w);
-        }
+        widen16<DT>(mine[0], w);
 #pragma unroll
         for (int i = 0; i < VN; ++i) p[i] = w.v[i];
-        issue(0);
       }
 #pragma unroll
       for (int k = 1; k < KMAX; ++k) {
@@ -269,17 +236,12 @@ __global__ void __launch_bounds__(kRtMaxRanks * 32, MINB) k_ring_cta(const __gri
           }
         }
         bo = bo == 0 ? other : 0;
+        refill(k - 1, chunk[k - 1], offs[k - 1]);  // cell k-1 was read before this barrier
+        wait_cells();
         Vec<DT> w;
-        if constexpr (D > 0) {
-          widen16<DT>(xin[k % D], w);
-        } else {
-          refill(k - 1, chunk[k - 1], offs[k - 1]);  // cell k-1 was read before this barrier
-          wait_cells();
-          widen16<DT>(mine[k * cells], w);
-        }
+        widen16<DT>(mine[k * cells], w);
 #pragma unroll
         for (int i = 0; i < VN; ++i) p[i] = op_step<OP>(p[i], w.v[i]);
-        issue(k);
       }
       // the one rounding, on rank r (chunk r is offs[n-1]); the rounded value travels on
       Vec<DT> v;
@@ -296,9 +258,7 @@ __global__ void __launch_bounds__(kRtMaxRanks * 32, MINB) k_ring_cta(const __gri
         __syncthreads();
         w = rx[bo];
         bo = bo == 0 ? other : 0;
-        if constexpr (D == 0) {
-          if (j == 1) refill(n - 1, chunk_last, off_last);  // the last cell, read before this barrier
-        }
+        if (j == 1) refill(n - 1, chunk_last, off_last);  // the last cell, read before this barrier
         put(chunk[j - 1], offs[j - 1], w);
       }
     };
@@ -317,7 +277,7 @@ static uint64_t ring_cta_tiles(uint64_t seg) {
   return std::max<uint64_t>(1, (seg + per_tile - 1) / per_tile);
 }
 
-template <int DT, int OP, int MINB, typename OFF, int NR, int D, bool WIRE>
+template <int DT, int OP, int MINB, typename OFF, int NR, bool WIRE>
 static int launch_ring_cta_t(RingCtaArgs a, cudaStream_t s) {
   constexpr int VN = Vec<DT>::kN;
   constexpr int NQ = WIRE ? 1 : VN / 4;
@@ -327,14 +287,13 @@ static int launch_ring_cta_t(RingCtaArgs a, cudaStream_t s) {
   // chunk when it is full in that one
   const uint64_t lead = static_cast<uint64_t>(a.n - 1) * a.seg;
   a.full_tiles = a.count > lead ? (a.count - lead) / per_tile : 0;
-  // hop slots, then (cells only) each thread's input cells
-  const size_t smem = (2ull * NQ + (D > 0 ? 0 : a.n)) * a.n * 32 * 16;
+  const size_t smem = (2ull * NQ + a.n) * a.n * 32 * 16;  // hop slots, then each thread's input cells
   static int smem_set[COLL_MAX_RANKS] = {0};  // per device ordinal: largest limit set so far
   const int st =
-      allow_dynamic_smem(reinterpret_cast<const void*>(k_ring_cta<DT, OP, MINB, OFF, NR, D, WIRE>), smem, smem_set);
+      allow_dynamic_smem(reinterpret_cast<const void*>(k_ring_cta<DT, OP, MINB, OFF, NR, WIRE>), smem, smem_set);
   if (st != COLL_OK) return st;
-  const uint64_t grid = std::min<uint64_t>(a.tiles, static_cast<uint64_t>(num_sms()) * MINB);
-  launch_pdl(k_ring_cta<DT, OP, MINB, OFF, NR, D, WIRE>, dim3(static_cast<unsigned>(grid)), dim3(32 * a.n), smem, s,
+  const uint64_t grid = std::min<uint64_t>(a.tiles, kMaxStreamGrid);  // one CTA per tile, launched in order
+  launch_pdl(k_ring_cta<DT, OP, MINB, OFF, NR, WIRE>, dim3(static_cast<unsigned>(grid)), dim3(32 * a.n), smem, s,
              a);
   return launch_status(cudaGetLastError());
 }
@@ -343,17 +302,10 @@ template <int DT, int OP, bool WIRE>
 static int launch_ring_cta_op(const RingCtaArgs& a, cudaStream_t s) {
   // byte offsets within one rank's buffer fit 32 bits below 4 GiB
   const uint64_t span = static_cast<uint64_t>(a.n) * a.seg * Elem<DT>::kSize;
-  if (span >= (1ull << 32)) return launch_ring_cta_t<DT, OP, 3, uint64_t, 0, 0, WIRE>(a, s);
-  // eight ranks (the workloads' count) get the fully unrolled kernel: with
-  // register prefetch when a CTA walks several tiles (measured on B200 at
-  // 3.5 MiB per rank: 12.97 against 13.64 us; 256 MiB: 717 against 764 us),
-  // with the cells when every CTA holds one tile (1 MiB: 5.21 against 5.47)
-  if (a.n == 8) {
-    const uint64_t slots = static_cast<uint64_t>(num_sms()) * 4;
-    if (ring_cta_tiles<DT>(a.seg) > slots) return launch_ring_cta_t<DT, OP, 4, uint32_t, 8, 4, WIRE>(a, s);
-    return launch_ring_cta_t<DT, OP, 4, uint32_t, 8, 0, WIRE>(a, s);
-  }
-  return launch_ring_cta_t<DT, OP, 4, uint32_t, 0, 0, WIRE>(a, s);
+  if (span >= (1ull << 32)) return launch_ring_cta_t<DT, OP, 3, uint64_t, 0, WIRE>(a, s);
+  // eight ranks (the workloads' count) get the fully unrolled kernel
+  if (a.n == 8) return launch_ring_cta_t<DT, OP, 4, uint32_t, 8, WIRE>(a, s);
+  return launch_ring_cta_t<DT, OP, 4, uint32_t, 0, WIRE>(a, s);
 }
 
 // Rounding a partial to the storage type changes nothing for fp32 / int32
