@@ -173,7 +173,7 @@ COLL_API int coll_reduce_scatter(const void* const* send, void* const* recv, int
  *    fp32 (int32 for int32); the result may differ from the rank-order
  *    reduction by rounding only.  When 2 <= N <= 8 and every buffer is
  *    16-byte aligned it runs in one launch, as the form measured fastest on
- *    B200: RING_LANE for N <= 3, for N == 4 up to 256 KiB and for N >= 5 up
+ *    B200: RING_LANE for N == 2, for N <= 4 up to 256 KiB and for N >= 5 up
  *    to 16 KiB per rank, RING_CTA above; otherwise as RING_STEPS.  Every
  *    form gives the same result bit for bit.
  *    coll_all_reduce_form() tells which.  `workspace`:

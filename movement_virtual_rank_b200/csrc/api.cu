@@ -374,14 +374,14 @@ int coll_reduce_scatter(const void* const* send, void* const* recv, int nranks, 
 // RING runs as the one-launch ring measured fastest on B200 for the rank
 // count and the bytes per rank (cold inputs, 1 KiB .. 256 MiB per rank at 2,
 // 3, 4 and 8 virtual ranks), when the buffers allow one: the ranks as lanes
-// of a warp (RING_LANE) at 2 and 3 ranks, at 4 ranks up to 256 KiB and at 5
+// of a warp (RING_LANE) at 2 ranks, at 3 and 4 ranks up to 256 KiB and at 5
 // and more up to 16 KiB; above those, where RING_LANE's per-rank 64-byte
 // accesses load the L1 data pipe, the ranks as warps of a CTA (RING_CTA).
 // The cluster form and the stream-ordered steps were slower at every size.
 // Every form gives the same bits.
 static coll_algo_t ring_form(int nranks, size_t bytes, bool vec) {
   if (!vec || !ring_cta_supported(nranks)) return COLL_ALGO_RING_STEPS;
-  if (nranks <= 3 || (nranks == 4 && bytes <= (256u << 10)) || bytes <= (16u << 10)) return COLL_ALGO_RING_LANE;
+  if (nranks == 2 || (nranks <= 4 && bytes <= (256u << 10)) || bytes <= (16u << 10)) return COLL_ALGO_RING_LANE;
   return COLL_ALGO_RING_CTA;
 }
 

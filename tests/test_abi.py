@@ -110,7 +110,7 @@ def test_workspace_sizes():
 # RING's one-launch form by rank count: the largest bytes per rank at which
 # the lane ring (RING_LANE) was measured fastest (None: every size); above
 # it the CTA ring (RING_CTA)
-RING_LANE_UP_TO = {2: None, 3: None, 4: 256 << 10, 5: 16 << 10, 6: 16 << 10, 7: 16 << 10, 8: 16 << 10}
+RING_LANE_UP_TO = {2: None, 3: 256 << 10, 4: 256 << 10, 5: 16 << 10, 6: 16 << 10, 7: 16 << 10, 8: 16 << 10}
 
 
 def test_ring_form_by_ranks_and_size():
