@@ -21,9 +21,8 @@
 
 namespace mvr {
 
-// The fan-out and the copy lists use bulk copies when every CTA gets at least
-// this many tiles to pipeline (below that a CTA waits for one load, then one
-// store round, and the element path is faster).
+// The fan-out and the copy lists use bulk copies from this many tiles per
+// resident CTA (6 per SM) up; below that the element path is faster.
 constexpr uint64_t kTmaMinTilesPerCta = 4;
 
 static int pick_unit(uint64_t bits) {
@@ -78,7 +77,11 @@ __global__ void __launch_bounds__(kThreads) k_fanout(const __grid_constant__ Fan
 // of shared-memory stages with cp.async.bulk and writes each landed tile to
 // every destination with bulk stores; a stage is refilled once its stores
 // have finished reading it.  Tiles of all sources are interleaved over the
-// grid so that every source progresses at once.
+// grid so that every source progresses at once.  The grid has one CTA per
+// kTmaStages tiles (CTA b takes tiles b, b + G, b + 2G, b + 3G), launched in
+// order, so each CTA fills its stages once and the next CTAs' loads overlap
+// its stores: measured faster than a resident grid walking every tile (all
+// 8 sources of 16 MiB to 8 ranks: 194.5 against 217 us).
 constexpr int kTmaTile = 8192;
 constexpr int kTmaStages = 4;
 
@@ -139,9 +142,9 @@ int launch_fanout(const FanoutArgs& a, cudaStream_t s) {
   for (int r = 0; r < a.ns; ++r) bits |= reinterpret_cast<uintptr_t>(a.src[r]);
   for (int q = 0; q < a.nd; ++q) bits |= reinterpret_cast<uintptr_t>(a.dst[q]);
   const uint64_t tiles = (a.bytes + kTmaTile - 1) / kTmaTile * a.ns;
-  const uint64_t tma_grid = static_cast<uint64_t>(num_sms()) * 6;  // 6 x 32 KB of stages per SM
-  if ((bits & 15) == 0 && (a.bytes & 15) == 0 && tiles >= kTmaMinTilesPerCta * tma_grid) {
-    const uint64_t grid = tma_grid;
+  const uint64_t resident = static_cast<uint64_t>(num_sms()) * 6;  // 6 x 32 KB of stages per SM
+  if ((bits & 15) == 0 && (a.bytes & 15) == 0 && tiles >= kTmaMinTilesPerCta * resident) {
+    const uint64_t grid = stream_grid(tiles, kTmaStages);  // one CTA per kTmaStages tiles
     launch_pdl(k_fanout_tma, dim3(static_cast<unsigned>(grid)), dim3(32), kTmaStages * kTmaTile, s, a);
     return launch_status(cudaGetLastError());
   }
@@ -295,8 +298,8 @@ int launch_copy_jobs(const CopyJob* jobs, int njobs, cudaStream_t s) {
   if (U == 16) {
     uint64_t tiles = 0;
     for (const CopyJob& j : v) tiles += (j.bytes + kTmaTile - 1) / kTmaTile;
-    const uint64_t tma_grid = static_cast<uint64_t>(num_sms()) * 6;
-    if (tiles >= kTmaMinTilesPerCta * tma_grid) {
+    const uint64_t resident = static_cast<uint64_t>(num_sms()) * 6;
+    if (tiles >= kTmaMinTilesPerCta * resident) {
       static thread_local TmaJobsArgs targs;  // ~29 KB: keep it off the stack
       for (size_t first = 0; first < v.size(); first += kMaxTmaJobs) {
         const int nj = static_cast<int>(std::min<size_t>(kMaxTmaJobs, v.size() - first));
@@ -310,7 +313,7 @@ int launch_copy_jobs(const CopyJob* jobs, int njobs, cudaStream_t s) {
         targs.total_tiles = acc;
         targs.njobs = nj;
         targs.status = nullptr;
-        const uint64_t grid = std::min<uint64_t>(acc, tma_grid);
+        const uint64_t grid = stream_grid(acc, kTmaStages);  // one CTA per kTmaStages tiles, in order
         launch_pdl(k_copy_jobs_tma, dim3(static_cast<unsigned>(grid)), dim3(32), kTmaStages * kTmaTile, s, targs);
         const int st = launch_status(cudaGetLastError());
         if (st != COLL_OK) return st;

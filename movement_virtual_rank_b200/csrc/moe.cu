@@ -377,13 +377,16 @@ int launch_moe_dispatch(const MoeMoveArgs& a, cudaStream_t s) {
   // whole rows through shared memory once there are enough of them
   const uint32_t stage_bytes = static_cast<uint32_t>((a.row_bytes + 127) / 128 * 128);
   const int64_t per_sm = std::max<int64_t>(1, (200 * 1024) / (kDispStages * static_cast<int64_t>(stage_bytes)));
-  const int64_t tma_grid = static_cast<int64_t>(num_sms()) * per_sm;
-  if ((bits & 15) == 0 && a.row_bytes <= kDispMaxRow && rows >= 4 * tma_grid) {
+  const int64_t resident = static_cast<int64_t>(num_sms()) * per_sm;
+  if ((bits & 15) == 0 && a.row_bytes <= kDispMaxRow && rows >= 4 * resident) {
     const size_t smem = static_cast<size_t>(kDispStages) * stage_bytes;
     static int smem_set[COLL_MAX_RANKS] = {0};  // per device ordinal: largest limit set so far
     const int ok = allow_dynamic_smem(reinterpret_cast<const void*>(k_moe_dispatch_tma), smem, smem_set);
     if (ok != COLL_OK) return ok;
-    launch_pdl(k_moe_dispatch_tma, dim3(static_cast<unsigned>(std::min<int64_t>(rows, tma_grid))), dim3(32), smem, s, a,
+    // one CTA per kDispStages rows, launched in order: measured faster than a
+    // resident grid walking the rows (8 x 4096 rows of 14 KB: 662 against 751 us)
+    const uint64_t grid = stream_grid(static_cast<uint64_t>(rows), kDispStages);
+    launch_pdl(k_moe_dispatch_tma, dim3(static_cast<unsigned>(grid)), dim3(32), smem, s, a,
                stage_bytes);
     return launch_status(cudaGetLastError());
   }
