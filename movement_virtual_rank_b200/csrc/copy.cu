@@ -78,12 +78,14 @@ __global__ void __launch_bounds__(kThreads) k_fanout(const __grid_constant__ Fan
 // every destination with bulk stores; a stage is refilled once its stores
 // have finished reading it.  Tiles of all sources are interleaved over the
 // grid so that every source progresses at once.  The grid has one CTA per
-// kTmaStages tiles (CTA b takes tiles b, b + G, b + 2G, b + 3G), launched in
-// order, so each CTA fills its stages once and the next CTAs' loads overlap
-// its stores: measured faster than a resident grid walking every tile (all
-// 8 sources of 16 MiB to 8 ranks: 194.5 against 217 us).
+// kTmaTilesPerCta tiles (CTA b takes tiles b and b + G), launched in order,
+// so a CTA's loads are all in flight at once and the next CTAs' loads
+// overlap its stores: measured faster than a resident grid walking every
+// tile (all 8 sources of 16 MiB to 8 ranks: 191 against 217 us; 4 tiles per
+// CTA 193).
 constexpr int kTmaTile = 8192;
 constexpr int kTmaStages = 4;
+constexpr uint64_t kTmaTilesPerCta = 2;
 
 __global__ void __launch_bounds__(32) k_fanout_tma(const __grid_constant__ FanoutArgs a) {
   extern __shared__ __align__(128) unsigned char stage_buf[];
@@ -144,7 +146,7 @@ int launch_fanout(const FanoutArgs& a, cudaStream_t s) {
   const uint64_t tiles = (a.bytes + kTmaTile - 1) / kTmaTile * a.ns;
   const uint64_t resident = static_cast<uint64_t>(num_sms()) * 6;  // 6 x 32 KB of stages per SM
   if ((bits & 15) == 0 && (a.bytes & 15) == 0 && tiles >= kTmaMinTilesPerCta * resident) {
-    const uint64_t grid = stream_grid(tiles, kTmaStages);  // one CTA per kTmaStages tiles
+    const uint64_t grid = stream_grid(tiles, kTmaTilesPerCta);
     launch_pdl(k_fanout_tma, dim3(static_cast<unsigned>(grid)), dim3(32), kTmaStages * kTmaTile, s, a);
     return launch_status(cudaGetLastError());
   }
@@ -313,7 +315,7 @@ int launch_copy_jobs(const CopyJob* jobs, int njobs, cudaStream_t s) {
         targs.total_tiles = acc;
         targs.njobs = nj;
         targs.status = nullptr;
-        const uint64_t grid = stream_grid(acc, kTmaStages);  // one CTA per kTmaStages tiles, in order
+        const uint64_t grid = stream_grid(acc, kTmaTilesPerCta);  // in order, as the fan-out
         launch_pdl(k_copy_jobs_tma, dim3(static_cast<unsigned>(grid)), dim3(32), kTmaStages * kTmaTile, s, targs);
         const int st = launch_status(cudaGetLastError());
         if (st != COLL_OK) return st;
@@ -379,10 +381,10 @@ int launch_gather_rows(const GatherRowsArgs& a, cudaStream_t s) {
                               : U == 4  ? k_gather_rows<4>
                               : U == 2  ? k_gather_rows<2>
                                         : k_gather_rows<1>;
-  // about 4 units per thread per row chunk; 8 CTAs per SM in total (more
-  // than fit at once for the 16-byte kernel: with rows split into fixed
-  // parts that measured faster, 45.1 against 48.0 us, than a resident-only grid)
-  const uint64_t parts = std::min<uint64_t>(a.rows, std::max<uint64_t>(1, static_cast<uint64_t>(num_sms()) * 8 / a.n));
+  // one CTA per row of every rank, launched in order: measured faster than 8
+  // CTAs per SM walking the rows (44.0 against 45.0 us for 8 ranks x 256
+  // rows of 64 KB) and than a resident-only grid (48.0 us)
+  const uint64_t parts = std::min<uint64_t>(a.rows, kMaxStreamGrid / a.n);
   launch_pdl(fn, dim3(static_cast<unsigned>(parts * a.n)), dim3(kThreads), 0, s, a);
   return launch_status(cudaGetLastError());
 }
