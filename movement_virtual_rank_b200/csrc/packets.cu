@@ -365,13 +365,15 @@ int launch_ll_pack(const CodecArgs& a0, int proto, cudaStream_t s) {
   if (proto == COLL_PROTO_LL && ((msg | pkt) & 15) == 0) {
     // whole tiles through the bulk-copy path from 4 tiles per resident CTA up
     // (4 x 48 KB of stages per SM, shared by the ranks' CTA rows), the rest
-    // below; one CTA per kPackStages tiles of a rank, launched in order:
-    // measured faster than a resident grid walking the tiles (8 x 256 MiB:
-    // 985 against 1081 us)
+    // below.  From 8 tiles per resident CTA up, one CTA per kPackStages tiles
+    // of a rank, launched in order: measured faster than a resident grid
+    // walking the tiles (8 x 256 MiB: 977 against 1081 us).  Below that the
+    // in-order grid would end on a partial second wave, and the resident grid
+    // is faster (one rank of 16 MiB: 9.35 against 10.24 us).
     const uint64_t resident = std::max<uint64_t>(1, static_cast<uint64_t>(num_sms()) * 4 / a.n);
     const uint64_t tiles = a.bytes / kPackMsg;  // per rank
     if (tiles >= 4 * resident) {
-      const unsigned gx = static_cast<unsigned>(stream_grid(tiles, kPackStages));
+      const unsigned gx = static_cast<unsigned>(tiles < 8 * resident ? resident : stream_grid(tiles, kPackStages));
       const size_t smem = static_cast<size_t>(kPackStages) * (kPackMsg + kPackPkt);
       static int smem_set[COLL_MAX_RANKS] = {0};  // per device ordinal: largest limit set so far
       const int ok = allow_dynamic_smem(reinterpret_cast<const void*>(k_ll_pack_tma), smem, smem_set);
