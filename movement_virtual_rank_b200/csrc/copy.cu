@@ -376,7 +376,18 @@ __global__ void __launch_bounds__(kThreads) k_gather_rows(const __grid_constant_
   for (uint64_t row = part; row < a.rows; row += parts) {
     const char* sp = src + row * a.row_bytes;
     char* dp = dst + row * a.dst_pitch;
-    for (uint64_t u = threadIdx.x; u < ru; u += blockDim.x) stu<U>(dp + u * U, ldu<U>(sp + u * U));
+    // four units in flight per thread, then their stores (44.0 -> 43.0 us for
+    // 8 ranks x 256 rows of 64 KB against one load-store pair at a time)
+    constexpr int kB = 4;
+    uint64_t u = threadIdx.x;
+    for (; u + (kB - 1) * blockDim.x < ru; u += kB * blockDim.x) {
+      typename UnitT<U>::T x[kB];
+#pragma unroll
+      for (int k = 0; k < kB; ++k) x[k] = ldu<U>(sp + (u + k * blockDim.x) * U);
+#pragma unroll
+      for (int k = 0; k < kB; ++k) stu<U>(dp + (u + k * blockDim.x) * U, x[k]);
+    }
+    for (; u < ru; u += blockDim.x) stu<U>(dp + u * U, ldu<U>(sp + u * U));
   }
 }
 
