@@ -263,14 +263,16 @@ __global__ void __launch_bounds__(kThreads) k_ll128_unpack(const __grid_constant
 // element kernels, so they stay there).  One warp per CTA bulk-loads 4096
 // message bytes into a shared-memory stage, the 32 lanes interleave them
 // with the flag into the stage's 8192-byte output buffer, and one lane
-// bulk-stores it; 4 stages overlap loads, rewrites and stores of consecutive
-// tiles.  The partial tile at the end goes to k_ll_pack.
-constexpr int kPackStages = 4;
+// bulk-stores it; STAGES stages overlap loads, rewrites and stores of the
+// tiles a CTA takes.  The partial tile at the end goes to k_ll_pack.
+constexpr int kPackStages = 4;     // a resident CTA walking many tiles
+constexpr int kPackStagesIo = 2;   // a CTA of the in-order grid, one tile per stage
 constexpr uint32_t kPackMsg = 4096, kPackPkt = 8192;
 
+template <int STAGES>
 __global__ void __launch_bounds__(32) k_ll_pack_tma(const __grid_constant__ CodecArgs a, uint64_t tiles) {
   extern __shared__ __align__(128) unsigned char smem[];  // [stage]{in[kPackMsg], out[kPackPkt]}
-  __shared__ __align__(8) uint64_t bar[kPackStages];
+  __shared__ __align__(8) uint64_t bar[STAGES];
   constexpr uint32_t kStage = kPackMsg + kPackPkt;
   pdl_wait();
   pdl_trigger();
@@ -280,7 +282,7 @@ __global__ void __launch_bounds__(32) k_ll_pack_tma(const __grid_constant__ Code
   const uint64_t total = tiles;
   const int lane = threadIdx.x;
   if (lane == 0) {
-    for (int st = 0; st < kPackStages; ++st) mbar_init(&bar[st], 1);
+    for (int st = 0; st < STAGES; ++st) mbar_init(&bar[st], 1);
     fence_barrier_init();
   }
   __syncwarp();
@@ -290,23 +292,23 @@ __global__ void __launch_bounds__(32) k_ll_pack_tma(const __grid_constant__ Code
     bulk_load(smem + st * kStage, src + t * kPackMsg, kPackMsg, &bar[st]);
   };
   int inflight = 0;
-  for (int st = 0; st < kPackStages && blockIdx.x + st * stride < total; ++st, ++inflight)
+  for (int st = 0; st < STAGES && blockIdx.x + st * stride < total; ++st, ++inflight)
     if (lane == 0) issue(blockIdx.x + st * stride, st);
   int i = 0;
   for (uint64_t t = blockIdx.x; t < total; t += stride, ++i) {
-    const int st = i % kPackStages;
-    const uint32_t par = (i / kPackStages) & 1;
+    const int st = i % STAGES;
+    const uint32_t par = (i / STAGES) & 1;
     int ok = 1;
     if (lane == 0) {
       ok = mbar_wait_bounded(&bar[st], par) ? 1 : 0;
-      bulk_wait_read<kPackStages - 1>();  // this stage's previous store has read its output buffer
+      bulk_wait_read<STAGES - 1>();  // this stage's previous store has read its output buffer
     }
     ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
     if (!ok) {
       if (lane == 0) {
         bulk_wait_all();
         for (int k = 1; k < inflight; ++k)
-          mbar_wait_bounded(&bar[(i + k) % kPackStages], ((i + k) / kPackStages) & 1);
+          mbar_wait_bounded(&bar[(i + k) % STAGES], ((i + k) / STAGES) & 1);
       }
       return;
     }
@@ -324,7 +326,7 @@ __global__ void __launch_bounds__(32) k_ll_pack_tma(const __grid_constant__ Code
     if (lane == 0) {
       bulk_store(packed + t * kPackPkt, out, kPackPkt);
       bulk_commit();
-      const uint64_t nxt = t + kPackStages * stride;
+      const uint64_t nxt = t + STAGES * stride;
       if (nxt < total) {
         issue(nxt, st);
         ++inflight;
@@ -333,6 +335,16 @@ __global__ void __launch_bounds__(32) k_ll_pack_tma(const __grid_constant__ Code
     inflight = __shfl_sync(0xFFFFFFFFu, inflight, 0);
   }
   if (lane == 0) bulk_wait_all();
+}
+
+template <int STAGES>
+static int launch_pack_tma(const CodecArgs& a, unsigned gx, uint64_t tiles, cudaStream_t s) {
+  const size_t smem = static_cast<size_t>(STAGES) * (kPackMsg + kPackPkt);
+  static int smem_set[COLL_MAX_RANKS] = {0};  // per device ordinal: largest limit set so far
+  const int ok = allow_dynamic_smem(reinterpret_cast<const void*>(k_ll_pack_tma<STAGES>), smem, smem_set);
+  if (ok != COLL_OK) return ok;
+  launch_pdl(k_ll_pack_tma<STAGES>, dim3(gx, a.n), dim3(32), smem, s, a, tiles);
+  return launch_status(cudaGetLastError());
 }
 
 // The codec grid for n ranks of `units` work items each: one CTA row per
@@ -365,21 +377,19 @@ int launch_ll_pack(const CodecArgs& a0, int proto, cudaStream_t s) {
   if (proto == COLL_PROTO_LL && ((msg | pkt) & 15) == 0) {
     // whole tiles through the bulk-copy path from 4 tiles per resident CTA up
     // (4 x 48 KB of stages per SM, shared by the ranks' CTA rows), the rest
-    // below.  From 8 tiles per resident CTA up, one CTA per kPackStages tiles
-    // of a rank, launched in order: measured faster than a resident grid
-    // walking the tiles (8 x 256 MiB: 977 against 1081 us).  Below that the
-    // in-order grid would end on a partial second wave, and the resident grid
-    // is faster (one rank of 16 MiB: 9.35 against 10.24 us).
+    // below.  From 8 tiles per resident CTA up, one CTA per 2 tiles of a
+    // rank with 2 stages (24 KB, so 9 CTAs fit on an SM), launched in order:
+    // measured faster than a resident grid walking the tiles (8 x 256 MiB:
+    // 935 against 1081 us; 4 tiles and 4 stages per CTA 977 us).  Below that
+    // the in-order grid would end on a partial second wave, and the resident
+    // grid with 4 stages is faster (one rank of 16 MiB: 9.35 against 10.24 us).
     const uint64_t resident = std::max<uint64_t>(1, static_cast<uint64_t>(num_sms()) * 4 / a.n);
     const uint64_t tiles = a.bytes / kPackMsg;  // per rank
     if (tiles >= 4 * resident) {
-      const unsigned gx = static_cast<unsigned>(tiles < 8 * resident ? resident : stream_grid(tiles, kPackStages));
-      const size_t smem = static_cast<size_t>(kPackStages) * (kPackMsg + kPackPkt);
-      static int smem_set[COLL_MAX_RANKS] = {0};  // per device ordinal: largest limit set so far
-      const int ok = allow_dynamic_smem(reinterpret_cast<const void*>(k_ll_pack_tma), smem, smem_set);
-      if (ok != COLL_OK) return ok;
-      launch_pdl(k_ll_pack_tma, dim3(gx, a.n), dim3(32), smem, s, a, tiles);
-      const int st = launch_status(cudaGetLastError());
+      const int st = tiles < 8 * resident
+                         ? launch_pack_tma<kPackStages>(a, static_cast<unsigned>(resident), tiles, s)
+                         : launch_pack_tma<kPackStagesIo>(a, static_cast<unsigned>(stream_grid(tiles, kPackStagesIo)),
+                                                          tiles, s);
       if (st != COLL_OK) return st;
       for (int r = 0; r < a.n; ++r) {
         a.in[r] += tiles * kPackMsg;

@@ -194,11 +194,14 @@ def test_ll_sweep_sizes(log2):
 
 
 @pytest.mark.parametrize("proto", [M.LL, M.LL128])
-@pytest.mark.parametrize("nbytes", [16 << 20, (16 << 20) + 4, (16 << 20) + 120 * 7 + 3, 10_000_000, 3 * (1 << 22) + 1000])
+@pytest.mark.parametrize("nbytes", [16 << 20, (16 << 20) + 4, (16 << 20) + 120 * 7 + 3, 10_000_000, 3 * (1 << 22) + 1000,
+                                    (20 << 20) + 4])
 def test_pack_unpack_bulk_path(proto, nbytes):
     """Long aligned messages take the bulk-copy codec for whole tiles and the
     element kernels for the tail: the packet bytes are the oracle's, the
-    round trip is exact, and bytes past either buffer stay untouched."""
+    round trip is exact, and bytes past either buffer stay untouched.  One
+    rank's LL pack takes the resident grid up to 8 tiles per resident CTA
+    (the sizes up to 16 MiB + 843 B) and the in-order grid above (20 MiB)."""
     need_gpu()
     msg = u8(nbytes, nbytes % 1000 + 5)
     step = 0x0BAD_CAFE if proto == M.LL else (0x5A5A << 36) + 3
@@ -245,7 +248,7 @@ def test_unpack_counts_bad_flags_bulk_path(proto):
 
 @pytest.mark.parametrize("proto", [M.LL, M.LL128])
 @pytest.mark.parametrize("n,nbytes", [(1, 1000), (3, 1), (3, 121), (8, 4097), (8, 65536 + 12), (5, (1 << 20) + 7),
-                                      (8, 16 << 20), (8, (16 << 20) + 120 * 3 + 5), (2, 10_000_000),
+                                      (8, (2 << 20) + 12), (8, 16 << 20), (8, (16 << 20) + 120 * 3 + 5), (2, 10_000_000),
                                       (2, (64 << 20) + 4097)])
 @pytest.mark.parametrize("unaligned_rank", [None, 1])
 def test_pack_unpack_ranks(proto, n, nbytes, unaligned_rank):
