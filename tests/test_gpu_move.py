@@ -62,9 +62,11 @@ def test_broadcast_unaligned_guards():
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
-@pytest.mark.parametrize("rows,cols", [(1, 1), (1, 1000), (3, 5), (17, 33), (64, 1000)])
+@pytest.mark.parametrize("rows,cols", [(1, 1), (1, 1000), (3, 5), (17, 33), (64, 1000), (3, 4097)])
 @pytest.mark.parametrize("n", [1, 3, 8])
 def test_gather(dtype, rows, cols, n):
+    """Flat and last-dimension gathers against the oracle; [3, 4097] rows
+    move in 2- or 4-byte units, more than four per thread of a CTA."""
     need_gpu()
     xs = rand(n, rows * cols, dtype, salt=rows * 7 + cols)
     send = [to_dev(x, dtype).reshape(rows, cols) if rows > 1 else to_dev(x, dtype) for x in xs]
@@ -134,6 +136,35 @@ def test_all_gather(dtype, n, count):
     want = oracle.all_gather(xs)
     for q in range(n):
         assert np.array_equal(from_dev(recv[q], dtype), want[q])
+
+
+@pytest.mark.parametrize("op", ["all_gather", "broadcast"])
+def test_bulk_fanout_partial_tile(op):
+    """Fan-outs long enough for the bulk-copy kernel (one CTA per 2 tiles of
+    8 KB) whose messages end 48 bytes into a tile: 8 sources of 4 MiB + 48 B
+    (all_gather), or one source of 29 MiB + 48 B to 8 ranks (broadcast).
+    Every output against the oracle, and guard bands past each buffer."""
+    need_gpu()
+    n = 8
+    if op == "all_gather":
+        count = (2 << 20) + 24
+        xs = rand(n, count, "bf16", salt=41)
+        send = [to_dev(x, "bf16") for x in xs]
+        grecv = [Guarded(n * count, "bf16") for _ in range(n)]
+        M.coll_all_gather(send, [b.t for b in grecv])
+        torch.cuda.synchronize()
+        want = oracle.all_gather(xs)
+        for q in range(n):
+            assert np.array_equal(grecv[q].host(), want[q]) and grecv[q].guards_intact(), q
+    else:
+        count = (29 << 19) + 24
+        xs = rand(n, count, "bf16", salt=43)
+        bufs = [Guarded(count, "bf16", fill=x) for x in xs]
+        M.coll_broadcast([b.t for b in bufs], 5)
+        torch.cuda.synchronize()
+        want = oracle.broadcast(xs, 5)
+        for q in range(n):
+            assert np.array_equal(bufs[q].host(), want[q]) and bufs[q].guards_intact(), q
 
 
 def test_all_gather_in_place_and_unaligned():
